@@ -1,0 +1,176 @@
+/*
+ * skv.h — C ABI of libskv.so: split-KV block-sparse cross-attention on B200.
+ *
+ * The operation (sources: the web pages "Split-KV: Efficient Context
+ * Parallelism for Training Diffusion Drafters", arXiv 2611.05926, Abstract;
+ * and "Split-KV: Breaking the Context Parallelism Bottleneck in Diffusion
+ * Drafter Training", sections "Split-KV's Core Mechanism" and "LPT
+ * Scheduling"): short draft-query blocks, one block of `block_q` tokens per
+ * sampled anchor, cross-attend to a much longer context under a block-sparse
+ * mask. The context K/V is split into chunks; every chunk yields a partial
+ * output and log-sum-exp for the whole query set, and the partials are merged
+ * exactly with a query-sized combine. Chunks are placed on P partitions by a
+ * longest-processing-time-first planner weighted by realized attention cost.
+ *
+ * Readings fixed by this library where the pages give no formula:
+ *   - the block of anchor a (1 <= a <= L_b) attends to keys [0, a) of its own
+ *     sample's context; scale 1/sqrt(head_dim); LSE is the natural log;
+ *   - q-head h uses kv-head h / (Hq / Hkv);
+ *   - item = (sample b, chunk c, kv-head g, key sub-chunk s); its cost is the
+ *     number of unmasked (query token, key) pairs times the q-heads per
+ *     kv-head; LPT sorts by (cost desc, b, c, g, s) and gives each item to the
+ *     partition with the smallest (load, index);
+ *   - the static split gives partition p the packed context tokens
+ *     [floor(p T / P), floor((p + 1) T / P)).
+ *
+ * Data layout (all device tensors contiguous, caller-owned):
+ *   q, o, dout, dq : bf16 [Nq][Hq][d], Nq = anchor_offsets[B] * block_q; the
+ *                    block of anchor j is tokens [j * block_q, (j+1) * block_q)
+ *   k, v, dk, dv   : bf16 [Ltot][Hkv][d], Ltot = ctx_offsets[B]
+ *   lse            : fp32 [Nq][Hq]
+ *
+ * Errors: every call returns an skv_status code; nothing throws across the
+ * ABI. Calls that take a stream only enqueue work; errors found on the device
+ * (a wait that gave up, a malformed plan) land in a status word inside the
+ * workspace, read back by skv_status(). Arguments are checked before any
+ * launch: bad values return SKV_EINVAL, unsupported shapes SKV_EUNSUPPORTED.
+ *
+ * Memory: the library allocates no device memory. The caller provides the
+ * workspace `ws` (device, 256-byte aligned) sized by skv_plan_size().
+ */
+#ifndef SKV_H_
+#define SKV_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* skv_stream_t; /* a cudaStream_t; NULL = legacy default stream */
+
+enum skv_status_code {
+  SKV_OK = 0,
+  SKV_EINVAL = 1,       /* an argument is out of range or inconsistent */
+  SKV_EWORKSPACE = 2,   /* buffer smaller than the size skv_plan_size() gave */
+  SKV_EUNSUPPORTED = 3, /* valid problem this build does not run (head_dim, group size, sizes) */
+  SKV_ECUDA = 4,        /* a CUDA runtime call failed (see skv_last_cuda_error) */
+  SKV_EPLAN = 5,        /* plan buffer not written by skv_plan, or for another problem */
+  SKV_ETIMEOUT = 6,     /* a device-side wait gave up; results are invalid */
+  SKV_EDEVICE = 7       /* a kernel found an inconsistent work list; results are invalid */
+};
+
+enum skv_plan_policy {
+  SKV_PLAN_LPT = 0,    /* cost-aware LPT over (b, c, g, s) items ("LPT Scheduling") */
+  SKV_PLAN_STATIC = 1  /* equal-token contiguous split, the baseline LPT replaces */
+};
+
+/* One split-KV problem. Host pointers; read during the call only. */
+typedef struct {
+  int32_t num_samples;           /* B >= 1 */
+  const int64_t* ctx_offsets;    /* [B+1], ctx_offsets[0] = 0, L_b = ctx_offsets[b+1] - ctx_offsets[b] >= 1 */
+  const int32_t* anchor_offsets; /* [B+1], anchor_offsets[0] = 0, non-decreasing */
+  const int64_t* anchors;        /* [anchor_offsets[B]], 1 <= a <= L_b; any order, duplicates allowed */
+  int32_t block_q;               /* draft tokens per anchor, >= 1 */
+  int32_t chunk_kv;              /* KV chunk length C >= 1 */
+  int32_t sub_chunks;            /* LPT items split each chunk into this many key ranges; C % sub_chunks == 0 */
+  int32_t num_partitions;        /* P >= 1 virtual partitions (the pages' CP ranks) */
+  int32_t num_q_heads;           /* Hq */
+  int32_t num_kv_heads;          /* Hkv; Hq % Hkv == 0 and 128 % (Hq / Hkv) == 0 */
+  int32_t head_dim;              /* d in {64, 128} */
+} skv_problem;
+
+/* One planned work item (a view into the plan buffer). */
+typedef struct {
+  int32_t b, c, g, sub;        /* sample, chunk, kv-head, sub-chunk (static: piece index in the chunk) */
+  int64_t key_begin, key_end;  /* absolute key range in the packed context, [begin, end) */
+  int64_t cost;                /* unmasked (query, key) pairs x q-heads of the group */
+  int32_t partition;           /* partition the planner placed the item on */
+  int32_t order;               /* position in the placement order (LPT: longest first) */
+} skv_item;
+
+/*
+ * skv_plan_size — sizes for one problem under one policy.
+ * Outputs (any may be NULL): number of items, bytes of the host plan buffer,
+ * device workspace bytes for skv_attn_fwd + skv_lse_merge, and for
+ * skv_attn_bwd. One workspace of max(ws_fwd, ws_bwd) bytes serves a
+ * forward, merge and backward issued in that order on one stream.
+ * Returns SKV_EINVAL / SKV_EUNSUPPORTED for a problem skv_plan would reject.
+ */
+int skv_plan_size(const skv_problem* prob, int policy, size_t* n_items, size_t* plan_bytes,
+                  size_t* ws_fwd_bytes, size_t* ws_bwd_bytes);
+
+/*
+ * skv_plan — realized cost of every item (pages: "LPT Scheduling", cost each
+ * KV block actually incurs), placement by `policy`, and the work lists the
+ * kernels read. Host only, deterministic: the same problem gives the same
+ * bytes. `plan` is a caller-owned host buffer of plan_bytes (from
+ * skv_plan_size); `partition_load` (may be NULL) receives [P] int64 loads.
+ */
+int skv_plan(const skv_problem* prob, int policy, void* plan, size_t plan_bytes, int64_t* partition_load);
+
+/* Items of a plan in (b, c, g, sub) order; *items points into `plan`. */
+int skv_plan_items(const void* plan, const skv_item** items, size_t* n_items);
+
+/* Scalars of a plan: total cost (sum over items), number of forward work
+ * units (item x 128-row query tile pairs with unmasked keys), number of
+ * backward work units (item x 128-key tiles with unmasked queries),
+ * imbalance max/mean - 1 of the partition loads. Any pointer may be NULL. */
+int skv_plan_stats(const void* plan, int64_t* total_cost, int64_t* n_fwd_units, int64_t* n_bwd_units,
+                   double* imbalance);
+
+/*
+ * skv_attn_fwd — split-KV forward ("Split-KV's Core Mechanism": every KV
+ * chunk's local attention for the global query set). For every forward work
+ * unit, writes the chunk's normalized partial output (fp32) and LSE into the
+ * workspace. Copies the device part of `plan` into `ws` first (the caller may
+ * reuse `plan` once the call returns). q, k, v: device bf16 in the layouts
+ * above. Enqueued on `stream`.
+ */
+int skv_attn_fwd(const void* plan, const void* q, const void* k, const void* v, void* ws, size_t ws_bytes,
+                 skv_stream_t stream);
+
+/*
+ * skv_lse_merge — exact query-sized combine of the partials left in `ws` by
+ * skv_attn_fwd (same plan, same stream order): per (token, q-head)
+ *   m = max_c LSE_c, LSE = m + ln sum_c exp(LSE_c - m),
+ *   O = sum_c exp(LSE_c - LSE) O_c, chunks taken in ascending key order.
+ * Writes o (device bf16 [Nq][Hq][d]) and lse (device fp32 [Nq][Hq]).
+ */
+int skv_lse_merge(const void* plan, const void* ws, void* o, float* lse, skv_stream_t stream);
+
+/*
+ * skv_attn_bwd — gradients of the attention through the split: per KV item,
+ * probabilities recomputed with the merged LSE; dK/dV of every key written
+ * by the one item that owns it (zero for keys no query attends to); dQ summed
+ * over items in fp32 inside the workspace, then rounded to bf16.
+ * Inputs: q, k, v, o (bf16), lse (fp32, from skv_lse_merge), dout (bf16).
+ * Outputs: dq, dk, dv (bf16, fully overwritten). Enqueued on `stream`.
+ */
+int skv_attn_bwd(const void* plan, const void* q, const void* k, const void* v, const void* o, const float* lse,
+                 const void* dout, void* dq, void* dk, void* dv, void* ws, size_t ws_bytes, skv_stream_t stream);
+
+/*
+ * skv_status — synchronizes `stream`, reads the status word in `ws` and
+ * returns it (SKV_OK when no kernel reported an error since the last
+ * skv_attn_fwd/skv_attn_bwd reset it). SKV_ECUDA if the synchronize failed.
+ */
+int skv_status(const void* ws, skv_stream_t stream);
+
+/* Static text for a status code. */
+const char* skv_strerror(int code);
+
+/* Last CUDA runtime error code seen by this thread's calls (0 if none). */
+int skv_last_cuda_error(void);
+
+/* Realized per-partition busy time: if enabled (non-zero), the next kernels
+ * record, per work unit, its start/end %globaltimer stamps into `stamps`
+ * (device int64 [2 * n_units], caller-owned; NULL disables). */
+int skv_set_unit_timer(void* fwd_stamps, void* bwd_stamps);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SKV_H_ */

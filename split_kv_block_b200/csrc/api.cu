@@ -1,0 +1,309 @@
+// C ABI entry points: argument checks, workspace layout, plan upload,
+// tensor maps and kernel launches. See include/skv.h for the contract.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstring>
+#include <mutex>
+
+#include "kernels.h"
+#include "plan_layout.h"
+
+namespace skv {
+namespace {
+
+thread_local int g_last_cuda = 0;
+long long* g_fwd_stamps = nullptr;
+long long* g_bwd_stamps = nullptr;
+constexpr unsigned long long kTimeoutNs = 2000000000ull;  // 2 s per device-side wait
+
+int cuda_fail(cudaError_t e) {
+  g_last_cuda = static_cast<int>(e);
+  return SKV_ECUDA;
+}
+
+const PlanHeader* header_of(const void* plan) {
+  if (!plan) return nullptr;
+  const PlanHeader* h = static_cast<const PlanHeader*>(plan);
+  if (h->magic != kPlanMagic || h->version != kPlanVersion) return nullptr;
+  return h;
+}
+
+// ------------------------------------------------------------ plan upload
+// The plan's device section is copied into the workspace from a pinned
+// staging slot owned by the library; each slot is reused only after the copy
+// that read it has completed, so the caller may reuse its plan buffer as soon
+// as a call returns.
+struct Staging {
+  void* host = nullptr;
+  size_t cap = 0;
+  cudaEvent_t done = nullptr;
+  bool pending = false;
+};
+constexpr int kSlots = 4;
+std::mutex g_stage_mu;
+Staging g_stage[kSlots];
+int g_stage_next = 0;
+
+int upload(const void* src, size_t n, void* dst, cudaStream_t stream) {
+  std::lock_guard<std::mutex> lock(g_stage_mu);
+  Staging& s = g_stage[g_stage_next];
+  g_stage_next = (g_stage_next + 1) % kSlots;
+  cudaError_t e;
+  if (s.pending) {
+    e = cudaEventSynchronize(s.done);
+    if (e != cudaSuccess) return cuda_fail(e);
+    s.pending = false;
+  }
+  if (!s.done) {
+    e = cudaEventCreateWithFlags(&s.done, cudaEventDisableTiming);
+    if (e != cudaSuccess) return cuda_fail(e);
+  }
+  if (s.cap < n) {
+    if (s.host) cudaFreeHost(s.host);
+    s.host = nullptr;
+    s.cap = 0;
+    e = cudaHostAlloc(&s.host, n, cudaHostAllocDefault);
+    if (e != cudaSuccess) return cuda_fail(e);
+    s.cap = n;
+  }
+  std::memcpy(s.host, src, n);
+  e = cudaMemcpyAsync(dst, s.host, n, cudaMemcpyHostToDevice, stream);
+  if (e != cudaSuccess) return cuda_fail(e);
+  e = cudaEventRecord(s.done, stream);
+  if (e != cudaSuccess) return cuda_fail(e);
+  s.pending = true;
+  return SKV_OK;
+}
+
+// ------------------------------------------------------------ tensor maps
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      f = nullptr;
+    return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+  }();
+  return fn;
+}
+
+// bf16 tensor [rows][heads][d] seen as a 3-D map with a {64, box_h, box_rows}
+// box and the 128-byte swizzle: one box fills box_h * box_rows rows of 128
+// bytes of shared memory.
+int make_map(CUtensorMap* map, const void* base, int64_t rows, int heads, int d, int box_h, int box_rows) {
+  auto enc = encode_fn();
+  if (!enc) return SKV_ECUDA;
+  if (reinterpret_cast<uintptr_t>(base) % 16 != 0) return SKV_EINVAL;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(heads), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(heads) * d * 2};
+  cuuint32_t box[3] = {64, static_cast<cuuint32_t>(box_h), static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t es[3] = {1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? SKV_OK : SKV_ECUDA;
+}
+
+int num_sms() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  return n;
+}
+
+template <class T>
+T* at(void* base, uint64_t off) {
+  return reinterpret_cast<T*>(static_cast<uint8_t*>(base) + off);
+}
+template <class T>
+const T* at(const void* base, uint64_t off) {
+  return reinterpret_cast<const T*>(static_cast<const uint8_t*>(base) + off);
+}
+
+bool aligned16(const void* p) { return reinterpret_cast<uintptr_t>(p) % 16 == 0; }
+
+// Device plan copy + zeroed control block and queue counters.
+int prepare_ws(const PlanHeader& h, const void* plan, void* ws, const WsLayout& w, cudaStream_t stream) {
+  cudaError_t e = cudaMemsetAsync(ws, 0, 256, stream);  // status word
+  if (e != cudaSuccess) return cuda_fail(e);
+  e = cudaMemsetAsync(at<uint8_t>(ws, w.counters), 0, 2 * sizeof(int32_t) * static_cast<size_t>(h.P), stream);
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (h.dev.bytes > 0) return upload(static_cast<const uint8_t*>(plan) + h.dev_off, h.dev.bytes, at<uint8_t>(ws, w.dev), stream);
+  return SKV_OK;
+}
+
+}  // namespace
+}  // namespace skv
+
+using namespace skv;
+
+extern "C" const char* skv_strerror(int code) {
+  switch (code) {
+    case SKV_OK: return "ok";
+    case SKV_EINVAL: return "invalid argument";
+    case SKV_EWORKSPACE: return "buffer smaller than required";
+    case SKV_EUNSUPPORTED: return "unsupported problem (head_dim, group size or sizes)";
+    case SKV_ECUDA: return "CUDA runtime error";
+    case SKV_EPLAN: return "not a plan written by skv_plan";
+    case SKV_ETIMEOUT: return "a device-side wait timed out";
+    case SKV_EDEVICE: return "a kernel found an inconsistent work list";
+    default: return "unknown status";
+  }
+}
+
+extern "C" int skv_last_cuda_error(void) { return g_last_cuda; }
+
+extern "C" int skv_set_unit_timer(void* fwd_stamps, void* bwd_stamps) {
+  g_fwd_stamps = static_cast<long long*>(fwd_stamps);
+  g_bwd_stamps = static_cast<long long*>(bwd_stamps);
+  return SKV_OK;
+}
+
+extern "C" int skv_attn_fwd(const void* plan, const void* q, const void* k, const void* v, void* ws,
+                            size_t ws_bytes, skv_stream_t stream_) {
+  const PlanHeader* h = header_of(plan);
+  if (!h) return SKV_EPLAN;
+  if (!q || !k || !v || !ws) return SKV_EINVAL;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || reinterpret_cast<uintptr_t>(ws) % 256 != 0)
+    return SKV_EINVAL;
+  const WsLayout w = ws_layout(*h);
+  if (ws_bytes < w.fwd_end) return SKV_EWORKSPACE;
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  int rc = prepare_ws(*h, plan, ws, w, stream);
+  if (rc != SKV_OK) return rc;
+  if (h->n_fwd == 0) return SKV_OK;
+  CUtensorMap tq, tk, tv;
+  if ((rc = make_map(&tq, q, h->Nq, h->Hq, h->d, h->G, h->tile_tokens)) != SKV_OK) return rc;
+  if ((rc = make_map(&tk, k, h->Ltot, h->Hkv, h->d, 1, kTileN)) != SKV_OK) return rc;
+  if ((rc = make_map(&tv, v, h->Ltot, h->Hkv, h->d, 1, kTileN)) != SKV_OK) return rc;
+  const uint8_t* dev = at<uint8_t>(ws, w.dev);
+  FwdParams p{};
+  p.mtiles = at<MTile>(dev, h->dev.mtiles);
+  p.tok_kend = at<int32_t>(dev, h->dev.tok_kend);
+  p.units = at<FwdUnit>(dev, h->dev.fwd_units);
+  p.part_off = at<int32_t>(dev, h->dev.fwd_part_off);
+  p.counters = at<int32_t>(ws, w.counters);
+  p.status = at<int>(ws, w.status);
+  p.part_o = at<float>(ws, w.fwd_o);
+  p.part_lse = at<float>(ws, w.fwd_lse);
+  p.stamps = g_fwd_stamps;
+  p.timeout_ns = kTimeoutNs;
+  p.P = h->P;
+  p.G = h->G;
+  p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(h->d)));
+  int sms = num_sms();
+  if (sms <= 0) return cuda_fail(cudaGetLastError());
+  const int grid = static_cast<int>(std::min<int64_t>(sms, h->n_fwd));
+  cudaError_t e = launch_fwd(h->d, tq, tk, tv, p, grid, stream);
+  if (e != cudaSuccess) return cuda_fail(e);
+  return SKV_OK;
+}
+
+extern "C" int skv_lse_merge(const void* plan, const void* ws, void* o, float* lse, skv_stream_t stream_) {
+  const PlanHeader* h = header_of(plan);
+  if (!h) return SKV_EPLAN;
+  if (!ws || !o || !lse || !aligned16(o) || !aligned16(lse)) return SKV_EINVAL;
+  const WsLayout w = ws_layout(*h);
+  const uint8_t* dev = at<uint8_t>(ws, w.dev);
+  MergeParams p{};
+  p.mtiles = at<MTile>(dev, h->dev.mtiles);
+  p.merge_off = at<int32_t>(dev, h->dev.merge_off);
+  p.merge_list = at<int32_t>(dev, h->dev.merge_list);
+  p.part_o = at<float>(ws, w.fwd_o);
+  p.part_lse = at<float>(ws, w.fwd_lse);
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  p.n_rows = h->n_mtiles * h->Hkv * kTileM;
+  p.Hkv = h->Hkv;
+  p.G = h->G;
+  p.Hq = h->Hq;
+  cudaError_t e = launch_merge(h->d, p, reinterpret_cast<cudaStream_t>(stream_));
+  if (e != cudaSuccess) return cuda_fail(e);
+  return SKV_OK;
+}
+
+extern "C" int skv_attn_bwd(const void* plan, const void* q, const void* k, const void* v, const void* o,
+                            const float* lse, const void* dout, void* dq, void* dk, void* dv, void* ws,
+                            size_t ws_bytes, skv_stream_t stream_) {
+  const PlanHeader* h = header_of(plan);
+  if (!h) return SKV_EPLAN;
+  if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv || !ws) return SKV_EINVAL;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse) || !aligned16(dout) ||
+      !aligned16(dq) || !aligned16(dk) || !aligned16(dv) || reinterpret_cast<uintptr_t>(ws) % 256 != 0)
+    return SKV_EINVAL;
+  const WsLayout w = ws_layout(*h);
+  if (ws_bytes < w.bwd_end) return SKV_EWORKSPACE;
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  int rc = prepare_ws(*h, plan, ws, w, stream);
+  if (rc != SKV_OK) return rc;
+  cudaError_t e;
+  // keys no query attends to: zero gradients
+  const int64_t* dead = at<int64_t>(plan, h->dead_off);
+  const size_t row_bytes = static_cast<size_t>(h->Hkv) * h->d * 2;
+  for (int b = 0; b < h->B; ++b) {
+    const int64_t k0 = dead[2 * b], k1 = dead[2 * b + 1];
+    if (k1 <= k0) continue;
+    e = cudaMemsetAsync(static_cast<uint8_t*>(dk) + k0 * row_bytes, 0, (k1 - k0) * row_bytes, stream);
+    if (e != cudaSuccess) return cuda_fail(e);
+    e = cudaMemsetAsync(static_cast<uint8_t*>(dv) + k0 * row_bytes, 0, (k1 - k0) * row_bytes, stream);
+    if (e != cudaSuccess) return cuda_fail(e);
+  }
+  float* delta = at<float>(ws, w.bwd_delta);
+  float* dq_acc = at<float>(ws, w.bwd_dq);
+  const long long n_rows = h->Nq * h->Hq;
+  e = launch_bwd_prep(h->d, static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dout), delta,
+                      dq_acc, n_rows, stream);
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (h->n_bwd > 0) {
+    CUtensorMap tq, tk, tv, tdo;
+    if ((rc = make_map(&tq, q, h->Nq, h->Hq, h->d, h->G, h->tile_tokens)) != SKV_OK) return rc;
+    if ((rc = make_map(&tdo, dout, h->Nq, h->Hq, h->d, h->G, h->tile_tokens)) != SKV_OK) return rc;
+    if ((rc = make_map(&tk, k, h->Ltot, h->Hkv, h->d, 1, kTileN)) != SKV_OK) return rc;
+    if ((rc = make_map(&tv, v, h->Ltot, h->Hkv, h->d, 1, kTileN)) != SKV_OK) return rc;
+    const uint8_t* dev = at<uint8_t>(ws, w.dev);
+    BwdParams p{};
+    p.mtiles = at<MTile>(dev, h->dev.mtiles);
+    p.tok_kend = at<int32_t>(dev, h->dev.tok_kend);
+    p.units = at<BwdUnit>(dev, h->dev.bwd_units);
+    p.part_off = at<int32_t>(dev, h->dev.bwd_part_off);
+    p.counters = at<int32_t>(ws, w.counters) + h->P;
+    p.status = at<int>(ws, w.status);
+    p.lse = lse;
+    p.delta = delta;
+    p.dq_acc = dq_acc;
+    p.dk = static_cast<__nv_bfloat16*>(dk);
+    p.dv = static_cast<__nv_bfloat16*>(dv);
+    p.stamps = g_bwd_stamps;
+    p.timeout_ns = kTimeoutNs;
+    p.P = h->P;
+    p.G = h->G;
+    p.Hq = h->Hq;
+    p.Hkv = h->Hkv;
+    p.scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(h->d)));
+    p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(h->d)));
+    int sms = num_sms();
+    if (sms <= 0) return cuda_fail(cudaGetLastError());
+    const int grid = static_cast<int>(std::min<int64_t>(sms, h->n_bwd));
+    e = launch_bwd(h->d, tq, tk, tv, tdo, p, grid, stream);
+    if (e != cudaSuccess) return cuda_fail(e);
+  }
+  e = launch_dq_cast(dq_acc, static_cast<__nv_bfloat16*>(dq),
+                     static_cast<float>(1.0 / std::sqrt(static_cast<double>(h->d))), n_rows * h->d, stream);
+  if (e != cudaSuccess) return cuda_fail(e);
+  return SKV_OK;
+}
+
+extern "C" int skv_status(const void* ws, skv_stream_t stream_) {
+  if (!ws) return SKV_EINVAL;
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  int st = 0;
+  cudaError_t e = cudaMemcpyAsync(&st, ws, sizeof(int), cudaMemcpyDeviceToHost, stream);
+  if (e != cudaSuccess) return cuda_fail(e);
+  e = cudaStreamSynchronize(stream);
+  if (e != cudaSuccess) return cuda_fail(e);
+  return st;
+}

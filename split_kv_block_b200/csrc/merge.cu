@@ -1,0 +1,179 @@
+// Memory-bound kernels around the split-KV attention:
+//   * the exact log-sum-exp merge of per-chunk partials ("Split-KV's Core
+//     Mechanism": partial results of every KV shard aggregated through
+//     query-sized tensors; exact, per the Abstract);
+//   * the backward preprocess D = rowsum(dO * O) with the zeroing of the fp32
+//     dQ accumulator;
+//   * the final dQ rounding to bf16 (the sum over chunks happened in fp32).
+// One warp per (query token, head) row, each lane owning d/32 consecutive
+// elements so every row is read and written as whole 128-byte lines.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "kernels.h"
+#include "sm100.cuh"
+
+namespace skv {
+
+namespace {
+
+template <int D>
+struct Vec;
+template <>
+struct Vec<128> {
+  static constexpr int N = 4;
+};
+template <>
+struct Vec<64> {
+  static constexpr int N = 2;
+};
+
+template <int D>
+__device__ __forceinline__ void load_row(const float* src, int lane, float (&x)[Vec<D>::N]) {
+  if constexpr (D == 128) {
+    float4 t = *reinterpret_cast<const float4*>(src + lane * 4);
+    x[0] = t.x; x[1] = t.y; x[2] = t.z; x[3] = t.w;
+  } else {
+    float2 t = *reinterpret_cast<const float2*>(src + lane * 2);
+    x[0] = t.x; x[1] = t.y;
+  }
+}
+
+template <int D>
+__device__ __forceinline__ void load_row_bf16(const __nv_bfloat16* src, int lane, float (&x)[Vec<D>::N]) {
+  if constexpr (D == 128) {
+    uint2 t = *reinterpret_cast<const uint2*>(src + lane * 4);
+    __nv_bfloat162 a = *reinterpret_cast<__nv_bfloat162*>(&t.x), b = *reinterpret_cast<__nv_bfloat162*>(&t.y);
+    float2 fa = __bfloat1622float2(a), fb = __bfloat1622float2(b);
+    x[0] = fa.x; x[1] = fa.y; x[2] = fb.x; x[3] = fb.y;
+  } else {
+    uint32_t t = *reinterpret_cast<const uint32_t*>(src + lane * 2);
+    float2 fa = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&t));
+    x[0] = fa.x; x[1] = fa.y;
+  }
+}
+
+template <int D>
+__device__ __forceinline__ void store_row_bf16(__nv_bfloat16* dst, int lane, const float (&x)[Vec<D>::N]) {
+  if constexpr (D == 128) {
+    uint2 t;
+    t.x = pack_bf16(x[0], x[1]);
+    t.y = pack_bf16(x[2], x[3]);
+    *reinterpret_cast<uint2*>(dst + lane * 4) = t;
+  } else {
+    *reinterpret_cast<uint32_t*>(dst + lane * 2) = pack_bf16(x[0], x[1]);
+  }
+}
+
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.69314718055994531f;
+
+// Per (query tile, kv head, row): m = max LSE_c, LSE = m + ln sum exp(LSE_c - m),
+// O = sum exp(LSE_c - LSE) O_c over the tile's partials in ascending key order.
+template <int D>
+__global__ void __launch_bounds__(256) merge_kernel(const MergeParams p) {
+  const long long row = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (row >= p.n_rows) return;
+  const int r = static_cast<int>(row % kTileM);
+  const long long slot = row / kTileM;  // mt * Hkv + g
+  const int g = static_cast<int>(slot % p.Hkv);
+  const int mt = static_cast<int>(slot / p.Hkv);
+  const MTile M = p.mtiles[mt];
+  const int tl = r / p.G;
+  if (tl >= M.ntok) return;
+  const int token = M.tok0 + tl;
+  const int h = g * p.G + r % p.G;
+  const int c0 = p.merge_off[slot], c1 = p.merge_off[slot + 1];
+  float m = -INFINITY;
+  for (int c = c0; c < c1; ++c) m = fmaxf(m, p.part_lse[static_cast<size_t>(p.merge_list[c]) * kTileM + r]);
+  float acc[Vec<D>::N] = {};
+  float den = 0.f;
+  if (m != -INFINITY) {
+    for (int c = c0; c < c1; ++c) {
+      const int u = p.merge_list[c];
+      const float lc = p.part_lse[static_cast<size_t>(u) * kTileM + r];
+      if (lc == -INFINITY) continue;
+      const float w = ex2((lc - m) * kLog2e);
+      float x[Vec<D>::N];
+      load_row<D>(p.part_o + (static_cast<size_t>(u) * kTileM + r) * D, lane, x);
+#pragma unroll
+      for (int i = 0; i < Vec<D>::N; ++i) acc[i] += w * x[i];
+      den += w;
+    }
+  }
+  const float inv = den > 0.f ? 1.f / den : 0.f;
+#pragma unroll
+  for (int i = 0; i < Vec<D>::N; ++i) acc[i] *= inv;
+  store_row_bf16<D>(p.o + (static_cast<size_t>(token) * p.Hq + h) * D, lane, acc);
+  if (lane == 0) p.lse[static_cast<size_t>(token) * p.Hq + h] = den > 0.f ? m + lg2(den) * kLn2 : -INFINITY;
+}
+
+// D = rowsum(dO * O) per (token, head); zeroes that row of the dQ accumulator.
+template <int D>
+__global__ void __launch_bounds__(256) bwd_prep_kernel(const __nv_bfloat16* o, const __nv_bfloat16* dout,
+                                                       float* delta, float* dq_acc, long long n_rows) {
+  const long long row = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (row >= n_rows) return;
+  float a[Vec<D>::N], b[Vec<D>::N];
+  load_row_bf16<D>(o + row * D, lane, a);
+  load_row_bf16<D>(dout + row * D, lane, b);
+  float s = 0.f;
+#pragma unroll
+  for (int i = 0; i < Vec<D>::N; ++i) s += a[i] * b[i];
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+  if (lane == 0) delta[row] = s;
+  float* z = dq_acc + row * D + lane * Vec<D>::N;
+  if constexpr (D == 128)
+    *reinterpret_cast<float4*>(z) = make_float4(0.f, 0.f, 0.f, 0.f);
+  else
+    *reinterpret_cast<float2*>(z) = make_float2(0.f, 0.f);
+}
+
+// dq = bf16(scale * dq_acc), 4 elements per thread.
+__global__ void __launch_bounds__(256) dq_cast_kernel(const float* acc, __nv_bfloat16* dq, float scale, long long n4) {
+  for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < n4;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const float4 x = reinterpret_cast<const float4*>(acc)[i];
+    uint2 t;
+    t.x = pack_bf16(x.x * scale, x.y * scale);
+    t.y = pack_bf16(x.z * scale, x.w * scale);
+    reinterpret_cast<uint2*>(dq)[i] = t;
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_merge(int d, const MergeParams& p, cudaStream_t stream) {
+  if (p.n_rows == 0) return cudaSuccess;
+  const long long blocks = (p.n_rows * 32 + 255) / 256;
+  if (d == 64)
+    merge_kernel<64><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(p);
+  else
+    merge_kernel<128><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_bwd_prep(int d, const __nv_bfloat16* o, const __nv_bfloat16* dout, float* delta, float* dq_acc,
+                            long long n_rows, cudaStream_t stream) {
+  if (n_rows == 0) return cudaSuccess;
+  const long long blocks = (n_rows * 32 + 255) / 256;
+  if (d == 64)
+    bwd_prep_kernel<64><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(o, dout, delta, dq_acc, n_rows);
+  else
+    bwd_prep_kernel<128><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(o, dout, delta, dq_acc, n_rows);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_dq_cast(const float* dq_acc, __nv_bfloat16* dq, float scale, long long n, cudaStream_t stream) {
+  if (n == 0) return cudaSuccess;
+  const long long n4 = n / 4;
+  long long blocks = (n4 + 255) / 256;
+  if (blocks > 148 * 16) blocks = 148 * 16;
+  dq_cast_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(dq_acc, dq, scale, n4);
+  return cudaGetLastError();
+}
+
+}  // namespace skv

@@ -1,0 +1,443 @@
+// Host planner: validation, work items with realized cost, LPT / static
+// placement, and the work lists the kernels read.
+//
+// Sources: "Split-KV: Breaking the Context Parallelism Bottleneck in
+// Diffusion Drafter Training", section "LPT Scheduling: Load Balancing with
+// Real Attention Costs" (cost of each KV block = attention it actually incurs;
+// longest first onto the least-loaded rank; the token-count split it
+// replaces) and "Split-KV: Efficient Context Parallelism for Training
+// Diffusion Drafters", Abstract (LPT over context K/V chunks by realized
+// attention cost, planned every step).
+//
+// Cost of an item (b, c, g, s) with relative key range [lo, hi):
+//   G * block_q * sum_j |[lo, hi) ∩ [0, a_j)|
+// computed from the sample's sorted anchors and their prefix sums in
+// O(log A) per item.
+#include <algorithm>
+#include <cstring>
+#include <functional>
+#include <numeric>
+#include <queue>
+#include <vector>
+
+#include "plan_layout.h"
+
+namespace skv {
+namespace {
+
+struct Prob {
+  int B, Hq, Hkv, d, S, C, sub, P, G, TT;
+  int64_t Nq, Ltot;
+  const int64_t* ctx;
+  const int32_t* aoff;
+  const int64_t* anchors;
+};
+
+int validate(const skv_problem* p, Prob& q) {
+  if (!p || p->num_samples < 1 || !p->ctx_offsets || !p->anchor_offsets) return SKV_EINVAL;
+  q.B = p->num_samples;
+  q.Hq = p->num_q_heads;
+  q.Hkv = p->num_kv_heads;
+  q.d = p->head_dim;
+  q.S = p->block_q;
+  q.C = p->chunk_kv;
+  q.sub = p->sub_chunks;
+  q.P = p->num_partitions;
+  q.ctx = p->ctx_offsets;
+  q.aoff = p->anchor_offsets;
+  q.anchors = p->anchors;
+  if (q.S < 1 || q.C < 1 || q.sub < 1 || q.P < 1 || q.Hq < 1 || q.Hkv < 1) return SKV_EINVAL;
+  if (q.C % q.sub != 0 || q.Hq % q.Hkv != 0) return SKV_EINVAL;
+  if (q.ctx[0] != 0 || q.aoff[0] != 0) return SKV_EINVAL;
+  for (int b = 0; b < q.B; ++b) {
+    if (q.ctx[b + 1] <= q.ctx[b]) return SKV_EINVAL;
+    if (q.aoff[b + 1] < q.aoff[b]) return SKV_EINVAL;
+  }
+  const int64_t A = q.aoff[q.B];
+  if (A > 0 && !q.anchors) return SKV_EINVAL;
+  for (int b = 0; b < q.B; ++b) {
+    const int64_t L = q.ctx[b + 1] - q.ctx[b];
+    for (int32_t j = q.aoff[b]; j < q.aoff[b + 1]; ++j)
+      if (q.anchors[j] < 1 || q.anchors[j] > L) return SKV_EINVAL;
+  }
+  q.G = q.Hq / q.Hkv;
+  if (q.d != 64 && q.d != 128) return SKV_EUNSUPPORTED;
+  if (q.G > kTileM || kTileM % q.G != 0) return SKV_EUNSUPPORTED;
+  q.TT = kTileM / q.G;
+  q.Nq = A * q.S;
+  q.Ltot = q.ctx[q.B];
+  // 32-bit indices on the device: keys and query tokens (with tile slack).
+  if (q.Ltot > (int64_t(1) << 31) - 4 * kTileN) return SKV_EUNSUPPORTED;
+  if (q.Nq > (int64_t(1) << 31) - 4 * kTileM) return SKV_EUNSUPPORTED;
+  if (q.P > (1 << 20)) return SKV_EUNSUPPORTED;
+  return SKV_OK;
+}
+
+struct SampleAnchors {
+  std::vector<int64_t> a;       // sorted
+  std::vector<int64_t> prefix;  // prefix[i] = a[0] + ... + a[i-1]
+  int64_t max_a = 0;
+};
+
+// sum_j max(0, min(hi, a_j) - lo), relative coordinates, lo < hi.
+int64_t pair_sum(const SampleAnchors& s, int64_t lo, int64_t hi) {
+  const auto& a = s.a;
+  const size_t i0 = std::upper_bound(a.begin(), a.end(), lo) - a.begin();  // first a > lo
+  const size_t i1 = std::lower_bound(a.begin(), a.end(), hi) - a.begin();  // first a >= hi
+  int64_t mid = 0;
+  if (i1 > i0) mid = (s.prefix[i1] - s.prefix[i0]) - static_cast<int64_t>(i1 - i0) * lo;
+  const int64_t top = static_cast<int64_t>(a.size() - i1) * (hi - lo);
+  return mid + top;
+}
+
+struct Built {
+  std::vector<skv_item> items;
+  std::vector<int64_t> load;
+  std::vector<int32_t> placement;  // item ids in placement order
+  std::vector<MTile> mtiles;
+  std::vector<int32_t> sample_mt;  // [B+1]
+  std::vector<int32_t> tok_kend;
+  std::vector<FwdUnit> fwd;
+  std::vector<int32_t> fwd_part_off;
+  std::vector<int32_t> merge_off, merge_list;
+  std::vector<BwdUnit> bwd;
+  std::vector<int32_t> bwd_part_off;
+  std::vector<int64_t> dead;  // [2B]
+  int64_t total_cost = 0;
+  double imbalance = 0.0;
+};
+
+void make_items(const Prob& q, int policy, const std::vector<SampleAnchors>& sa, Built& out) {
+  auto cost = [&](int b, int64_t lo_abs, int64_t hi_abs) {
+    return static_cast<int64_t>(q.G) * q.S * pair_sum(sa[b], lo_abs - q.ctx[b], hi_abs - q.ctx[b]);
+  };
+  out.items.clear();
+  if (policy == SKV_PLAN_LPT) {
+    const int64_t cs = q.C / q.sub;
+    for (int b = 0; b < q.B; ++b) {
+      const int64_t k0 = q.ctx[b], L = q.ctx[b + 1] - k0;
+      const int64_t nc = (L + q.C - 1) / q.C;
+      for (int64_t c = 0; c < nc; ++c) {
+        const int64_t c_end = std::min<int64_t>((c + 1) * q.C, L);
+        for (int g = 0; g < q.Hkv; ++g)
+          for (int s = 0; s < q.sub; ++s) {
+            const int64_t lo = c * q.C + s * cs, hi = std::min<int64_t>(c * q.C + (s + 1) * cs, c_end);
+            if (hi <= lo) continue;
+            skv_item it{};
+            it.b = b;
+            it.c = static_cast<int32_t>(c);
+            it.g = g;
+            it.sub = s;
+            it.key_begin = k0 + lo;
+            it.key_end = k0 + hi;
+            it.cost = cost(b, k0 + lo, k0 + hi);
+            it.partition = -1;
+            it.order = -1;
+            out.items.push_back(it);
+          }
+      }
+    }
+  } else {
+    // Pieces of the equal-token split cut at chunk boundaries, in stream order.
+    struct Piece { int b; int64_t c, lo, hi; int p, s; };
+    std::vector<Piece> pieces;
+    const int64_t T = q.Ltot;
+    int b = 0;
+    for (int p = 0; p < q.P; ++p) {
+      const int64_t t0 = (static_cast<int64_t>(p) * T) / q.P, t1 = (static_cast<int64_t>(p + 1) * T) / q.P;
+      if (t1 <= t0) continue;
+      while (b < q.B && q.ctx[b + 1] <= t0) ++b;
+      for (int bb = b; bb < q.B && q.ctx[bb] < t1; ++bb) {
+        const int64_t k0 = q.ctx[bb], k1 = q.ctx[bb + 1];
+        const int64_t lo_rel = std::max(t0, k0) - k0, hi_rel = std::min(t1, k1) - k0;
+        for (int64_t c = lo_rel / q.C; c * q.C < hi_rel; ++c) {
+          const int64_t lo = std::max(t0, k0 + c * q.C), hi = std::min({t1, k0 + (c + 1) * q.C, k1});
+          if (hi > lo) pieces.push_back({bb, c, lo, hi, p, 0});
+        }
+      }
+    }
+    for (size_t i = 0; i < pieces.size(); ++i)
+      if (i > 0 && pieces[i - 1].b == pieces[i].b && pieces[i - 1].c == pieces[i].c)
+        pieces[i].s = pieces[i - 1].s + 1;
+    size_t i = 0;
+    while (i < pieces.size()) {
+      size_t e = i;
+      while (e < pieces.size() && pieces[e].b == pieces[i].b && pieces[e].c == pieces[i].c) ++e;
+      for (int g = 0; g < q.Hkv; ++g)
+        for (size_t k = i; k < e; ++k) {
+          const Piece& pc = pieces[k];
+          skv_item it{};
+          it.b = pc.b;
+          it.c = static_cast<int32_t>(pc.c);
+          it.g = g;
+          it.sub = pc.s;
+          it.key_begin = pc.lo;
+          it.key_end = pc.hi;
+          it.cost = cost(pc.b, pc.lo, pc.hi);
+          it.partition = pc.p;
+          it.order = -1;
+          out.items.push_back(it);
+        }
+      i = e;
+    }
+  }
+}
+
+void place(const Prob& q, int policy, Built& out) {
+  const size_t n = out.items.size();
+  out.placement.resize(n);
+  std::iota(out.placement.begin(), out.placement.end(), 0);
+  out.load.assign(q.P, 0);
+  if (policy == SKV_PLAN_LPT) {
+    // Items are generated in (b, c, g, s) order, so the index breaks ties.
+    std::sort(out.placement.begin(), out.placement.end(), [&](int32_t x, int32_t y) {
+      if (out.items[x].cost != out.items[y].cost) return out.items[x].cost > out.items[y].cost;
+      return x < y;
+    });
+    using Slot = std::pair<int64_t, int32_t>;  // (load, partition): smallest first
+    std::priority_queue<Slot, std::vector<Slot>, std::greater<Slot>> heap;
+    for (int32_t p = 0; p < q.P; ++p) heap.push({0, p});
+    for (size_t r = 0; r < n; ++r) {
+      skv_item& it = out.items[out.placement[r]];
+      Slot s = heap.top();
+      heap.pop();
+      it.partition = s.second;
+      it.order = static_cast<int32_t>(r);
+      s.first += it.cost;
+      heap.push(s);
+    }
+  } else {
+    for (size_t r = 0; r < n; ++r) out.items[r].order = static_cast<int32_t>(r);
+  }
+  out.total_cost = 0;
+  for (const auto& it : out.items) {
+    out.load[it.partition] += it.cost;
+    out.total_cost += it.cost;
+  }
+  const int64_t mx = *std::max_element(out.load.begin(), out.load.end());
+  out.imbalance = out.total_cost > 0 ? static_cast<double>(mx) * q.P / static_cast<double>(out.total_cost) - 1.0 : 0.0;
+}
+
+void make_lists(const Prob& q, const std::vector<SampleAnchors>& sa, Built& out) {
+  // query tiles
+  out.mtiles.clear();
+  out.sample_mt.assign(q.B + 1, 0);
+  out.tok_kend.assign(static_cast<size_t>(q.Nq), 0);
+  for (int b = 0; b < q.B; ++b) {
+    out.sample_mt[b] = static_cast<int32_t>(out.mtiles.size());
+    const int64_t t_begin = static_cast<int64_t>(q.aoff[b]) * q.S, t_end = static_cast<int64_t>(q.aoff[b + 1]) * q.S;
+    for (int64_t t = t_begin; t < t_end; ++t)
+      out.tok_kend[t] = static_cast<int32_t>(q.ctx[b] + q.anchors[t / q.S]);
+    for (int64_t t0 = t_begin; t0 < t_end; t0 += q.TT) {
+      const int64_t nt = std::min<int64_t>(q.TT, t_end - t0);
+      int64_t amax = 0;
+      for (int64_t j = t0 / q.S; j <= (t0 + nt - 1) / q.S; ++j) amax = std::max(amax, q.anchors[j]);
+      out.mtiles.push_back({b, static_cast<int32_t>(t0), static_cast<int32_t>(nt), static_cast<int32_t>(q.ctx[b] + amax)});
+    }
+  }
+  out.sample_mt[q.B] = static_cast<int32_t>(out.mtiles.size());
+
+  // items of every partition in placement order
+  std::vector<std::vector<int32_t>> by_part(q.P);
+  for (int32_t id : out.placement) by_part[out.items[id].partition].push_back(id);
+
+  out.fwd.clear();
+  out.fwd_part_off.assign(q.P + 1, 0);
+  out.bwd.clear();
+  out.bwd_part_off.assign(q.P + 1, 0);
+  std::vector<std::pair<int64_t, int32_t>> tiles;
+  for (int p = 0; p < q.P; ++p) {
+    out.fwd_part_off[p] = static_cast<int32_t>(out.fwd.size());
+    out.bwd_part_off[p] = static_cast<int32_t>(out.bwd.size());
+    for (int32_t id : by_part[p]) {
+      const skv_item& it = out.items[id];
+      // forward: live query tiles, longest key range first
+      tiles.clear();
+      for (int32_t mt = out.sample_mt[it.b]; mt < out.sample_mt[it.b + 1]; ++mt) {
+        const int64_t ke = std::min<int64_t>(it.key_end, out.mtiles[mt].kmax);
+        if (ke > it.key_begin) tiles.push_back({-(ke - it.key_begin), mt});
+      }
+      std::sort(tiles.begin(), tiles.end());
+      for (auto& t : tiles) {
+        FwdUnit u{};
+        u.mt = t.second;
+        u.g = it.g;
+        u.kbeg = static_cast<int32_t>(it.key_begin);
+        u.kend = static_cast<int32_t>(it.key_begin - t.first);
+        u.item = id;
+        u.part = p;
+        out.fwd.push_back(u);
+      }
+      // backward: key tiles below the sample's largest anchor
+      const int64_t kmax_b = q.ctx[it.b] + sa[it.b].max_a;
+      for (int64_t kb = it.key_begin; kb < it.key_end && kb < kmax_b; kb += kTileN) {
+        BwdUnit u{};
+        u.b = it.b;
+        u.g = it.g;
+        u.kbeg = static_cast<int32_t>(kb);
+        u.kend = static_cast<int32_t>(std::min<int64_t>(kb + kTileN, it.key_end));
+        u.mt_begin = out.sample_mt[it.b];
+        u.mt_end = out.sample_mt[it.b + 1];
+        u.item = id;
+        u.part = p;
+        out.bwd.push_back(u);
+      }
+    }
+  }
+  out.fwd_part_off[q.P] = static_cast<int32_t>(out.fwd.size());
+  out.bwd_part_off[q.P] = static_cast<int32_t>(out.bwd.size());
+
+  // merge lists: per (query tile, kv head), forward units in ascending key order
+  const size_t nslots = out.mtiles.size() * static_cast<size_t>(q.Hkv);
+  out.merge_off.assign(nslots + 1, 0);
+  for (const auto& u : out.fwd) out.merge_off[static_cast<size_t>(u.mt) * q.Hkv + u.g + 1]++;
+  for (size_t i = 0; i < nslots; ++i) out.merge_off[i + 1] += out.merge_off[i];
+  out.merge_list.assign(out.fwd.size(), 0);
+  std::vector<int32_t> fill(out.merge_off.begin(), out.merge_off.end() - 1);
+  for (size_t i = 0; i < out.fwd.size(); ++i) {
+    const auto& u = out.fwd[i];
+    out.merge_list[fill[static_cast<size_t>(u.mt) * q.Hkv + u.g]++] = static_cast<int32_t>(i);
+  }
+  for (size_t sidx = 0; sidx < nslots; ++sidx)
+    std::sort(out.merge_list.begin() + out.merge_off[sidx], out.merge_list.begin() + out.merge_off[sidx + 1],
+              [&](int32_t x, int32_t y) { return out.fwd[x].kbeg < out.fwd[y].kbeg; });
+
+  // keys whose gradients are zero: past the last backward tile of the sample
+  out.dead.assign(2 * static_cast<size_t>(q.B), 0);
+  std::vector<int64_t> live_end(q.B);
+  for (int b = 0; b < q.B; ++b) live_end[b] = q.ctx[b];
+  for (const auto& u : out.bwd) live_end[u.b] = std::max<int64_t>(live_end[u.b], u.kend);
+  for (int b = 0; b < q.B; ++b) {
+    out.dead[2 * b] = live_end[b];
+    out.dead[2 * b + 1] = q.ctx[b + 1];
+  }
+}
+
+int build(const skv_problem* prob, int policy, Built& out, Prob& q) {
+  if (policy != SKV_PLAN_LPT && policy != SKV_PLAN_STATIC) return SKV_EINVAL;
+  int rc = validate(prob, q);
+  if (rc != SKV_OK) return rc;
+  std::vector<SampleAnchors> sa(q.B);
+  for (int b = 0; b < q.B; ++b) {
+    sa[b].a.assign(q.anchors + q.aoff[b], q.anchors + q.aoff[b + 1]);
+    std::sort(sa[b].a.begin(), sa[b].a.end());
+    sa[b].prefix.assign(sa[b].a.size() + 1, 0);
+    for (size_t i = 0; i < sa[b].a.size(); ++i) sa[b].prefix[i + 1] = sa[b].prefix[i] + sa[b].a[i];
+    sa[b].max_a = sa[b].a.empty() ? 0 : sa[b].a.back();
+  }
+  make_items(q, policy, sa, out);
+  place(q, policy, out);
+  make_lists(q, sa, out);
+  return SKV_OK;
+}
+
+PlanHeader layout_of(const Prob& q, int policy, const Built& b) {
+  PlanHeader h{};
+  h.magic = kPlanMagic;
+  h.version = kPlanVersion;
+  h.policy = policy;
+  h.B = q.B; h.Hq = q.Hq; h.Hkv = q.Hkv; h.d = q.d; h.block_q = q.S; h.chunk_kv = q.C;
+  h.sub_chunks = q.sub; h.P = q.P; h.G = q.G; h.tile_tokens = q.TT;
+  h.Nq = q.Nq; h.Ltot = q.Ltot;
+  h.total_cost = b.total_cost;
+  h.n_items = static_cast<int64_t>(b.items.size());
+  h.n_mtiles = static_cast<int64_t>(b.mtiles.size());
+  h.n_fwd = static_cast<int64_t>(b.fwd.size());
+  h.n_bwd = static_cast<int64_t>(b.bwd.size());
+  h.imbalance = b.imbalance;
+  uint64_t off = align_up(sizeof(PlanHeader), 256);
+  h.items_off = off;
+  off = align_up(off + b.items.size() * sizeof(skv_item), 64);
+  h.load_off = off;
+  off = align_up(off + static_cast<uint64_t>(q.P) * sizeof(int64_t), 64);
+  h.dead_off = off;
+  off = align_up(off + b.dead.size() * sizeof(int64_t), 256);
+  h.dev_off = off;
+  uint64_t d = 0;
+  auto put = [&](uint64_t bytes) { uint64_t at = d; d = align_up(d + bytes, 256); return at; };
+  h.dev.mtiles = put(b.mtiles.size() * sizeof(MTile));
+  h.dev.tok_kend = put(b.tok_kend.size() * sizeof(int32_t));
+  h.dev.fwd_units = put(b.fwd.size() * sizeof(FwdUnit));
+  h.dev.fwd_part_off = put(b.fwd_part_off.size() * sizeof(int32_t));
+  h.dev.merge_off = put(b.merge_off.size() * sizeof(int32_t));
+  h.dev.merge_list = put(b.merge_list.size() * sizeof(int32_t));
+  h.dev.bwd_units = put(b.bwd.size() * sizeof(BwdUnit));
+  h.dev.bwd_part_off = put(b.bwd_part_off.size() * sizeof(int32_t));
+  h.dev.bytes = d;
+  h.total_bytes = h.dev_off + d;
+  return h;
+}
+
+template <class T>
+void copy_to(uint8_t* base, uint64_t off, const std::vector<T>& v) {
+  if (!v.empty()) std::memcpy(base + off, v.data(), v.size() * sizeof(T));
+}
+
+}  // namespace
+}  // namespace skv
+
+using namespace skv;
+
+extern "C" int skv_plan_size(const skv_problem* prob, int policy, size_t* n_items, size_t* plan_bytes,
+                             size_t* ws_fwd_bytes, size_t* ws_bwd_bytes) {
+  Built b;
+  Prob q;
+  int rc = build(prob, policy, b, q);
+  if (rc != SKV_OK) return rc;
+  PlanHeader h = layout_of(q, policy, b);
+  WsLayout w = ws_layout(h);
+  if (n_items) *n_items = b.items.size();
+  if (plan_bytes) *plan_bytes = h.total_bytes;
+  if (ws_fwd_bytes) *ws_fwd_bytes = w.fwd_end;
+  if (ws_bwd_bytes) *ws_bwd_bytes = w.bwd_end;
+  return SKV_OK;
+}
+
+extern "C" int skv_plan(const skv_problem* prob, int policy, void* plan, size_t plan_bytes,
+                        int64_t* partition_load) {
+  if (!plan) return SKV_EINVAL;
+  Built b;
+  Prob q;
+  int rc = build(prob, policy, b, q);
+  if (rc != SKV_OK) return rc;
+  PlanHeader h = layout_of(q, policy, b);
+  if (plan_bytes < h.total_bytes) return SKV_EWORKSPACE;
+  uint8_t* base = static_cast<uint8_t*>(plan);
+  std::memset(base, 0, h.total_bytes);
+  std::memcpy(base, &h, sizeof(h));
+  copy_to(base, h.items_off, b.items);
+  copy_to(base, h.load_off, b.load);
+  copy_to(base, h.dead_off, b.dead);
+  uint8_t* dev = base + h.dev_off;
+  copy_to(dev, h.dev.mtiles, b.mtiles);
+  copy_to(dev, h.dev.tok_kend, b.tok_kend);
+  copy_to(dev, h.dev.fwd_units, b.fwd);
+  copy_to(dev, h.dev.fwd_part_off, b.fwd_part_off);
+  copy_to(dev, h.dev.merge_off, b.merge_off);
+  copy_to(dev, h.dev.merge_list, b.merge_list);
+  copy_to(dev, h.dev.bwd_units, b.bwd);
+  copy_to(dev, h.dev.bwd_part_off, b.bwd_part_off);
+  if (partition_load) std::memcpy(partition_load, b.load.data(), b.load.size() * sizeof(int64_t));
+  return SKV_OK;
+}
+
+extern "C" int skv_plan_items(const void* plan, const skv_item** items, size_t* n_items) {
+  if (!plan) return SKV_EINVAL;
+  const PlanHeader* h = static_cast<const PlanHeader*>(plan);
+  if (h->magic != kPlanMagic || h->version != kPlanVersion) return SKV_EPLAN;
+  if (items) *items = reinterpret_cast<const skv_item*>(static_cast<const uint8_t*>(plan) + h->items_off);
+  if (n_items) *n_items = static_cast<size_t>(h->n_items);
+  return SKV_OK;
+}
+
+extern "C" int skv_plan_stats(const void* plan, int64_t* total_cost, int64_t* n_fwd_units, int64_t* n_bwd_units,
+                              double* imbalance) {
+  if (!plan) return SKV_EINVAL;
+  const PlanHeader* h = static_cast<const PlanHeader*>(plan);
+  if (h->magic != kPlanMagic || h->version != kPlanVersion) return SKV_EPLAN;
+  if (total_cost) *total_cost = h->total_cost;
+  if (n_fwd_units) *n_fwd_units = h->n_fwd;
+  if (n_bwd_units) *n_bwd_units = h->n_bwd;
+  if (imbalance) *imbalance = h->imbalance;
+  return SKV_OK;
+}

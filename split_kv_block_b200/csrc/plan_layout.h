@@ -1,0 +1,115 @@
+// Internal layout of the host plan buffer written by skv_plan and of the
+// device workspace. Shared by the planner (plan.cpp), the API layer (api.cu)
+// and the kernels; not part of the public ABI.
+#pragma once
+#include <cstddef>
+#include <cstdint>
+
+#include "../../include/skv.h"
+
+namespace skv {
+
+constexpr uint64_t kPlanMagic = 0x31764b5374696c53ull;  // "SlitSKv1"
+constexpr uint32_t kPlanVersion = 1;
+constexpr int kTileM = 128;  // query rows per tile (TMEM lanes)
+constexpr int kTileN = 128;  // keys per tile
+
+// One 128-row query tile of one sample. Rows are ordered (token, head within
+// the kv group): row r is token tok0 + r / G, q-head g * G + r % G.
+struct MTile {
+  int32_t b;
+  int32_t tok0;  // first query token (packed index)
+  int32_t ntok;  // tokens in the tile, <= 128 / G
+  int32_t kmax;  // absolute key end: ctx_offsets[b] + max anchor over its tokens
+};
+
+// Forward unit: one item's key range restricted to one query tile.
+struct FwdUnit {
+  int32_t mt;    // query tile
+  int32_t g;     // kv head
+  int32_t kbeg;  // absolute keys [kbeg, kend)
+  int32_t kend;
+  int32_t item;  // index into the plan's items
+  int32_t part;  // partition
+  int32_t pad0, pad1;
+};
+
+// Backward unit: one tile of <= 128 keys of one item, against every query
+// tile of the sample whose kmax exceeds kbeg.
+struct BwdUnit {
+  int32_t b;
+  int32_t g;
+  int32_t kbeg;
+  int32_t kend;
+  int32_t mt_begin;  // query tiles of sample b: [mt_begin, mt_end)
+  int32_t mt_end;
+  int32_t item;
+  int32_t part;
+};
+
+// Offsets (bytes) of the arrays of the device section, relative to its start.
+struct DevSection {
+  uint64_t mtiles;        // MTile[n_mtiles]
+  uint64_t tok_kend;      // int32[Nq]: absolute key end of every query token
+  uint64_t fwd_units;     // FwdUnit[n_fwd]
+  uint64_t fwd_part_off;  // int32[P+1]: units of partition p are [off[p], off[p+1])
+  uint64_t merge_off;     // int32[n_mtiles * Hkv + 1]
+  uint64_t merge_list;    // int32[n_fwd]: fwd unit ids per (tile, kv head), ascending kbeg
+  uint64_t bwd_units;     // BwdUnit[n_bwd]
+  uint64_t bwd_part_off;  // int32[P+1]
+  uint64_t bytes;         // total
+};
+
+struct PlanHeader {
+  uint64_t magic;
+  uint32_t version;
+  int32_t policy;
+  // problem scalars
+  int32_t B, Hq, Hkv, d, block_q, chunk_kv, sub_chunks, P;
+  int32_t G, tile_tokens;  // G = Hq / Hkv, tile_tokens = 128 / G
+  int64_t Nq, Ltot;
+  int64_t total_cost;
+  int64_t n_items, n_mtiles, n_fwd, n_bwd;
+  double imbalance;
+  uint64_t fingerprint;  // hash of the problem (shapes, offsets, anchors)
+  // host-side arrays, offsets from the start of the plan buffer
+  uint64_t items_off;      // skv_item[n_items]
+  uint64_t load_off;       // int64[P]
+  uint64_t dead_off;       // int64[2 * B]: [begin, end) keys of sample b whose dK/dV are zero
+  uint64_t dev_off;        // start of the device section (256-aligned)
+  DevSection dev;
+  uint64_t total_bytes;
+};
+
+// Workspace layout: control block, device plan section, queue counters, then
+// the pass-specific scratch.
+struct WsLayout {
+  uint64_t status;    // int32 status word at offset 0
+  uint64_t dev;       // device section copy
+  uint64_t counters;  // int32[2 * P] queue heads (forward, backward)
+  uint64_t fwd_o;     // fp32 [n_fwd][128][d] partial outputs
+  uint64_t fwd_lse;   // fp32 [n_fwd][128] partial LSE
+  uint64_t fwd_end;
+  uint64_t bwd_delta; // fp32 [Nq][Hq]: D = rowsum(dO * O)
+  uint64_t bwd_dq;    // fp32 [Nq][Hq][d]: dQ accumulator
+  uint64_t bwd_end;
+};
+
+inline uint64_t align_up(uint64_t x, uint64_t a) { return (x + a - 1) / a * a; }
+
+inline WsLayout ws_layout(const PlanHeader& h) {
+  WsLayout w{};
+  w.status = 0;
+  w.dev = 256;
+  w.counters = align_up(w.dev + h.dev.bytes, 256);
+  uint64_t scratch = align_up(w.counters + 2 * sizeof(int32_t) * static_cast<uint64_t>(h.P), 256);
+  w.fwd_o = scratch;
+  w.fwd_lse = align_up(w.fwd_o + static_cast<uint64_t>(h.n_fwd) * kTileM * h.d * 4, 256);
+  w.fwd_end = align_up(w.fwd_lse + static_cast<uint64_t>(h.n_fwd) * kTileM * 4, 256);
+  w.bwd_delta = scratch;
+  w.bwd_dq = align_up(w.bwd_delta + static_cast<uint64_t>(h.Nq) * h.Hq * 4, 256);
+  w.bwd_end = align_up(w.bwd_dq + static_cast<uint64_t>(h.Nq) * h.Hq * h.d * 4, 256);
+  return w;
+}
+
+}  // namespace skv

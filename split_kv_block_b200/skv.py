@@ -1,0 +1,237 @@
+"""Thin Python binding of libskv.so (ctypes). Argument marshalling only:
+planning runs in the library's C++ planner, every step of the attention in
+its CUDA kernels. torch provides device memory and streams.
+
+The library must be built (split_kv_block_b200.build); there is no fallback:
+calls raise if libskv.so is missing or a call fails.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+from typing import Optional
+
+import numpy as np
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libskv.so")
+
+SKV_PLAN_LPT = 0
+SKV_PLAN_STATIC = 1
+
+# Every function include/skv.h declares.
+EXPORTS = ("skv_plan_size", "skv_plan", "skv_plan_items", "skv_plan_stats", "skv_attn_fwd", "skv_lse_merge",
+           "skv_attn_bwd", "skv_status", "skv_strerror", "skv_last_cuda_error", "skv_set_unit_timer")
+
+
+class SkvError(RuntimeError):
+    def __init__(self, fn: str, code: int, msg: str):
+        super().__init__(f"{fn} failed: {msg} (status {code})")
+        self.code = code
+
+
+class _Problem(ctypes.Structure):
+    _fields_ = [("num_samples", ctypes.c_int32), ("ctx_offsets", ctypes.c_void_p), ("anchor_offsets", ctypes.c_void_p),
+                ("anchors", ctypes.c_void_p), ("block_q", ctypes.c_int32), ("chunk_kv", ctypes.c_int32),
+                ("sub_chunks", ctypes.c_int32), ("num_partitions", ctypes.c_int32), ("num_q_heads", ctypes.c_int32),
+                ("num_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32)]
+
+
+ITEM_DTYPE = np.dtype([("b", np.int32), ("c", np.int32), ("g", np.int32), ("sub", np.int32),
+                       ("key_begin", np.int64), ("key_end", np.int64), ("cost", np.int64),
+                       ("partition", np.int32), ("order", np.int32)])
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is not built; run `python -m split_kv_block_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, sz = ctypes.c_void_p, ctypes.c_size_t
+        L.skv_plan_size.argtypes = [vp, ctypes.c_int, ctypes.POINTER(sz), ctypes.POINTER(sz), ctypes.POINTER(sz),
+                                    ctypes.POINTER(sz)]
+        L.skv_plan.argtypes = [vp, ctypes.c_int, vp, sz, vp]
+        L.skv_plan_items.argtypes = [vp, ctypes.POINTER(vp), ctypes.POINTER(sz)]
+        L.skv_plan_stats.argtypes = [vp, vp, vp, vp, vp]
+        L.skv_attn_fwd.argtypes = [vp, vp, vp, vp, vp, sz, vp]
+        L.skv_lse_merge.argtypes = [vp, vp, vp, vp, vp]
+        L.skv_attn_bwd.argtypes = [vp] * 11 + [sz, vp]
+        L.skv_status.argtypes = [vp, vp]
+        L.skv_strerror.argtypes = [ctypes.c_int]
+        L.skv_strerror.restype = ctypes.c_char_p
+        L.skv_set_unit_timer.argtypes = [vp, vp]
+        for name in EXPORTS:
+            if name not in ("skv_strerror",):
+                getattr(L, name).restype = ctypes.c_int
+        _lib = L
+    return _lib
+
+
+def _check(fn: str, rc: int):
+    if rc != 0:
+        msg = lib().skv_strerror(rc).decode()
+        if rc == 4:
+            msg += f" (cuda error {lib().skv_last_cuda_error()})"
+        raise SkvError(fn, rc, msg)
+
+
+def _ptr(a) -> ctypes.c_void_p:
+    if a is None:
+        return ctypes.c_void_p(0)
+    if isinstance(a, np.ndarray):
+        return ctypes.c_void_p(a.ctypes.data)
+    return ctypes.c_void_p(a.data_ptr())
+
+
+def _stream_ptr(stream) -> ctypes.c_void_p:
+    if stream is None:
+        import torch
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(int(stream.cuda_stream))
+
+
+class _ProblemArgs:
+    """Keeps the arrays referenced by a skv_problem alive."""
+
+    def __init__(self, prob):
+        self.ctx = np.ascontiguousarray(prob.ctx_offsets, dtype=np.int64)
+        self.aoff = np.ascontiguousarray(prob.anchor_offsets, dtype=np.int32)
+        self.anchors = np.ascontiguousarray(prob.anchors, dtype=np.int64)
+        self.s = _Problem(len(self.ctx) - 1, self.ctx.ctypes.data, self.aoff.ctypes.data,
+                          self.anchors.ctypes.data if self.anchors.size else 0, prob.block_q, prob.chunk_kv,
+                          prob.sub_chunks, prob.num_partitions, prob.num_q_heads, prob.num_kv_heads, prob.head_dim)
+
+    def ref(self):
+        return ctypes.byref(self.s)
+
+
+@dataclass
+class PlanSizes:
+    n_items: int
+    plan_bytes: int
+    ws_fwd_bytes: int
+    ws_bwd_bytes: int
+
+    @property
+    def ws_bytes(self) -> int:
+        return max(self.ws_fwd_bytes, self.ws_bwd_bytes)
+
+
+def skv_plan_size(prob, policy: int = SKV_PLAN_LPT) -> PlanSizes:
+    args = _ProblemArgs(prob)
+    out = [ctypes.c_size_t() for _ in range(4)]
+    _check("skv_plan_size", lib().skv_plan_size(args.ref(), policy, *[ctypes.byref(o) for o in out]))
+    return PlanSizes(*[o.value for o in out])
+
+
+class Plan:
+    """Host plan buffer written by skv_plan."""
+
+    def __init__(self, buf: np.ndarray, loads: np.ndarray, sizes: PlanSizes, policy: int, prob):
+        self.buf = buf
+        self.partition_load = loads
+        self.sizes = sizes
+        self.policy = policy
+        self.problem = prob
+
+    @property
+    def ptr(self):
+        return ctypes.c_void_p(self.buf.ctypes.data)
+
+    def items(self) -> np.ndarray:
+        p, n = ctypes.c_void_p(), ctypes.c_size_t()
+        _check("skv_plan_items", lib().skv_plan_items(self.ptr, ctypes.byref(p), ctypes.byref(n)))
+        if n.value == 0:
+            return np.zeros(0, dtype=ITEM_DTYPE)
+        raw = (ctypes.c_uint8 * (n.value * ITEM_DTYPE.itemsize)).from_address(p.value)
+        return np.frombuffer(raw, dtype=ITEM_DTYPE).copy()
+
+    def stats(self) -> dict:
+        tc, nf, nb = ctypes.c_int64(), ctypes.c_int64(), ctypes.c_int64()
+        im = ctypes.c_double()
+        _check("skv_plan_stats", lib().skv_plan_stats(self.ptr, ctypes.byref(tc), ctypes.byref(nf), ctypes.byref(nb),
+                                                      ctypes.byref(im)))
+        return {"total_cost": tc.value, "n_fwd_units": nf.value, "n_bwd_units": nb.value, "imbalance": im.value}
+
+
+def skv_plan(prob, policy: int = SKV_PLAN_LPT, sizes: Optional[PlanSizes] = None, buf: Optional[np.ndarray] = None) -> Plan:
+    args = _ProblemArgs(prob)
+    if sizes is None:
+        sizes = skv_plan_size(prob, policy)
+    if buf is None or buf.nbytes < sizes.plan_bytes:
+        buf = np.empty(sizes.plan_bytes, dtype=np.uint8)
+    loads = np.zeros(prob.num_partitions, dtype=np.int64)
+    _check("skv_plan", lib().skv_plan(args.ref(), policy, ctypes.c_void_p(buf.ctypes.data), buf.nbytes,
+                                      ctypes.c_void_p(loads.ctypes.data)))
+    return Plan(buf, loads, sizes, policy, prob)
+
+
+def alloc_workspace(plan: Plan, device="cuda"):
+    import torch
+    return torch.empty(plan.sizes.ws_bytes, dtype=torch.uint8, device=device)
+
+
+def skv_attn_fwd(plan: Plan, q, k, v, ws, stream=None):
+    _check("skv_attn_fwd", lib().skv_attn_fwd(plan.ptr, _ptr(q), _ptr(k), _ptr(v), _ptr(ws), ws.numel(),
+                                              _stream_ptr(stream)))
+
+
+def skv_lse_merge(plan: Plan, ws, o, lse, stream=None):
+    _check("skv_lse_merge", lib().skv_lse_merge(plan.ptr, _ptr(ws), _ptr(o), _ptr(lse), _stream_ptr(stream)))
+
+
+def skv_attn_bwd(plan: Plan, q, k, v, o, lse, do, dq, dk, dv, ws, stream=None):
+    _check("skv_attn_bwd", lib().skv_attn_bwd(plan.ptr, _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(do),
+                                              _ptr(dq), _ptr(dk), _ptr(dv), _ptr(ws), ws.numel(),
+                                              _stream_ptr(stream)))
+
+
+def skv_status(ws, stream=None) -> int:
+    return lib().skv_status(_ptr(ws), _stream_ptr(stream))
+
+
+def skv_set_unit_timer(fwd_stamps=None, bwd_stamps=None):
+    _check("skv_set_unit_timer", lib().skv_set_unit_timer(_ptr(fwd_stamps), _ptr(bwd_stamps)))
+
+
+# ------------------------------------------------------------- conveniences
+def check_inputs(plan: Plan, q, k, v, do=None):
+    import torch
+    p = plan.problem
+    Nq, L = p.num_tokens_q, p.num_tokens_kv
+    for name, t, shape in (("q", q, (Nq, p.num_q_heads, p.head_dim)), ("k", k, (L, p.num_kv_heads, p.head_dim)),
+                           ("v", v, (L, p.num_kv_heads, p.head_dim))) + ((("do", do, (Nq, p.num_q_heads, p.head_dim)),)
+                                                                          if do is not None else ()):
+        if tuple(t.shape) != shape or t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"{name}: expected contiguous cuda bf16 {shape}, got {tuple(t.shape)} {t.dtype} {t.device}")
+
+
+def forward(plan: Plan, q, k, v, ws=None, stream=None):
+    """Split-KV forward + LSE merge. Returns (o bf16 [Nq,Hq,d], lse fp32 [Nq,Hq])."""
+    import torch
+    check_inputs(plan, q, k, v)
+    if ws is None:
+        ws = alloc_workspace(plan, q.device)
+    p = plan.problem
+    o = torch.empty(p.num_tokens_q, p.num_q_heads, p.head_dim, dtype=torch.bfloat16, device=q.device)
+    lse = torch.empty(p.num_tokens_q, p.num_q_heads, dtype=torch.float32, device=q.device)
+    skv_attn_fwd(plan, q, k, v, ws, stream)
+    skv_lse_merge(plan, ws, o, lse, stream)
+    return o, lse
+
+
+def backward(plan: Plan, q, k, v, o, lse, do, ws=None, stream=None):
+    """Split-KV backward. Returns (dq, dk, dv) bf16."""
+    import torch
+    check_inputs(plan, q, k, v, do)
+    if ws is None:
+        ws = alloc_workspace(plan, q.device)
+    dq = torch.empty_like(q)
+    dk = torch.empty_like(k)
+    dv = torch.empty_like(v)
+    skv_attn_bwd(plan, q, k, v, o, lse, do, dq, dk, dv, ws, stream)
+    return dq, dk, dv

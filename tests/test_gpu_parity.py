@@ -1,0 +1,142 @@
+"""CUDA path (through the C ABI) against the fp64 oracle, element by element.
+
+Tolerances (bf16 inputs, fp32 accumulation): forward output max-abs <= 2e-2,
+LSE max-abs <= 1e-3, gradients relative Frobenius <= 1e-2 per tensor.
+Heads are independent, so where the oracle would be slow it runs on a subset
+of kv-head groups (exact for those heads).
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import attention as A
+from split_kv_block_b200 import skv, synth
+
+pytestmark = pytest.mark.gpu
+
+O_TOL, LSE_TOL, GRAD_TOL = 2e-2, 1e-3, 1e-2
+
+
+def _dev(*ts):
+    return [t.cuda() if t is not None else None for t in ts]
+
+
+def _heads_subset(prob, groups):
+    G = prob.num_q_heads // prob.num_kv_heads
+    qh = [g * G + i for g in groups for i in range(G)]
+    return qh, list(groups), prob.replace(num_q_heads=len(qh), num_kv_heads=len(groups))
+
+
+def _rel_fro(a, b):
+    a, b = a.double(), b.double()
+    return float((a - b).norm() / b.norm().clamp_min(1e-30))
+
+
+def run_gpu(prob, q, k, v, do=None, policy=skv.SKV_PLAN_LPT):
+    plan = skv.skv_plan(prob, policy)
+    qd, kd, vd, dod = _dev(q, k, v, do)
+    ws = skv.alloc_workspace(plan)
+    o, lse = skv.forward(plan, qd, kd, vd, ws)
+    assert skv.skv_status(ws) == 0
+    grads = None
+    if do is not None:
+        grads = skv.backward(plan, qd, kd, vd, o, lse, dod, ws)
+        assert skv.skv_status(ws) == 0
+    torch.cuda.synchronize()
+    return o.cpu(), lse.cpu(), (None if grads is None else [g.cpu() for g in grads]), plan
+
+
+def check_forward(prob, q, k, v, o, lse, groups=None):
+    if groups is not None:
+        qh, kh, sub = _heads_subset(prob, groups)
+        q, k, v = q[:, qh].contiguous(), k[:, kh].contiguous(), v[:, kh].contiguous()
+        o, lse, prob = o[:, qh], lse[:, qh], sub
+    O_ref, L_ref = A.attention_forward(prob, q, k, v)
+    err_o = float((o.double() - O_ref).abs().max()) if o.numel() else 0.0
+    err_l = float((lse.double() - L_ref).abs().max()) if lse.numel() else 0.0
+    assert err_o <= O_TOL, f"O max-abs {err_o}"
+    assert err_l <= LSE_TOL, f"LSE max-abs {err_l}"
+    return O_ref, L_ref, err_o, err_l
+
+
+def check_backward(prob, q, k, v, do, grads, groups=None):
+    dq, dk, dv = grads
+    if groups is not None:
+        qh, kh, sub = _heads_subset(prob, groups)
+        q, k, v, do = q[:, qh].contiguous(), k[:, kh].contiguous(), v[:, kh].contiguous(), do[:, qh].contiguous()
+        dq, dk, dv, prob = dq[:, qh], dk[:, kh], dv[:, kh], sub
+    O_ref, L_ref = A.attention_forward(prob, q, k, v)
+    rq, rk, rv = A.attention_backward(prob, q, k, v, O_ref, L_ref, do)
+    errs = (_rel_fro(dq, rq), _rel_fro(dk, rk), _rel_fro(dv, rv))
+    assert max(errs) <= GRAD_TOL, f"rel fro dq/dk/dv {errs}"
+    # keys no query sees: exactly zero
+    for b in range(prob.num_samples):
+        j0, j1 = int(prob.anchor_offsets[b]), int(prob.anchor_offsets[b + 1])
+        amax = int(prob.anchors[j0:j1].max()) if j1 > j0 else 0
+        k0, k1 = int(prob.ctx_offsets[b]), int(prob.ctx_offsets[b + 1])
+        assert torch.all(dk[k0 + amax:k1] == 0) and torch.all(dv[k0 + amax:k1] == 0)
+    return errs
+
+
+def _case(prob, seed=0, backward=True, policy=skv.SKV_PLAN_LPT, groups=None):
+    q, k, v, do = synth.make_tensors(prob, seed=seed, backward=backward)
+    o, lse, grads, plan = run_gpu(prob, q, k, v, do, policy)
+    check_forward(prob, q, k, v, o, lse, groups)
+    if backward:
+        check_backward(prob, q, k, v, do, grads, groups)
+    return plan
+
+
+def test_tiny_4k_forward_and_backward():
+    prob = synth.make_problem(synth.WORKLOADS["tiny_4k"], seed=0)
+    _case(prob)
+
+
+def test_tiny_4k_static_plan():
+    prob = synth.make_problem(synth.WORKLOADS["tiny_4k"], seed=1)
+    _case(prob, seed=1, policy=skv.SKV_PLAN_STATIC)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_random_ragged_problems(d):
+    rng = np.random.default_rng(100 + d)
+    for i in range(6):
+        prob = synth.random_small_problem(rng, max_len=900, max_anchors=7, d=d,
+                                          heads=((4, 1), (8, 2), (4, 4), (8, 1), (16, 2), (2, 2)))
+        _case(prob, seed=i, policy=skv.SKV_PLAN_LPT if i % 3 else skv.SKV_PLAN_STATIC)
+
+
+def test_edge_anchors():
+    """a = 1, a = L, duplicates, unsorted anchors, block_q = 1."""
+    prob = synth.small_problem([517, 260], [[1, 517, 517, 3, 200], [260, 1, 129]], block_q=1, chunk_kv=128,
+                               sub_chunks=2, num_partitions=5, hq=8, hkv=2, d=128)
+    _case(prob)
+
+
+def test_partitions_exceed_items_and_single_partition():
+    prob = synth.small_problem([300], [[299, 10, 150]], block_q=16, chunk_kv=256, num_partitions=32, hq=4, hkv=1,
+                               d=64)
+    _case(prob)
+    _case(prob.replace(num_partitions=1))
+
+
+def test_sample_without_anchors():
+    prob = synth.small_problem([400, 333, 128], [[390], [], [128, 5]], block_q=16, chunk_kv=128, num_partitions=3,
+                               hq=4, hkv=1, d=64)
+    _case(prob)
+
+
+def test_ragged_tiles_many_samples():
+    """Odd anchor counts (query tiles half empty), chunk not a multiple of the
+    key tile, context lengths not multiples of anything."""
+    prob = synth.small_problem([1001, 777, 1500], [[1000, 3, 555], [777], [1, 1499, 700, 64, 1200]], block_q=16,
+                               chunk_kv=320, num_partitions=4, hq=8, hkv=2, d=128)
+    _case(prob, seed=3)
+
+
+def test_ctx32k_two_groups():
+    """The 32K workload at full size; oracle on 2 of the 8 kv-head groups."""
+    prob = synth.make_problem(synth.WORKLOADS["ctx32k"], seed=0)
+    _case(prob, groups=(0, 5))

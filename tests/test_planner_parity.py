@@ -1,0 +1,118 @@
+"""The C++ planner (skv_plan through the C ABI) against the planner oracle:
+items, realized costs, partitions and partition loads must be bit-exact
+("Split-KV: Breaking the Context Parallelism Bottleneck ...", section "LPT
+Scheduling"). Host-only: runs without a GPU."""
+import numpy as np
+import pytest
+
+from oracle import planner as PL
+from split_kv_block_b200 import skv, synth
+
+
+def _compare(prob, policy):
+    plan = skv.skv_plan(prob, policy)
+    got = plan.items()
+    if policy == skv.SKV_PLAN_LPT:
+        ref, loads = PL.lpt_plan(prob)
+    else:
+        ref, loads = PL.static_plan(prob)
+    assert len(got) == len(ref)
+    mine = [(int(r["b"]), int(r["c"]), int(r["g"]), int(r["sub"]), int(r["key_begin"]), int(r["key_end"]),
+             int(r["cost"]), int(r["partition"])) for r in got]
+    theirs = [(it.b, it.c, it.g, it.sub, it.key_begin, it.key_end, it.cost, it.partition) for it in ref]
+    assert mine == theirs
+    assert plan.partition_load.tolist() == loads
+    st = plan.stats()
+    assert st["total_cost"] == sum(loads)
+    assert st["imbalance"] == pytest.approx(PL.imbalance(loads), abs=1e-12)
+    return plan
+
+
+@pytest.mark.parametrize("name", sorted(synth.WORKLOADS))
+@pytest.mark.parametrize("policy", [skv.SKV_PLAN_LPT, skv.SKV_PLAN_STATIC])
+def test_workloads_bit_exact(name, policy):
+    for seed in range(3):
+        prob = synth.make_problem(synth.WORKLOADS[name], seed=seed)
+        _compare(prob, policy)
+
+
+def test_ctx128k_subchunks_bit_exact():
+    prob = synth.make_problem(synth.WORKLOADS["ctx128k"], seed=0, sub_chunks=4)
+    _compare(prob, skv.SKV_PLAN_LPT)
+
+
+def test_random_small_problems_bit_exact():
+    rng = np.random.default_rng(2024)
+    for i in range(1000):
+        prob = synth.random_small_problem(rng)
+        _compare(prob, skv.SKV_PLAN_LPT if i % 2 == 0 else skv.SKV_PLAN_STATIC)
+
+
+def test_more_partitions_than_items():
+    prob = synth.small_problem([100], [[50]], chunk_kv=64, num_partitions=9, hq=2, hkv=1)
+    plan = _compare(prob, skv.SKV_PLAN_LPT)
+    parts = sorted(int(x) for x in plan.items()["partition"])
+    assert parts == [0, 1]
+
+
+def test_single_partition():
+    prob = synth.small_problem([300, 70], [[300, 2], [5]], chunk_kv=64, num_partitions=1)
+    plan = _compare(prob, skv.SKV_PLAN_LPT)
+    assert plan.stats()["imbalance"] == 0.0
+
+
+def test_zero_anchor_sample():
+    prob = synth.small_problem([200, 90], [[150], []], chunk_kv=64, num_partitions=3)
+    _compare(prob, skv.SKV_PLAN_LPT)
+    _compare(prob, skv.SKV_PLAN_STATIC)
+
+
+def _status(prob, policy=skv.SKV_PLAN_LPT):
+    try:
+        skv.skv_plan_size(prob, policy)
+        return 0
+    except skv.SkvError as e:
+        return e.code
+
+
+def test_invalid_arguments_rejected():
+    ok = synth.small_problem([100], [[50]])
+    assert _status(ok) == 0
+    assert _status(ok.replace(anchors=np.array([0]))) == 1            # a < 1
+    assert _status(ok.replace(anchors=np.array([101]))) == 1          # a > L
+    assert _status(ok.replace(num_kv_heads=3)) == 1                   # Hq % Hkv
+    assert _status(ok.replace(chunk_kv=100, sub_chunks=3)) == 1       # C % sub
+    assert _status(ok.replace(num_partitions=0)) == 1
+    assert _status(ok.replace(block_q=0)) == 1
+    assert _status(ok, policy=7) == 1
+    assert _status(ok.replace(ctx_offsets=np.array([0, 0]), anchors=np.zeros(0, np.int64),
+                              anchor_offsets=np.array([0, 0], np.int32))) == 1   # empty sample
+    assert _status(ok.replace(head_dim=96)) == 3                      # unsupported d
+    assert _status(ok.replace(num_q_heads=24, num_kv_heads=1)) == 3   # group of 24 rows does not tile 128
+
+
+def test_plan_buffer_too_small():
+    prob = synth.small_problem([100], [[50]])
+    sizes = skv.skv_plan_size(prob)
+    small = np.empty(sizes.plan_bytes - 1, dtype=np.uint8)
+    with pytest.raises(skv.SkvError) as e:
+        skv.skv_plan(prob, sizes=skv.PlanSizes(sizes.n_items, sizes.plan_bytes - 1, 0, 0), buf=small)
+    assert e.value.code == 2
+
+
+def test_plan_is_deterministic():
+    prob = synth.make_problem(synth.WORKLOADS["batch8_logu"], seed=1)
+    a = skv.skv_plan(prob)
+    b = skv.skv_plan(prob)
+    assert a.buf.tobytes() == b.buf.tobytes()
+
+
+def test_library_exports_every_declared_symbol():
+    import os
+    import re
+    hdr = open(os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "skv.h")).read()
+    declared = set(re.findall(r"^\s*(?:const\s+)?[a-z_0-9]+\s*\*?\s*(skv_[a-z_0-9]+)\s*\(", hdr, re.M))
+    assert declared == set(skv.EXPORTS)
+    L = skv.lib()
+    for name in declared:
+        assert hasattr(L, name), name
