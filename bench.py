@@ -1,0 +1,496 @@
+"""Benchmark of the split-KV hot path on B200.
+
+One step = one pass of the whole path over one batch of synthetic input:
+host planning (realized cost + LPT, skv_plan), split-KV forward, LSE merge,
+backward (preprocess, main kernel, dQ cast). Default workload: the 32K
+context fwd+bwd problem (1 sample, 32768-token context, 32 anchors x 16 draft
+tokens, 32 q / 8 kv heads, d = 128, KV chunk 2048, 16 partitions).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+    python bench.py --impl reference ...     # the CPU fp64 oracle, timed on host cores
+
+Prints one JSON line (rank 0). Multi-GPU (torchrun): every rank runs its own
+independent problem (seed + rank); no data-path collective; value is the
+whole-job throughput over the max-over-ranks device time.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from split_kv_block_b200 import synth  # noqa: E402
+
+WORKLOAD_TEXT = {
+    "tiny_4k": "1 sample, 4096-token context, 4 anchors x 16 draft tokens, 8/2 heads, d=64, KV chunk 512, 4 partitions",
+    "ctx32k_fwd": "1 sample, 32768-token context, 32 anchors x 16 draft tokens, 32/8 heads, d=128, KV chunk 2048, "
+                  "16 partitions, forward + LSE merge",
+    "ctx32k": "1 sample, 32768-token context, 32 anchors x 16 draft tokens, 32/8 heads, d=128, KV chunk 2048, "
+              "16 partitions, fwd+bwd",
+    "ctx128k": "1 sample, 131072-token context, 64 Beta(5,1) anchors x 16 draft tokens, 32/8 heads, d=128, "
+               "KV chunk 4096, 64 partitions, fwd+bwd",
+    "batch8_logu": "8 samples, contexts log-uniform in [8192, 262144], 128 anchors x 16 draft tokens each, 32/8 heads, "
+                   "d=128, KV chunk 4096, 128 partitions, fwd+bwd, anchors redrawn and replanned every step",
+}
+METRIC = "split-KV attn fwd+bwd effective TFLOP/s"
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": p["hbm_gbs"], "bf16_tflops": p["bf16_tflops"],
+                "bf16_tflops_sustained": p.get("bf16_tflops_sustained"), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def flops_of(prob, backward=True):
+    """Unmasked work: 4 d block_q Hq sum(a) forward, 2.5x that backward."""
+    f_fwd = 4.0 * prob.head_dim * prob.block_q * prob.num_q_heads * float(np.sum(prob.anchors))
+    return f_fwd, (2.5 * f_fwd if backward else 0.0)
+
+
+def bwd_bytes(prob):
+    """Algorithmic HBM bytes of the backward attention kernel: Q, dO, LSE, D
+    read once, K/V of the attended prefix read once, dK/dV of that prefix
+    written once, dQ accumulated once (fp32 read + write)."""
+    Nq, Hq, Hkv, d = prob.num_tokens_q, prob.num_q_heads, prob.num_kv_heads, prob.head_dim
+    keys = 0
+    for b in range(prob.num_samples):
+        j0, j1 = int(prob.anchor_offsets[b]), int(prob.anchor_offsets[b + 1])
+        if j1 > j0:
+            keys += int(prob.anchors[j0:j1].max())
+    return 2 * Nq * Hq * d * 2 + 2 * Nq * Hq * 4 + 4 * keys * Hkv * d * 2 + 2 * Nq * Hq * d * 4
+
+
+KERNEL_SOURCES = {"fwd_kernel": ["fwd.cu", "sm100.cuh", "kernels.h", "plan_layout.h"],
+                  "bwd_kernel": ["bwd.cu", "sm100.cuh", "kernels.h", "plan_layout.h"],
+                  "merge_kernel": ["merge.cu", "sm100.cuh", "kernels.h", "plan_layout.h"]}
+
+
+def kernel_digest(kernel):
+    import hashlib
+    h = hashlib.sha256()
+    for name in KERNEL_SOURCES[kernel]:
+        with open(os.path.join(ROOT, "split_kv_block_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(kernel, workload):
+    """DRAM bytes (read + write) per launch from the committed ncu summary,
+    or None when the kernel's sources changed since that capture."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f).get(kernel, {}).get(workload)
+    except (OSError, ValueError):
+        return None
+    if not rec or rec.get("source_digest") != kernel_digest(kernel):
+        return None
+    return rec.get("dram_bytes_per_launch")
+
+
+# ----------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "50"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            time.sleep(0.3)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.rows = []
+        if self.proc is None:
+            return False
+        time.sleep(0.1)
+        self.proc.terminate()
+        out, _ = self.proc.communicate(timeout=10)
+        for line in out.strip().splitlines():
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) == 7:
+                self.rows.append(parts)
+        return False
+
+    def summary(self):
+        if not getattr(self, "rows", None):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+        sm = [num(r[0]) for r in self.rows if num(r[0]) is not None]
+        mx = [num(r[1]) for r in self.rows if num(r[1]) is not None]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in self.rows for i in range(4) if r[3 + i].lower() == "active"})
+        loaded = [s for s in sm if s >= 0.5 * max(sm)] if sm else []
+        return {"sm_mhz": statistics.median(loaded) if loaded else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(self.rows)}
+
+
+# ------------------------------------------------------------- GPU arm
+def run_gpu(args, rank, world, local_rank):
+    from split_kv_block_b200 import skv
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    w = synth.WORKLOADS[args.workload]
+    seed = args.seed + rank
+    prob = synth.make_problem(w, seed=seed, sub_chunks=args.sub_chunks)
+    backward = w.backward
+    q, k, v, do = synth.make_tensors(prob, seed=seed, backward=backward)
+    q, k, v = q.to(dev), k.to(dev), v.to(dev)
+    do = do.to(dev) if backward else None
+    policy = skv.SKV_PLAN_STATIC if args.policy == "static" else skv.SKV_PLAN_LPT
+    redraw = args.workload == "batch8_logu"
+
+    # anchors of every step (the batched workload redraws them each step)
+    step_probs = [synth.redraw_anchors(prob, w, seed * 1000 + i) if redraw else prob
+                  for i in range(args.warmup + args.steps)]
+    sizes = [skv.skv_plan_size(p, policy) for p in step_probs]
+    ws_bytes = max(s.ws_bytes for s in sizes)
+    plan_bytes = max(s.plan_bytes for s in sizes)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    plan_buf = np.empty(plan_bytes, dtype=np.uint8)
+    Nq, Hq, d = prob.num_tokens_q, prob.num_q_heads, prob.head_dim
+    o = torch.empty(Nq, Hq, d, dtype=torch.bfloat16, device=dev)
+    lse = torch.empty(Nq, Hq, dtype=torch.float32, device=dev)
+    if backward:
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)  # > 126 MB L2
+    stream = torch.cuda.current_stream()
+
+    planner_s = []
+
+    def step(i):
+        p = step_probs[i]
+        t0 = time.perf_counter()
+        plan = skv.skv_plan(p, policy, sizes=sizes[i], buf=plan_buf)
+        planner_s.append(time.perf_counter() - t0)
+        skv.skv_attn_fwd(plan, q, k, v, ws, stream)
+        skv.skv_lse_merge(plan, ws, o, lse, stream)
+        if backward:
+            skv.skv_attn_bwd(plan, q, k, v, o, lse, do, dq, dk, dv, ws, stream)
+        return plan
+
+    def mk_event():
+        e = torch.cuda.Event(enable_timing=True)
+        e.record(stream)
+        return e
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    assert skv.skv_status(ws) == 0, "device status error during warm-up"
+    planner_s.clear()
+
+    K = args.steps
+    ev = [(mk_event(), mk_event()) for _ in range(K)]
+    kev = {kid: [(mk_event(), mk_event()) for _ in range(K)] for kid in (skv.SKV_KERNEL_FWD, skv.SKV_KERNEL_MERGE,
+                                                                          skv.SKV_KERNEL_BWD)}
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local_rank) as clocks:
+        for i in range(K):
+            flush.zero_()  # evict L2 between steps (outside the step's event window)
+            for kid, lst in kev.items():
+                skv.skv_set_timing_events(kid, lst[i][0], lst[i][1])
+            ev[i][0].record(stream)
+            step(args.warmup + i)
+            ev[i][1].record(stream)
+        torch.cuda.synchronize()
+    for kid in kev:
+        skv.skv_set_timing_events(kid, None, None)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    status = skv.skv_status(ws)
+    if status != 0:
+        raise RuntimeError(f"device status {status} after the timed steps")
+    t_steps = [a.elapsed_time(b) / 1e3 for a, b in ev]
+    t_kern = {kid: [a.elapsed_time(b) / 1e3 for a, b in lst] for kid, lst in kev.items()}
+    total = sum(t_steps)
+    if world > 1:
+        tt = torch.tensor([total], dtype=torch.float64, device=dev)
+        torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
+        total = float(tt.item())
+
+    f_fwd_all, f_bwd_all = 0.0, 0.0
+    for i in range(K):
+        a, b = flops_of(step_probs[args.warmup + i], backward)
+        f_fwd_all += a
+        f_bwd_all += b
+    flops_rank = f_fwd_all + f_bwd_all
+    flops_job = flops_rank * world
+    value = flops_job / total / 1e12
+    ctx_tokens = float(prob.num_tokens_kv) * K * world
+
+    # plan quality (LPT vs static) on this step's problem
+    p0 = step_probs[args.warmup]
+    lpt = skv.skv_plan(p0, skv.SKV_PLAN_LPT).stats()["imbalance"]
+    static = skv.skv_plan(p0, skv.SKV_PLAN_STATIC).stats()["imbalance"]
+
+    peaks = load_peaks()
+    dom = skv.SKV_KERNEL_BWD if backward else skv.SKV_KERNEL_FWD
+    dom_t = statistics.mean(t_kern[dom])
+    dom_flops = (f_bwd_all if backward else f_fwd_all) / K
+    achieved = dom_flops / dom_t / 1e12
+    roof_step = max(flops_rank / K / (peaks["bf16_tflops"] * 1e12), 0.0)
+    kernels_per_step = 2 + (3 if backward else 0)
+
+    out = {
+        "metric": METRIC, "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": round(total / K * 1e3, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": f"{args.workload}: {WORKLOAD_TEXT[args.workload]}", "seed": args.seed,
+                   "policy": args.policy, "sub_chunks": prob.sub_chunks,
+                   "l2": "flushed before every step (256 MiB write outside the step's event window)",
+                   "parallelism": f"replicas x{world}" if world > 1 else "1 GPU, P virtual partitions"},
+        "roofline": {"bound": "tensor", "kernel": "bwd_kernel" if backward else "fwd_kernel",
+                     "achieved": round(achieved, 2), "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                     "frac": round(achieved / peaks["bf16_tflops"], 4),
+                     "traffic": profiled_traffic("bwd_kernel" if backward else "fwd_kernel", args.workload),
+                     "peak_source": f"{peaks['source']} bf16 dense (burst)",
+                     "step_frac": round(roof_step / (total / K), 4)},
+        "kernel_ms": {"fwd": round(statistics.mean(t_kern[skv.SKV_KERNEL_FWD]) * 1e3, 4),
+                      "merge": round(statistics.mean(t_kern[skv.SKV_KERNEL_MERGE]) * 1e3, 4),
+                      "bwd": round(statistics.mean(t_kern[skv.SKV_KERNEL_BWD]) * 1e3, 4) if backward else None},
+        "context_tokens_per_s": round(ctx_tokens / total, 1),
+        "imbalance": {"lpt": lpt, "static": static},
+        "planner_us": round(statistics.median(planner_s) * 1e6, 1),
+        "gpu_launches": kernels_per_step * K,
+        "clocks": clocks.summary(),
+    }
+    if not args.no_e2e:
+        out["e2e"] = run_e2e(args, prob, step_probs, sizes, policy, q, k, v, do, dev, world)
+    return out, prob
+
+
+def run_e2e(args, prob, step_probs, sizes, policy, q, k, v, do, dev, world):
+    """Same metric through the public API from pinned host buffers: every step
+    copies the inputs host->device, runs the path and reads all outputs back."""
+    from split_kv_block_b200 import skv
+    backward = do is not None
+    hq, hk, hv = q.cpu().pin_memory(), k.cpu().pin_memory(), v.cpu().pin_memory()
+    hdo = do.cpu().pin_memory() if backward else None
+    qd, kd, vd = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    dod = torch.empty_like(do) if backward else None
+    ws = torch.empty(max(s.ws_bytes for s in sizes), dtype=torch.uint8, device=dev)
+    Nq, Hq, d = prob.num_tokens_q, prob.num_q_heads, prob.head_dim
+    o = torch.empty(Nq, Hq, d, dtype=torch.bfloat16, device=dev)
+    lse = torch.empty(Nq, Hq, dtype=torch.float32, device=dev)
+    ho, hl = torch.empty(o.shape, dtype=o.dtype).pin_memory(), torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+    if backward:
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        hdq, hdk, hdv = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in (dq, dk, dv)]
+    stream = torch.cuda.current_stream()
+    n = min(args.steps, args.e2e_steps)
+    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv) + ((hdo,) if backward else ()))
+    d2h = o.numel() * 2 + lse.numel() * 4 + (sum(t.numel() * 2 for t in (dq, dk, dv)) if backward else 0)
+    times, flops = [], 0.0
+    for i in range(args.warmup + n):
+        p = step_probs[i % len(step_probs)]
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        qd.copy_(hq, non_blocking=True)
+        kd.copy_(hk, non_blocking=True)
+        vd.copy_(hv, non_blocking=True)
+        if backward:
+            dod.copy_(hdo, non_blocking=True)
+        plan = skv.skv_plan(p, policy, sizes=sizes[i % len(sizes)])
+        skv.skv_attn_fwd(plan, qd, kd, vd, ws, stream)
+        skv.skv_lse_merge(plan, ws, o, lse, stream)
+        ho.copy_(o, non_blocking=True)
+        hl.copy_(lse, non_blocking=True)
+        if backward:
+            skv.skv_attn_bwd(plan, qd, kd, vd, o, lse, dod, dq, dk, dv, ws, stream)
+            hdq.copy_(dq, non_blocking=True)
+            hdk.copy_(dk, non_blocking=True)
+            hdv.copy_(dv, non_blocking=True)
+        b.record(stream)
+        b.synchronize()
+        if i >= args.warmup:
+            times.append(a.elapsed_time(b) / 1e3)
+            ff, fb = flops_of(p, backward)
+            flops += ff + fb
+    total = sum(times)
+    if world > 1:
+        tt = torch.tensor([total], dtype=torch.float64, device=dev)
+        torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
+        total = float(tt.item())
+    return {"value": round(flops * world / total / 1e12, 4), "unit": "TFLOP/s", "h2d_bytes_per_step": int(h2d),
+            "d2h_bytes_per_step": int(d2h), "steps": n, "ms_per_step": round(total / n * 1e3, 3)}
+
+
+# ------------------------------------------------------------- CPU oracle
+def oracle_sample(prob, groups, anchor_stride):
+    """Sub-problem: the kv-head groups `groups` and every `anchor_stride`-th
+    anchor of each sample (exact for those rows and heads: rows and heads are
+    independent)."""
+    G = prob.num_q_heads // prob.num_kv_heads
+    qh = [g * G + i for g in groups for i in range(G)]
+    keep = []
+    aoff = [0]
+    for b in range(prob.num_samples):
+        j = list(range(int(prob.anchor_offsets[b]), int(prob.anchor_offsets[b + 1])))[::anchor_stride]
+        keep += j
+        aoff.append(aoff[-1] + len(j))
+    sub = prob.replace(num_q_heads=len(qh), num_kv_heads=len(groups), anchors=prob.anchors[keep],
+                       anchor_offsets=np.array(aoff, dtype=np.int32))
+    return sub, qh, keep
+
+
+def time_oracle(prob, q, k, v, do, groups, anchor_stride):
+    from oracle import attention as A
+    sub, qh, keep = oracle_sample(prob, groups, anchor_stride)
+    S = prob.block_q
+    rows = np.concatenate([np.arange(j * S, (j + 1) * S) for j in keep]) if keep else np.zeros(0, dtype=np.int64)
+    rows_t = torch.from_numpy(rows)
+    qs = q[rows_t][:, qh].contiguous()
+    ks, vs = k[:, list(groups)].contiguous(), v[:, list(groups)].contiguous()
+    t0 = time.perf_counter()
+    O, L = A.attention_forward(sub, qs, ks, vs)
+    if do is not None:
+        dos = do[rows_t][:, qh].contiguous()
+        A.attention_backward(sub, qs, ks, vs, O, L, dos)
+    dt = time.perf_counter() - t0
+    ff, fb = flops_of(sub, do is not None)
+    return (ff + fb), dt, sub
+
+
+def cpu_baseline(prob, backward, seed):
+    q, k, v, do = synth.make_tensors(prob, seed=seed, backward=backward)
+    threads = os.cpu_count() or 1
+    torch.set_num_threads(threads)
+    # calibrate on one kv-head group and every 8th anchor, then take as many
+    # groups / anchors as make ~15 s of CPU work (heads and rows are independent)
+    f, dt, sub = time_oracle(prob, q, k, v, do if backward else None, (0,), 8)
+    per_group_all = dt * 8
+    n_groups = max(1, min(prob.num_kv_heads, int(15.0 / max(per_group_all, 1e-3))))
+    stride = 1 if per_group_all <= 15.0 else int(math.ceil(per_group_all / 15.0))
+    groups = tuple(range(n_groups))
+    f, dt, sub = time_oracle(prob, q, k, v, do if backward else None, groups, stride)
+    return {"value": round(f / dt / 1e12, 6), "unit": "TFLOP/s", "cores": torch.get_num_threads(), "kind": "oracle",
+            "sample": f"fp64 oracle fwd{'+bwd' if backward else ''} on {n_groups} of {prob.num_kv_heads} kv-head "
+                      f"groups, every {stride}th anchor ({int(sub.anchor_offsets[-1])} anchors), {dt:.1f} s",
+            "cpu": _cpu_name()}
+
+
+def _cpu_name():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+def run_reference(args):
+    """The oracle as the reference arm: every step a bounded sample of the workload."""
+    w = synth.WORKLOADS[args.workload]
+    prob = synth.make_problem(w, seed=args.seed, sub_chunks=args.sub_chunks)
+    backward = w.backward
+    q, k, v, do = synth.make_tensors(prob, seed=args.seed, backward=backward)
+    torch.set_num_threads(os.cpu_count() or 1)
+    n_anchor = int(prob.anchor_offsets[-1])
+    # calibrate: one group, a thin anchor sample
+    f, dt, _ = time_oracle(prob, q, k, v, do if backward else None, (0,), max(1, n_anchor // 2))
+    budget = min(5.0, 150.0 / max(1, args.steps + args.warmup))
+    per_anchor = dt / max(1, len(range(0, n_anchor, max(1, n_anchor // 2))))
+    n_take = max(1, min(n_anchor, int(budget / max(per_anchor, 1e-6))))
+    stride = max(1, n_anchor // n_take)
+    times, flops = [], 0.0
+    for i in range(args.warmup + args.steps):
+        g = i % prob.num_kv_heads
+        f, dt, sub = time_oracle(prob, q, k, v, do if backward else None, (g,), stride)
+        if i >= args.warmup:
+            times.append(dt)
+            flops += f
+    total = sum(times)
+    value = flops / total / 1e12
+    sample = (f"fp64 oracle fwd{'+bwd' if backward else ''} per step on one kv-head group (rotating) and every "
+              f"{stride}th anchor of the workload")
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s", "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(total / args.steps * 1e3, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": f"{args.workload}: {WORKLOAD_TEXT[args.workload]}", "seed": args.seed,
+                   "parallelism": "CPU host cores"},
+        "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": torch.get_num_threads(),
+                         "kind": "oracle", "sample": sample, "cpu": _cpu_name()},
+        "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="skv", choices=["skv", "reference"])
+    ap.add_argument("--workload", default="ctx32k", choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--policy", default="lpt", choices=["lpt", "static"])
+    ap.add_argument("--sub-chunks", type=int, default=None)
+    ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)), flush=True)
+        return
+
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    try:
+        out, prob = run_gpu(args, rank, world, local_rank)
+        if rank == 0:
+            if world == 1 and not args.no_cpu_baseline:
+                out["cpu_baseline"] = cpu_baseline(prob, synth.WORKLOADS[args.workload].backward, args.seed)
+            print(json.dumps(out), flush=True)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

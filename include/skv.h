@@ -164,10 +164,20 @@ const char* skv_strerror(int code);
 /* Last CUDA runtime error code seen by this thread's calls (0 if none). */
 int skv_last_cuda_error(void);
 
-/* Realized per-partition busy time: if enabled (non-zero), the next kernels
- * record, per work unit, its start/end %globaltimer stamps into `stamps`
- * (device int64 [2 * n_units], caller-owned; NULL disables). */
+/* Realized per-partition busy time: while set (non-NULL), the forward /
+ * backward kernels record, per work unit u, its %globaltimer start and end
+ * (ns) into stamps[2u], stamps[2u+1] (device int64 [2 * n_units],
+ * caller-owned). NULL disables. Process-wide setting. */
 int skv_set_unit_timer(void* fwd_stamps, void* bwd_stamps);
+
+enum skv_kernel_id { SKV_KERNEL_FWD = 0, SKV_KERNEL_MERGE = 1, SKV_KERNEL_BWD = 2 };
+
+/* Kernel timing: while set, the library records the caller-created CUDA
+ * events `start` / `end` (cudaEvent_t) on the launch stream immediately
+ * before and after every launch of the given kernel (the forward attention
+ * kernel, the LSE merge kernel, or the backward attention kernel). NULL
+ * disables. Process-wide setting. */
+int skv_set_timing_events(int kernel, void* start_event, void* end_event);
 
 #ifdef __cplusplus
 }

@@ -17,6 +17,11 @@ namespace {
 thread_local int g_last_cuda = 0;
 long long* g_fwd_stamps = nullptr;
 long long* g_bwd_stamps = nullptr;
+cudaEvent_t g_ev[3][2] = {};  // per SKV_KERNEL_*: start, end
+
+cudaError_t mark(int kernel, int which, cudaStream_t stream) {
+  return g_ev[kernel][which] ? cudaEventRecord(g_ev[kernel][which], stream) : cudaSuccess;
+}
 constexpr unsigned long long kTimeoutNs = 2000000000ull;  // 2 s per device-side wait
 
 int cuda_fail(cudaError_t e) {
@@ -163,6 +168,14 @@ extern "C" int skv_set_unit_timer(void* fwd_stamps, void* bwd_stamps) {
   return SKV_OK;
 }
 
+extern "C" int skv_set_timing_events(int kernel, void* start_event, void* end_event) {
+  if (kernel < SKV_KERNEL_FWD || kernel > SKV_KERNEL_BWD) return SKV_EINVAL;
+  if ((start_event == nullptr) != (end_event == nullptr)) return SKV_EINVAL;
+  g_ev[kernel][0] = static_cast<cudaEvent_t>(start_event);
+  g_ev[kernel][1] = static_cast<cudaEvent_t>(end_event);
+  return SKV_OK;
+}
+
 extern "C" int skv_attn_fwd(const void* plan, const void* q, const void* k, const void* v, void* ws,
                             size_t ws_bytes, skv_stream_t stream_) {
   const PlanHeader* h = header_of(plan);
@@ -198,7 +211,9 @@ extern "C" int skv_attn_fwd(const void* plan, const void* q, const void* k, cons
   int sms = num_sms();
   if (sms <= 0) return cuda_fail(cudaGetLastError());
   const int grid = static_cast<int>(std::min<int64_t>(sms, h->n_fwd));
-  cudaError_t e = launch_fwd(h->d, tq, tk, tv, p, grid, stream);
+  cudaError_t e = mark(SKV_KERNEL_FWD, 0, stream);
+  if (e == cudaSuccess) e = launch_fwd(h->d, tq, tk, tv, p, grid, stream);
+  if (e == cudaSuccess) e = mark(SKV_KERNEL_FWD, 1, stream);
   if (e != cudaSuccess) return cuda_fail(e);
   return SKV_OK;
 }
@@ -221,7 +236,10 @@ extern "C" int skv_lse_merge(const void* plan, const void* ws, void* o, float* l
   p.Hkv = h->Hkv;
   p.G = h->G;
   p.Hq = h->Hq;
-  cudaError_t e = launch_merge(h->d, p, reinterpret_cast<cudaStream_t>(stream_));
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  cudaError_t e = mark(SKV_KERNEL_MERGE, 0, stream);
+  if (e == cudaSuccess) e = launch_merge(h->d, p, stream);
+  if (e == cudaSuccess) e = mark(SKV_KERNEL_MERGE, 1, stream);
   if (e != cudaSuccess) return cuda_fail(e);
   return SKV_OK;
 }
@@ -288,7 +306,9 @@ extern "C" int skv_attn_bwd(const void* plan, const void* q, const void* k, cons
     int sms = num_sms();
     if (sms <= 0) return cuda_fail(cudaGetLastError());
     const int grid = static_cast<int>(std::min<int64_t>(sms, h->n_bwd));
-    e = launch_bwd(h->d, tq, tk, tv, tdo, p, grid, stream);
+    e = mark(SKV_KERNEL_BWD, 0, stream);
+    if (e == cudaSuccess) e = launch_bwd(h->d, tq, tk, tv, tdo, p, grid, stream);
+    if (e == cudaSuccess) e = mark(SKV_KERNEL_BWD, 1, stream);
     if (e != cudaSuccess) return cuda_fail(e);
   }
   e = launch_dq_cast(dq_acc, static_cast<__nv_bfloat16*>(dq),

@@ -22,7 +22,9 @@ SKV_PLAN_STATIC = 1
 
 # Every function include/skv.h declares.
 EXPORTS = ("skv_plan_size", "skv_plan", "skv_plan_items", "skv_plan_stats", "skv_attn_fwd", "skv_lse_merge",
-           "skv_attn_bwd", "skv_status", "skv_strerror", "skv_last_cuda_error", "skv_set_unit_timer")
+           "skv_attn_bwd", "skv_status", "skv_strerror", "skv_last_cuda_error", "skv_set_unit_timer",
+           "skv_set_timing_events")
+SKV_KERNEL_FWD, SKV_KERNEL_MERGE, SKV_KERNEL_BWD = 0, 1, 2
 
 
 class SkvError(RuntimeError):
@@ -64,6 +66,7 @@ def lib() -> ctypes.CDLL:
         L.skv_strerror.argtypes = [ctypes.c_int]
         L.skv_strerror.restype = ctypes.c_char_p
         L.skv_set_unit_timer.argtypes = [vp, vp]
+        L.skv_set_timing_events.argtypes = [ctypes.c_int, vp, vp]
         for name in EXPORTS:
             if name not in ("skv_strerror",):
                 getattr(L, name).restype = ctypes.c_int
@@ -196,6 +199,13 @@ def skv_status(ws, stream=None) -> int:
 
 def skv_set_unit_timer(fwd_stamps=None, bwd_stamps=None):
     _check("skv_set_unit_timer", lib().skv_set_unit_timer(_ptr(fwd_stamps), _ptr(bwd_stamps)))
+
+
+def skv_set_timing_events(kernel: int, start=None, end=None):
+    """start/end: torch.cuda.Event (already recorded once, so the CUDA event exists) or None."""
+    h0 = ctypes.c_void_p(start.cuda_event) if start is not None else ctypes.c_void_p(0)
+    h1 = ctypes.c_void_p(end.cuda_event) if end is not None else ctypes.c_void_p(0)
+    _check("skv_set_timing_events", lib().skv_set_timing_events(kernel, h0, h1))
 
 
 # ------------------------------------------------------------- conveniences
