@@ -58,7 +58,8 @@ enum skv_status_code {
   SKV_ECUDA = 4,        /* a CUDA runtime call failed (see skv_last_cuda_error) */
   SKV_EPLAN = 5,        /* plan buffer not written by skv_plan, or for another problem */
   SKV_ETIMEOUT = 6,     /* a device-side wait gave up; results are invalid */
-  SKV_EDEVICE = 7       /* a kernel found an inconsistent work list; results are invalid */
+  SKV_EDEVICE = 7,      /* a kernel found an inconsistent work list; results are invalid */
+  SKV_ESCRATCH = 8      /* skv_attn_fwd_noalloc: workspace larger than SKV_NOALLOC_SCRATCH_BYTES */
 };
 
 enum skv_plan_policy {
@@ -178,6 +179,44 @@ enum skv_kernel_id { SKV_KERNEL_FWD = 0, SKV_KERNEL_MERGE = 1, SKV_KERNEL_BWD = 
  * kernel, the LSE merge kernel, or the backward attention kernel). NULL
  * disables. Process-wide setting. */
 int skv_set_timing_events(int kernel, void* start_event, void* end_event);
+
+/* Size of the library-owned scratch array used by skv_attn_fwd_noalloc. */
+#define SKV_NOALLOC_SCRATCH_BYTES ((size_t)32 << 20)
+
+/*
+ * skv_attn_fwd_noalloc — skv_attn_fwd followed by skv_lse_merge, for callers
+ * that cannot allocate device memory. The pages have no counterpart of this
+ * call; it is a deployment convenience of this library.
+ *
+ * Which callers: code given only input and output pointers by a host
+ * framework that owns all device memory (a plugin without an allocator of
+ * its own), and latency-critical code that must not call cudaMalloc/cudaFree
+ * because they can synchronize the device and stall other streams. Neither
+ * can provide the workspace skv_attn_fwd needs.
+ *
+ * The workspace lives instead in one file-scope device array of
+ * SKV_NOALLOC_SCRATCH_BYTES (32 MiB) per GPU, held by every GPU that loads the
+ * library until the process exits. The call allocates nothing: no
+ * cudaMalloc, cudaFree, pinned staging or library allocator. The caller
+ * passes the plan (host, from skv_plan), q, k, v (device bf16) and the outputs
+ * o (device bf16 [Nq][Hq][d]) and lse (device fp32 [Nq][Hq]), as for
+ * skv_attn_fwd + skv_lse_merge. The plan's device section is copied from
+ * `plan` with cudaMemcpyAsync: from pageable memory the copy is staged before
+ * the call returns; if `plan` is pinned, keep it unchanged until `stream`
+ * has passed this call.
+ *
+ * The first call on a device looks up the array's device address (this may
+ * load the library's device code); make it before any stream capture.
+ * Every call shares the array and it keeps the last call's contents; the
+ * call clears what must start at zero. Calls whose GPU work overlaps (other
+ * streams or threads) race on the array. Returns SKV_ESCRATCH, before
+ * enqueuing anything, when the problem's forward workspace (ws_fwd_bytes of
+ * skv_plan_size) exceeds SKV_NOALLOC_SCRATCH_BYTES. A device-side wait that
+ * gives up ends the kernels early but is not reported here; use skv_attn_fwd
+ * and skv_status when that report is needed.
+ */
+int skv_attn_fwd_noalloc(const void* plan, const void* q, const void* k, const void* v, void* o, float* lse,
+                         skv_stream_t stream);
 
 #ifdef __cplusplus
 }

@@ -142,6 +142,13 @@ int prepare_ws(const PlanHeader& h, const void* plan, void* ws, const WsLayout& 
 }
 
 }  // namespace
+
+int skv_record_cuda_error(int cuda_error) { return cuda_fail(static_cast<cudaError_t>(cuda_error)); }
+
+int skv_make_tile_map(CUtensorMap* map, const void* base, int64_t rows, int heads, int d, int box_h, int box_rows) {
+  return make_map(map, base, rows, heads, d, box_h, box_rows);
+}
+
 }  // namespace skv
 
 using namespace skv;
@@ -156,6 +163,7 @@ extern "C" const char* skv_strerror(int code) {
     case SKV_EPLAN: return "not a plan written by skv_plan";
     case SKV_ETIMEOUT: return "a device-side wait timed out";
     case SKV_EDEVICE: return "a kernel found an inconsistent work list";
+    case SKV_ESCRATCH: return "workspace exceeds the library's static scratch (SKV_NOALLOC_SCRATCH_BYTES)";
     default: return "unknown status";
   }
 }

@@ -67,4 +67,8 @@ cudaError_t launch_bwd(int d, const CUtensorMap& tq, const CUtensorMap& tk, cons
                        const CUtensorMap& tdo, const BwdParams& p, int grid, cudaStream_t stream);
 cudaError_t launch_dq_cast(const float* dq_acc, __nv_bfloat16* dq, float scale, long long n, cudaStream_t stream);
 
+// Helpers of the API layer shared with other entry-point files.
+int skv_record_cuda_error(int cuda_error);  // remembers the error, returns SKV_ECUDA
+int skv_make_tile_map(CUtensorMap* map, const void* base, int64_t rows, int heads, int d, int box_h, int box_rows);
+
 }  // namespace skv

@@ -23,7 +23,8 @@ SKV_PLAN_STATIC = 1
 # Every function include/skv.h declares.
 EXPORTS = ("skv_plan_size", "skv_plan", "skv_plan_items", "skv_plan_stats", "skv_attn_fwd", "skv_lse_merge",
            "skv_attn_bwd", "skv_status", "skv_strerror", "skv_last_cuda_error", "skv_set_unit_timer",
-           "skv_set_timing_events")
+           "skv_set_timing_events", "skv_attn_fwd_noalloc")
+SKV_NOALLOC_SCRATCH_BYTES = 32 << 20
 SKV_KERNEL_FWD, SKV_KERNEL_MERGE, SKV_KERNEL_BWD = 0, 1, 2
 
 
@@ -67,6 +68,7 @@ def lib() -> ctypes.CDLL:
         L.skv_strerror.restype = ctypes.c_char_p
         L.skv_set_unit_timer.argtypes = [vp, vp]
         L.skv_set_timing_events.argtypes = [ctypes.c_int, vp, vp]
+        L.skv_attn_fwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp]
         for name in EXPORTS:
             if name not in ("skv_strerror",):
                 getattr(L, name).restype = ctypes.c_int
@@ -191,6 +193,13 @@ def skv_attn_bwd(plan: Plan, q, k, v, o, lse, do, dq, dk, dv, ws, stream=None):
     _check("skv_attn_bwd", lib().skv_attn_bwd(plan.ptr, _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(do),
                                               _ptr(dq), _ptr(dk), _ptr(dv), _ptr(ws), ws.numel(),
                                               _stream_ptr(stream)))
+
+
+def skv_attn_fwd_noalloc(plan: Plan, q, k, v, o, lse, stream=None):
+    """Forward + merge with the library's static scratch: for callers that
+    cannot allocate device memory (see include/skv.h)."""
+    _check("skv_attn_fwd_noalloc", lib().skv_attn_fwd_noalloc(plan.ptr, _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse),
+                                                              _stream_ptr(stream)))
 
 
 def skv_status(ws, stream=None) -> int:
