@@ -76,7 +76,7 @@ def bwd_bytes(prob):
 
 
 KERNEL_SOURCES = {"fwd_kernel": ["fwd.cu", "sm100.cuh", "kernels.h", "plan_layout.h"],
-                  "bwd_kernel": ["bwd.cu", "sm100.cuh", "kernels.h", "plan_layout.h"],
+                  "bwd_kernel": ["bwd.cu", "bwd2.cu", "sm100.cuh", "kernels.h", "plan_layout.h"],
                   "merge_kernel": ["merge.cu", "sm100.cuh", "kernels.h", "plan_layout.h"]}
 
 

@@ -1,4 +1,5 @@
-// Split-KV backward on sm_100a.
+// Split-KV backward on sm_100a (head_dim 64; head_dim 128 runs the pipelined
+// kernel of bwd2.cu).
 //
 // Gradients through the split ("Split-KV: Breaking the Context Parallelism
 // Bottleneck in Diffusion Drafter Training", section "Split-KV's Core
@@ -345,21 +346,15 @@ __global__ void __launch_bounds__(256, 1)
   }
 }
 
-int bwd_smem_bytes(int d) { return d == 64 ? BwdSmem<64>::kDyn : BwdSmem<128>::kDyn; }
+int bwd_smem_bytes(int d) { return d == 64 ? BwdSmem<64>::kDyn : bwd2_smem_bytes(); }
 
 cudaError_t launch_bwd(int d, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                        const CUtensorMap& tdo, const BwdParams& p, int grid, cudaStream_t stream) {
-  if (d == 64) {
-    auto k = bwd_kernel<64>;
-    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, BwdSmem<64>::kDyn);
-    if (e != cudaSuccess) return e;
-    k<<<grid, 256, BwdSmem<64>::kDyn, stream>>>(tq, tk, tv, tdo, p);
-  } else {
-    auto k = bwd_kernel<128>;
-    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, BwdSmem<128>::kDyn);
-    if (e != cudaSuccess) return e;
-    k<<<grid, 256, BwdSmem<128>::kDyn, stream>>>(tq, tk, tv, tdo, p);
-  }
+  if (d == 128) return launch_bwd2(tq, tk, tv, tdo, p, grid, stream);
+  auto k = bwd_kernel<64>;
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, BwdSmem<64>::kDyn);
+  if (e != cudaSuccess) return e;
+  k<<<grid, 256, BwdSmem<64>::kDyn, stream>>>(tq, tk, tv, tdo, p);
   return cudaGetLastError();
 }
 

@@ -1,0 +1,427 @@
+// Split-KV backward on sm_100a, head_dim 128: pipelined version.
+//
+// Same mathematics as bwd.cu (gradients through the split with P recomputed
+// from the merged LSE; "Split-KV: Breaking the Context Parallelism Bottleneck
+// in Diffusion Drafter Training", section "Split-KV's Core Mechanism"), laid
+// out so that the tensor core is rarely idle:
+//   * TMEM: two 128-column regions R0/R1 that swap roles every query tile
+//     (S^T of tile i and dQ^T of tile i in R_p, dP^T of tile i and then P^T
+//     (bf16, packed) in R_{1-p}, p = i & 1), plus dV and dK accumulators;
+//     S^T of tile i+1 is computed while tile i's gradient MMAs run.
+//   * Two softmax-gradient warpgroups, each owning 64 of the tile's 128 query
+//     rows (TMEM columns); the gradient MMAs of a half start as soon as that
+//     half is ready.
+//   * P^T stays in TMEM and feeds dV += P^T dO as the A operand; dS^T goes to
+//     shared memory once and serves as the A operand of dK += dS^T Q and the
+//     B operand of dQ^T = K^T dS^T.
+//   * dQ is produced transposed (TMEM lane = head-dim index), so the fp32
+//     reduction into the shared dQ accumulator writes 128 consecutive floats
+//     of a row per warpgroup instruction.
+//   * Q and dO tiles are double-buffered.
+// Warp roles: 0 scheduler + TMA producer, 1 MMA issuer, 2 TMEM allocator,
+// 4..7 warpgroup 0 (rows 0..63), 8..11 warpgroup 1 (rows 64..127).
+#include <cuda_runtime.h>
+
+#include "kernels.h"
+#include "sm100.cuh"
+
+namespace skv {
+namespace {
+
+constexpr int kD = 128;
+constexpr int kTileBytes = 128 * kD * 2;  // 128 rows x 128 bf16
+
+struct Ctl {
+  uint64_t sched_full[2], sched_empty[2];
+  uint64_t kv_full, kv_empty;
+  uint64_t q_full[2], q_empty[2], do_full[2], do_empty[2];
+  uint64_t sdp_full;
+  uint64_t pds_full[2];
+  uint64_t dv_done;
+  uint64_t dq_full[2], dq_free[2];
+  uint64_t acc_full, acc_free;
+  uint64_t meta_full[2][2];  // [warpgroup][tile parity]
+  uint64_t final_mma;
+  int32_t sched[2];
+  uint32_t tmem_base;
+  float lse2[2][128];    // [tile parity][row]: log2-domain LSE (+inf for absent rows)
+  float delta[2][128];   // D of the row
+  int16_t kend[2][128];  // keys of this unit the row attends: t < kend (0..128)
+};
+
+constexpr int kK = 0;
+constexpr int kV = kK + kTileBytes;
+constexpr int kQ0 = kV + kTileBytes;          // two stages
+constexpr int kDO0 = kQ0 + 2 * kTileBytes;    // two stages
+constexpr int kDS = kDO0 + 2 * kTileBytes;    // dS^T [128 keys][128 rows] bf16
+constexpr int kCtl = kDS + 128 * 128 * 2;
+constexpr int kSmemBytes = kCtl + static_cast<int>(sizeof(Ctl));
+static_assert(kSmemBytes <= 232448, "shared memory budget");
+
+__device__ __forceinline__ uint32_t col_r(uint32_t i) { return 128u * (i & 1u); }  // region R0 or R1
+constexpr uint32_t kColDV = 256, kColDK = 384;
+
+__global__ void __launch_bounds__(384, 1)
+    bwd2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
+                const BwdParams p) {
+  extern __shared__ __align__(1024) uint8_t smem[];
+  Ctl& c = *reinterpret_cast<Ctl*>(smem + kCtl);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  int* status = p.status;
+  const uint64_t lim = p.timeout_ns;
+
+  // The 128-byte swizzle needs 1024-byte aligned tiles.
+  if ((smem_u32(smem) & 1023u) != 0) {
+    if (tid == 0) atomicCAS(status, 0, kStatusBadPlan);
+    return;
+  }
+  if (tid == 0) {
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&c.sched_full[i], 1);
+      mbar_init(&c.sched_empty[i], 1 + 8);
+      mbar_init(&c.q_full[i], 1);
+      mbar_init(&c.q_empty[i], 1);
+      mbar_init(&c.do_full[i], 1);
+      mbar_init(&c.do_empty[i], 1);
+      mbar_init(&c.pds_full[i], 128);
+      mbar_init(&c.dq_full[i], 1);
+      mbar_init(&c.dq_free[i], 128);
+      mbar_init(&c.meta_full[i][0], 128);
+      mbar_init(&c.meta_full[i][1], 128);
+    }
+    mbar_init(&c.kv_full, 1);
+    mbar_init(&c.kv_empty, 1);
+    mbar_init(&c.sdp_full, 1);
+    mbar_init(&c.dv_done, 1);
+    mbar_init(&c.acc_full, 1);
+    mbar_init(&c.acc_free, 256);
+    mbar_init(&c.final_mma, 1);
+    fence_mbar_init();
+  }
+  if (warp == 2) {
+    tmem_alloc(&c.tmem_base, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = c.tmem_base;
+
+  if (warp == 0) {
+    // ------------------------------------------------ scheduler + producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tmQ);
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
+      tma_prefetch_desc(&tmDO);
+      int part = static_cast<int>((static_cast<long long>(blockIdx.x) * p.P) / gridDim.x);
+      int visited = 0;
+      uint32_t n_units = 0, qc = 0, kv_issued = 0;
+      bool ok = true;
+      auto load_tile = [&](const MTile& M, int g) -> bool {
+        const int s = qc & 1;
+        const uint32_t use = qc >> 1;
+        if (use >= 1 && !mbar_wait(&c.q_empty[s], (use - 1) & 1, status, lim)) return false;
+        mbar_arrive_expect_tx(&c.q_full[s], kTileBytes);
+        for (int db = 0; db < 2; ++db)
+          tma_load_3d(smem + kQ0 + s * kTileBytes + db * 16384, &tmQ, &c.q_full[s], db * 64, g * p.G, M.tok0);
+        if (use >= 1 && !mbar_wait(&c.do_empty[s], (use - 1) & 1, status, lim)) return false;
+        mbar_arrive_expect_tx(&c.do_full[s], kTileBytes);
+        for (int db = 0; db < 2; ++db)
+          tma_load_3d(smem + kDO0 + s * kTileBytes + db * 16384, &tmDO, &c.do_full[s], db * 64, g * p.G, M.tok0);
+        ++qc;
+        return true;
+      };
+      while (ok) {
+        int u = -1;
+        while (visited < p.P) {
+          const int cnt = p.part_off[part + 1] - p.part_off[part];
+          const int idx = atomicAdd(&p.counters[part], 1);
+          if (idx < cnt) {
+            u = p.part_off[part] + idx;
+            break;
+          }
+          part = (part + 1 == p.P) ? 0 : part + 1;
+          ++visited;
+        }
+        const int slot = n_units & 1;
+        if (n_units >= 2 && !mbar_wait(&c.sched_empty[slot], ((n_units >> 1) - 1) & 1, status, lim)) break;
+        c.sched[slot] = u;
+        mbar_arrive(&c.sched_full[slot]);
+        if (u < 0) break;
+        const BwdUnit U = p.units[u];
+        bool kv_loaded = false;
+        for (int mt = U.mt_begin; mt < U.mt_end && ok; ++mt) {
+          const MTile M = p.mtiles[mt];
+          if (M.kmax <= U.kbeg) continue;
+          if (!load_tile(M, U.g)) { ok = false; break; }
+          if (!kv_loaded) {  // after the first Q/dO tile: K/V wait for the previous unit's last MMA
+            if (kv_issued >= 1 && !mbar_wait(&c.kv_empty, (kv_issued - 1) & 1, status, lim)) { ok = false; break; }
+            mbar_arrive_expect_tx(&c.kv_full, 2 * kTileBytes);
+            for (int db = 0; db < 2; ++db) {
+              tma_load_3d(smem + kK + db * 16384, &tmK, &c.kv_full, db * 64, U.g, U.kbeg);
+              tma_load_3d(smem + kV + db * 16384, &tmV, &c.kv_full, db * 64, U.g, U.kbeg);
+            }
+            ++kv_issued;
+            kv_loaded = true;
+          }
+        }
+        ++n_units;
+      }
+      // let every issued load land before the CTA may exit
+      if (kv_issued > 0) mbar_wait(&c.kv_full, (kv_issued - 1) & 1, nullptr, lim);
+      for (int s = 0; s < 2; ++s) {
+        const uint32_t uses = (qc + 1 - s) >> 1;
+        if (uses > 0) {
+          mbar_wait(&c.q_full[s], (uses - 1) & 1, nullptr, lim);
+          mbar_wait(&c.do_full[s], (uses - 1) & 1, nullptr, lim);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idS = idesc_bf16(128, 128, false, false);  // S^T = K Q^T, dP^T = V dO^T
+      constexpr uint32_t idKV = idesc_bf16(128, kD, false, true);   // dV += P^T dO, dK += dS^T Q
+      constexpr uint32_t idQ = idesc_bf16(128, 64, true, true);     // dQ^T(half) = K^T dS^T(half)
+      const uint32_t sK = smem_u32(smem + kK), sV = smem_u32(smem + kV), sQ0 = smem_u32(smem + kQ0),
+                     sDO0 = smem_u32(smem + kDO0), sDS = smem_u32(smem + kDS);
+      uint32_t n_units = 0, qc = 0, kv_waits = 0;
+      bool ok = true;
+      while (ok) {
+        const int slot = n_units & 1;
+        if (!mbar_wait(&c.sched_full[slot], (n_units >> 1) & 1, status, lim)) break;
+        const int u = c.sched[slot];
+        mbar_arrive(&c.sched_empty[slot]);
+        if (u < 0) break;
+        const BwdUnit U = p.units[u];
+        bool first = true;
+        for (int mt = U.mt_begin; mt < U.mt_end; ++mt) {
+          if (p.mtiles[mt].kmax <= U.kbeg) continue;
+          const int s = qc & 1;
+          const uint32_t use = qc >> 1;
+          const uint32_t rS = tmem + col_r(qc), rP = tmem + col_r(qc + 1);
+          const uint32_t sQ = sQ0 + s * kTileBytes, sDO = sDO0 + s * kTileBytes;
+          if (first && !mbar_wait(&c.kv_full, (kv_waits++) & 1, status, lim)) { ok = false; break; }
+          if (!mbar_wait(&c.q_full[s], use & 1, status, lim)) { ok = false; break; }
+          // S^T -> R_p, where the previous tile's P^T lived: its dV MMA must be done
+          if (qc >= 1 && !mbar_wait(&c.dv_done, (qc - 1) & 1, status, lim)) { ok = false; break; }
+          tc_fence_after();
+#pragma unroll
+          for (int ks = 0; ks < kD / 16; ++ks) {
+            const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
+            umma_bf16(rS, sdesc_sw128(sK + off, 16, 1024), sdesc_sw128(sQ + off, 16, 1024), idS, ks > 0);
+          }
+          // dP^T -> R_{1-p}, where the previous tile's dQ^T lived: it must be drained
+          if (!mbar_wait(&c.do_full[s], use & 1, status, lim)) { ok = false; break; }
+          if (qc >= 1 && (!mbar_wait(&c.dq_free[0], (qc - 1) & 1, status, lim) ||
+                          !mbar_wait(&c.dq_free[1], (qc - 1) & 1, status, lim))) { ok = false; break; }
+          tc_fence_after();
+#pragma unroll
+          for (int ks = 0; ks < kD / 16; ++ks) {
+            const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
+            umma_bf16(rP, sdesc_sw128(sV + off, 16, 1024), sdesc_sw128(sDO + off, 16, 1024), idS, ks > 0);
+          }
+          umma_commit(&c.sdp_full);
+          for (int h = 0; h < 2 && ok; ++h) {
+            if (!mbar_wait(&c.pds_full[h], qc & 1, status, lim)) { ok = false; break; }
+            if (first && h == 0 && n_units >= 1 && !mbar_wait(&c.acc_free, (n_units - 1) & 1, status, lim)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            // dV += P^T dO over the half's 64 rows (A = P^T from TMEM)
+#pragma unroll
+            for (int k4 = 0; k4 < 4; ++k4) {
+              const uint32_t acc = (first && h == 0 && k4 == 0) ? 0u : 1u;
+              umma_bf16_ts(tmem + kColDV, rP + 64 * h + 8 * k4,
+                           sdesc_sw128(sDO + (64 * h + 16 * k4) * 128, 16384, 1024), idKV, acc);
+            }
+            if (h == 1) {
+              umma_commit(&c.dv_done);
+              umma_commit(&c.do_empty[s]);
+            }
+            // dK += dS^T Q over the half's rows
+#pragma unroll
+            for (int k4 = 0; k4 < 4; ++k4) {
+              const uint32_t acc = (first && h == 0 && k4 == 0) ? 0u : 1u;
+              umma_bf16(tmem + kColDK, sdesc_sw128(sDS + h * 16384 + k4 * 32, 16, 1024),
+                        sdesc_sw128(sQ + (64 * h + 16 * k4) * 128, 16384, 1024), idKV, acc);
+            }
+            if (h == 1) umma_commit(&c.q_empty[s]);
+            // dQ^T of the half's rows = K^T dS^T -> R_p columns [64h, 64h + 64)
+#pragma unroll
+            for (int ks = 0; ks < 128 / 16; ++ks)
+              umma_bf16(rS + 64 * h, sdesc_sw128(sK + ks * 2048, 16384, 1024),
+                        sdesc_sw128(sDS + h * 16384 + ks * 2048, 16384, 1024), idQ, ks > 0);
+            umma_commit(&c.dq_full[h]);
+          }
+          if (!ok) break;
+          first = false;
+          ++qc;
+        }
+        if (!ok) break;
+        if (!first) umma_commit(&c.kv_empty);  // K/V were loaded for this unit
+        umma_commit(&c.acc_full);
+        ++n_units;
+      }
+      umma_commit(&c.final_mma);
+      mbar_wait(&c.final_mma, 0, nullptr, lim);
+    }
+  } else if (warp >= 4) {
+    // ------------------------- softmax gradient, dQ drain, dK/dV epilogue
+    const int wg = (warp - 4) >> 2;          // warpgroup: rows [64 wg, 64 wg + 64) of the tile
+    const int t = (warp & 3) * 32 + lane;    // TMEM lane: key (S^T, dP^T, dV, dK) or d index (dQ^T)
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    constexpr float kLog2e = 1.4426950408889634f;
+    uint32_t n_units = 0, qc = 0;
+    bool ok = true;
+    while (ok) {
+      const int slot = n_units & 1;
+      if (!mbar_wait_warp(&c.sched_full[slot], (n_units >> 1) & 1, status, lim)) break;
+      const int u = c.sched[slot];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&c.sched_empty[slot]);
+      if (u < 0) break;
+      const BwdUnit U = p.units[u];
+      if (p.stamps && tid == 128) p.stamps[2 * u] = static_cast<long long>(globaltimer_ns());
+      const int nkeys = U.kend - U.kbeg;
+      bool had_tiles = false;
+      for (int mt = U.mt_begin; mt < U.mt_end; ++mt) {
+        const MTile M = p.mtiles[mt];
+        if (M.kmax <= U.kbeg) continue;
+        had_tiles = true;
+        const int par = qc & 1;
+        const uint32_t rS = tmem + lane_off + col_r(par), rP = tmem + lane_off + col_r(par + 1);
+        // stage the metadata of this warpgroup's 64 rows
+        if (t < 64) {
+          const int r = 64 * wg + t;
+          const int tl = r / p.G;
+          const bool valid = tl < M.ntok;
+          const int token = M.tok0 + tl, head = U.g * p.G + r % p.G;
+          c.lse2[par][r] = valid ? p.lse[static_cast<size_t>(token) * p.Hq + head] * kLog2e : INFINITY;
+          c.delta[par][r] = valid ? p.delta[static_cast<size_t>(token) * p.Hq + head] : 0.f;
+          const int ke = valid ? min(p.tok_kend[token], U.kend) - U.kbeg : 0;
+          c.kend[par][r] = static_cast<int16_t>(max(0, min(ke, nkeys)));
+        }
+        mbar_arrive(&c.meta_full[wg][par]);
+        if (!mbar_wait_warp(&c.meta_full[wg][par], (qc >> 1) & 1, status, lim)) { ok = false; break; }
+        if (!mbar_wait_warp(&c.sdp_full, qc & 1, status, lim)) { ok = false; break; }
+        tc_fence_after();
+        uint8_t* dsrow = smem + kDS + wg * 16384;
+#pragma unroll 1
+        for (int ch = 0; ch < 2; ++ch) {
+          const int col = 64 * wg + 32 * ch;  // first tile row of this chunk
+          uint32_t vs[32], vd[32];
+          tmem_ld32(rS + col, vs);
+          tmem_ld32(rP + col, vd);
+          tmem_wait_ld();
+          uint32_t pk[16];
+          uint32_t dk[16];
+#pragma unroll
+          for (int i = 0; i < 32; i += 2) {
+            float pv[2], dv[2];
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+              const int r = col + i + e;
+              const float x = (t < c.kend[par][r]) ? ex2(__uint_as_float(vs[i + e]) * p.scale_log2 - c.lse2[par][r]) : 0.f;
+              pv[e] = x;
+              dv[e] = x * (__uint_as_float(vd[i + e]) - c.delta[par][r]);
+            }
+            pk[i >> 1] = pack_bf16(pv[0], pv[1]);
+            dk[i >> 1] = pack_bf16(dv[0], dv[1]);
+          }
+          // P^T (bf16 pairs) over the dP^T columns already read
+          tmem_st16(rP + 64 * wg + 16 * ch, pk);
+          // dS^T row t of this warpgroup's 64-row block: 16-byte chunks 4 ch .. 4 ch + 3
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            *reinterpret_cast<uint4*>(dsrow + sw128_off(t, 4 * ch + q)) =
+                make_uint4(dk[4 * q], dk[4 * q + 1], dk[4 * q + 2], dk[4 * q + 3]);
+        }
+        tmem_wait_st();
+        fence_proxy_async_smem();
+        tc_fence_before();
+        mbar_arrive(&c.pds_full[wg]);
+        // dQ^T of this warpgroup's rows: lane t = head-dim index t
+        if (!mbar_wait_warp(&c.dq_full[wg], qc & 1, status, lim)) { ok = false; break; }
+        tc_fence_after();
+        uint32_t q0[32], q1[32];
+        tmem_ld32(rS + 64 * wg, q0);
+        tmem_ld32(rS + 64 * wg + 32, q1);
+        tmem_wait_ld();
+        tc_fence_before();
+        mbar_arrive(&c.dq_free[wg]);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          const int r = 64 * wg + j;
+          const int tl = r / p.G;
+          if (tl < M.ntok) {
+            const int token = M.tok0 + tl, head = U.g * p.G + r % p.G;
+            atomicAdd(p.dq_acc + (static_cast<size_t>(token) * p.Hq + head) * kD + t, __uint_as_float(q0[j]));
+          }
+        }
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          const int r = 64 * wg + 32 + j;
+          const int tl = r / p.G;
+          if (tl < M.ntok) {
+            const int token = M.tok0 + tl, head = U.g * p.G + r % p.G;
+            atomicAdd(p.dq_acc + (static_cast<size_t>(token) * p.Hq + head) * kD + t, __uint_as_float(q1[j]));
+          }
+        }
+        ++qc;
+      }
+      if (!ok) break;
+      // dV (warpgroup 0) / dK (warpgroup 1) of the unit's keys
+      if (!mbar_wait_warp(&c.acc_full, n_units & 1, status, lim)) break;
+      tc_fence_after();
+      const uint32_t acc_col = wg == 0 ? kColDV : kColDK;
+      // a unit without live query tiles (none are planned) would own zero gradients
+      const float mul = !had_tiles ? 0.f : (wg == 0 ? 1.f : p.scale);
+      __nv_bfloat16* dst = (wg == 0 ? p.dv : p.dk) + (static_cast<size_t>(U.kbeg + t) * p.Hkv + U.g) * kD;
+#pragma unroll 1
+      for (int cc = 0; cc < kD; cc += 32) {
+        uint32_t v[32];
+        tmem_ld32(tmem + lane_off + acc_col + cc, v);
+        tmem_wait_ld();
+        if (t < nkeys) {
+#pragma unroll
+          for (int i = 0; i < 32; i += 8) {
+            uint4 w;
+            w.x = pack_bf16(__uint_as_float(v[i]) * mul, __uint_as_float(v[i + 1]) * mul);
+            w.y = pack_bf16(__uint_as_float(v[i + 2]) * mul, __uint_as_float(v[i + 3]) * mul);
+            w.z = pack_bf16(__uint_as_float(v[i + 4]) * mul, __uint_as_float(v[i + 5]) * mul);
+            w.w = pack_bf16(__uint_as_float(v[i + 6]) * mul, __uint_as_float(v[i + 7]) * mul);
+            *reinterpret_cast<uint4*>(dst + cc + i) = w;
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&c.acc_free);
+      if (p.stamps && tid == 128) p.stamps[2 * u + 1] = static_cast<long long>(globaltimer_ns());
+      ++n_units;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 2) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace
+
+int bwd2_smem_bytes() { return kSmemBytes; }
+
+cudaError_t launch_bwd2(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tdo,
+                        const BwdParams& p, int grid, cudaStream_t stream) {
+  cudaError_t e = cudaFuncSetAttribute(bwd2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  if (e != cudaSuccess) return e;
+  bwd2_kernel<<<grid, 384, kSmemBytes, stream>>>(tq, tk, tv, tdo, p);
+  return cudaGetLastError();
+}
+
+}  // namespace skv

@@ -65,6 +65,9 @@ cudaError_t launch_bwd_prep(int d, const __nv_bfloat16* o, const __nv_bfloat16* 
                             long long n_rows, cudaStream_t stream);
 cudaError_t launch_bwd(int d, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                        const CUtensorMap& tdo, const BwdParams& p, int grid, cudaStream_t stream);
+cudaError_t launch_bwd2(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tdo,
+                        const BwdParams& p, int grid, cudaStream_t stream);  // head_dim 128
+int bwd2_smem_bytes();
 cudaError_t launch_dq_cast(const float* dq_acc, __nv_bfloat16* dq, float scale, long long n, cudaStream_t stream);
 
 // Helpers of the API layer shared with other entry-point files.
