@@ -309,7 +309,9 @@ extern "C" int skv_attn_bwd(const void* plan, const void* q, const void* k, cons
     p.G = h->G;
     p.Hq = h->Hq;
     p.Hkv = h->Hkv;
-    p.scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(h->d)));
+    p.lgG = 0;
+    while ((1 << p.lgG) < h->G) ++p.lgG;
+    p.scale =static_cast<float>(1.0 / std::sqrt(static_cast<double>(h->d)));
     p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(h->d)));
     int sms = num_sms();
     if (sms <= 0) return cuda_fail(cudaGetLastError());

@@ -32,6 +32,10 @@ constexpr int kD = 128;
 constexpr int kTileBytes = 128 * kD * 2;  // 128 rows x 128 bf16
 
 struct Ctl {
+  float lse2[2][128];    // [tile parity][row]: log2-domain LSE (+inf for absent rows)
+  float delta[2][128];   // D of the row
+  uint8_t kend[2][128];  // keys of this unit the row attends: t < kend (0..128)
+  int32_t kmin[2][2][2]; // [warpgroup][tile parity][warp]: min of kend over 32 rows
   uint64_t sched_full[2], sched_empty[2];
   uint64_t kv_full, kv_empty;
   uint64_t q_full[2], q_empty[2], do_full[2], do_empty[2];
@@ -44,9 +48,6 @@ struct Ctl {
   uint64_t final_mma;
   int32_t sched[2];
   uint32_t tmem_base;
-  float lse2[2][128];    // [tile parity][row]: log2-domain LSE (+inf for absent rows)
-  float delta[2][128];   // D of the row
-  int16_t kend[2][128];  // keys of this unit the row attends: t < kend (0..128)
 };
 
 constexpr int kK = 0;
@@ -61,6 +62,8 @@ static_assert(kSmemBytes <= 232448, "shared memory budget");
 __device__ __forceinline__ uint32_t col_r(uint32_t i) { return 128u * (i & 1u); }  // region R0 or R1
 constexpr uint32_t kColDV = 256, kColDK = 384;
 
+// kG: compile-time q-heads per kv-head (0 = runtime value p.G)
+template <int kG>
 __global__ void __launch_bounds__(384, 1)
     bwd2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                 const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
@@ -275,8 +278,25 @@ __global__ void __launch_bounds__(384, 1)
     const int t = (warp & 3) * 32 + lane;    // TMEM lane: key (S^T, dP^T, dV, dK) or d index (dQ^T)
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
     constexpr float kLog2e = 1.4426950408889634f;
+    const int G = kG > 0 ? kG : p.G;
+    const int lgG = kG > 0 ? (31 - __clz(kG)) : p.lgG;
+    const size_t tok_stride = static_cast<size_t>(p.Hq) * kD;
     uint32_t n_units = 0, qc = 0;
     bool ok = true;
+    // metadata of the next live query tile, fetched one tile ahead (threads t < 64: row 64 wg + t)
+    float pf_lse = INFINITY, pf_del = 0.f;
+    int pf_ke = 0;
+    auto fetch = [&](const MTile& M, const BwdUnit& U, int nkeys) {
+      if (t < 64) {
+        const int r = 64 * wg + t;
+        const int tl = r >> lgG;
+        const bool valid = tl < M.ntok;
+        const int token = M.tok0 + tl, head = U.g * G + (r & (G - 1));
+        pf_lse = valid ? p.lse[static_cast<size_t>(token) * p.Hq + head] * kLog2e : INFINITY;
+        pf_del = valid ? p.delta[static_cast<size_t>(token) * p.Hq + head] : 0.f;
+        pf_ke = valid ? max(0, min(min(p.tok_kend[token], U.kend) - U.kbeg, nkeys)) : 0;
+      }
+    };
     while (ok) {
       const int slot = n_units & 1;
       if (!mbar_wait_warp(&c.sched_full[slot], (n_units >> 1) & 1, status, lim)) break;
@@ -287,29 +307,42 @@ __global__ void __launch_bounds__(384, 1)
       const BwdUnit U = p.units[u];
       if (p.stamps && tid == 128) p.stamps[2 * u] = static_cast<long long>(globaltimer_ns());
       const int nkeys = U.kend - U.kbeg;
+      int mt = U.mt_begin;
+      while (mt < U.mt_end && p.mtiles[mt].kmax <= U.kbeg) ++mt;
+      MTile M{};
+      if (mt < U.mt_end) {
+        M = p.mtiles[mt];
+        fetch(M, U, nkeys);
+      }
       bool had_tiles = false;
-      for (int mt = U.mt_begin; mt < U.mt_end; ++mt) {
-        const MTile M = p.mtiles[mt];
-        if (M.kmax <= U.kbeg) continue;
+      while (mt < U.mt_end) {
         had_tiles = true;
         const int par = qc & 1;
         const uint32_t rS = tmem + lane_off + col_r(par), rP = tmem + lane_off + col_r(par + 1);
-        // stage the metadata of this warpgroup's 64 rows
+        // stage this tile's metadata, then fetch the next live tile's
         if (t < 64) {
           const int r = 64 * wg + t;
-          const int tl = r / p.G;
-          const bool valid = tl < M.ntok;
-          const int token = M.tok0 + tl, head = U.g * p.G + r % p.G;
-          c.lse2[par][r] = valid ? p.lse[static_cast<size_t>(token) * p.Hq + head] * kLog2e : INFINITY;
-          c.delta[par][r] = valid ? p.delta[static_cast<size_t>(token) * p.Hq + head] : 0.f;
-          const int ke = valid ? min(p.tok_kend[token], U.kend) - U.kbeg : 0;
-          c.kend[par][r] = static_cast<int16_t>(max(0, min(ke, nkeys)));
+          c.lse2[par][r] = pf_lse;
+          c.delta[par][r] = pf_del;
+          c.kend[par][r] = static_cast<uint8_t>(pf_ke);
+          const int wmin = __reduce_min_sync(0xffffffffu, pf_ke);
+          if (lane == 0) c.kmin[wg][par][warp & 1] = wmin;
+        }
+        int nxt = mt + 1;
+        while (nxt < U.mt_end && p.mtiles[nxt].kmax <= U.kbeg) ++nxt;
+        MTile Mn = M;
+        if (nxt < U.mt_end) {
+          Mn = p.mtiles[nxt];
+          fetch(Mn, U, nkeys);
         }
         mbar_arrive(&c.meta_full[wg][par]);
         if (!mbar_wait_warp(&c.meta_full[wg][par], (qc >> 1) & 1, status, lim)) { ok = false; break; }
+        // every row of this half attends key t of every lane of the warp: no per-element mask
+        const bool unmasked = __all_sync(0xffffffffu, t < min(c.kmin[wg][par][0], c.kmin[wg][par][1]));
         if (!mbar_wait_warp(&c.sdp_full, qc & 1, status, lim)) { ok = false; break; }
         tc_fence_after();
         uint8_t* dsrow = smem + kDS + wg * 16384;
+        const float sl2 = p.scale_log2;
 #pragma unroll 1
         for (int ch = 0; ch < 2; ++ch) {
           const int col = 64 * wg + 32 * ch;  // first tile row of this chunk
@@ -320,17 +353,24 @@ __global__ void __launch_bounds__(384, 1)
           uint32_t pk[16];
           uint32_t dk[16];
 #pragma unroll
-          for (int i = 0; i < 32; i += 2) {
-            float pv[2], dv[2];
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-              const int r = col + i + e;
-              const float x = (t < c.kend[par][r]) ? ex2(__uint_as_float(vs[i + e]) * p.scale_log2 - c.lse2[par][r]) : 0.f;
-              pv[e] = x;
-              dv[e] = x * (__uint_as_float(vd[i + e]) - c.delta[par][r]);
+          for (int i = 0; i < 32; i += 4) {
+            const float4 L4 = *reinterpret_cast<const float4*>(&c.lse2[par][col + i]);
+            const float4 D4 = *reinterpret_cast<const float4*>(&c.delta[par][col + i]);
+            float x0 = ex2(fmaf(__uint_as_float(vs[i + 0]), sl2, -L4.x));
+            float x1 = ex2(fmaf(__uint_as_float(vs[i + 1]), sl2, -L4.y));
+            float x2 = ex2(fmaf(__uint_as_float(vs[i + 2]), sl2, -L4.z));
+            float x3 = ex2(fmaf(__uint_as_float(vs[i + 3]), sl2, -L4.w));
+            if (!unmasked) {
+              const uint32_t k4 = *reinterpret_cast<const uint32_t*>(&c.kend[par][col + i]);
+              x0 = t < static_cast<int>(k4 & 0xffu) ? x0 : 0.f;
+              x1 = t < static_cast<int>((k4 >> 8) & 0xffu) ? x1 : 0.f;
+              x2 = t < static_cast<int>((k4 >> 16) & 0xffu) ? x2 : 0.f;
+              x3 = t < static_cast<int>(k4 >> 24) ? x3 : 0.f;
             }
-            pk[i >> 1] = pack_bf16(pv[0], pv[1]);
-            dk[i >> 1] = pack_bf16(dv[0], dv[1]);
+            pk[(i >> 1) + 0] = pack_bf16(x0, x1);
+            pk[(i >> 1) + 1] = pack_bf16(x2, x3);
+            dk[(i >> 1) + 0] = pack_bf16(x0 * (__uint_as_float(vd[i + 0]) - D4.x), x1 * (__uint_as_float(vd[i + 1]) - D4.y));
+            dk[(i >> 1) + 1] = pack_bf16(x2 * (__uint_as_float(vd[i + 2]) - D4.z), x3 * (__uint_as_float(vd[i + 3]) - D4.w));
           }
           // P^T (bf16 pairs) over the dP^T columns already read
           tmem_st16(rP + 64 * wg + 16 * ch, pk);
@@ -353,33 +393,46 @@ __global__ void __launch_bounds__(384, 1)
         tmem_wait_ld();
         tc_fence_before();
         mbar_arrive(&c.dq_free[wg]);
+        // fp32 reduction: row r -> dq_acc[(tok0 + r / G) * Hq + g * G + r % G][t]
+        float* base = p.dq_acc + (static_cast<size_t>(M.tok0) * p.Hq + static_cast<size_t>(U.g) * G) * kD + t;
+        if constexpr (kG > 0) {
+          static_assert(64 % (kG > 0 ? kG : 1) == 0, "group size must divide 64");
+          constexpr int kTok = 64 / (kG > 0 ? kG : 1);  // tokens per half tile
+          const int tl0 = (64 * wg) / (kG > 0 ? kG : 1);
+          float* row0 = base + static_cast<size_t>(tl0) * tok_stride;
+          const int ntok_here = min(M.ntok - tl0, kTok);  // tokens of this half that exist
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          const int r = 64 * wg + j;
-          const int tl = r / p.G;
-          if (tl < M.ntok) {
-            const int token = M.tok0 + tl, head = U.g * p.G + r % p.G;
-            atomicAdd(p.dq_acc + (static_cast<size_t>(token) * p.Hq + head) * kD + t, __uint_as_float(q0[j]));
+          for (int j = 0; j < 32; ++j)
+            if (j / kG < ntok_here)
+              atomicAdd(row0 + static_cast<size_t>(j / kG) * tok_stride + (j % kG) * kD, __uint_as_float(q0[j]));
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            if ((32 + j) / kG < ntok_here)
+              atomicAdd(row0 + static_cast<size_t>((32 + j) / kG) * tok_stride + ((32 + j) % kG) * kD,
+                        __uint_as_float(q1[j]));
+        } else {
+          const int nrows = M.ntok << lgG;
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const int r = 64 * wg + j;
+            if (r < nrows) atomicAdd(base + (r >> lgG) * tok_stride + (r & (G - 1)) * kD, __uint_as_float(q0[j]));
           }
-        }
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          const int r = 64 * wg + 32 + j;
-          const int tl = r / p.G;
-          if (tl < M.ntok) {
-            const int token = M.tok0 + tl, head = U.g * p.G + r % p.G;
-            atomicAdd(p.dq_acc + (static_cast<size_t>(token) * p.Hq + head) * kD + t, __uint_as_float(q1[j]));
+          for (int j = 0; j < 32; ++j) {
+            const int r = 64 * wg + 32 + j;
+            if (r < nrows) atomicAdd(base + (r >> lgG) * tok_stride + (r & (G - 1)) * kD, __uint_as_float(q1[j]));
           }
         }
         ++qc;
+        M = Mn;
+        mt = nxt;
       }
       if (!ok) break;
       // dV (warpgroup 0) / dK (warpgroup 1) of the unit's keys
       if (!mbar_wait_warp(&c.acc_full, n_units & 1, status, lim)) break;
       tc_fence_after();
       const uint32_t acc_col = wg == 0 ? kColDV : kColDK;
-      // a unit without live query tiles (none are planned) would own zero gradients
-      const float mul = !had_tiles ? 0.f : (wg == 0 ? 1.f : p.scale);
+      const float mul = wg == 0 ? 1.f : p.scale;
       __nv_bfloat16* dst = (wg == 0 ? p.dv : p.dk) + (static_cast<size_t>(U.kbeg + t) * p.Hkv + U.g) * kD;
 #pragma unroll 1
       for (int cc = 0; cc < kD; cc += 32) {
@@ -389,11 +442,13 @@ __global__ void __launch_bounds__(384, 1)
         if (t < nkeys) {
 #pragma unroll
           for (int i = 0; i < 32; i += 8) {
-            uint4 w;
-            w.x = pack_bf16(__uint_as_float(v[i]) * mul, __uint_as_float(v[i + 1]) * mul);
-            w.y = pack_bf16(__uint_as_float(v[i + 2]) * mul, __uint_as_float(v[i + 3]) * mul);
-            w.z = pack_bf16(__uint_as_float(v[i + 4]) * mul, __uint_as_float(v[i + 5]) * mul);
-            w.w = pack_bf16(__uint_as_float(v[i + 6]) * mul, __uint_as_float(v[i + 7]) * mul);
+            uint4 w = make_uint4(0u, 0u, 0u, 0u);
+            if (had_tiles) {  // a unit without live query tiles (none are planned) owns zero gradients
+              w.x = pack_bf16(__uint_as_float(v[i]) * mul, __uint_as_float(v[i + 1]) * mul);
+              w.y = pack_bf16(__uint_as_float(v[i + 2]) * mul, __uint_as_float(v[i + 3]) * mul);
+              w.z = pack_bf16(__uint_as_float(v[i + 4]) * mul, __uint_as_float(v[i + 5]) * mul);
+              w.w = pack_bf16(__uint_as_float(v[i + 6]) * mul, __uint_as_float(v[i + 7]) * mul);
+            }
             *reinterpret_cast<uint4*>(dst + cc + i) = w;
           }
         }
@@ -418,9 +473,10 @@ int bwd2_smem_bytes() { return kSmemBytes; }
 
 cudaError_t launch_bwd2(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tdo,
                         const BwdParams& p, int grid, cudaStream_t stream) {
-  cudaError_t e = cudaFuncSetAttribute(bwd2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  auto kern = p.G == 4 ? bwd2_kernel<4> : bwd2_kernel<0>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
   if (e != cudaSuccess) return e;
-  bwd2_kernel<<<grid, 384, kSmemBytes, stream>>>(tq, tk, tv, tdo, p);
+  kern<<<grid, 384, kSmemBytes, stream>>>(tq, tk, tv, tdo, p);
   return cudaGetLastError();
 }
 

@@ -52,6 +52,7 @@ struct BwdParams {
   long long* stamps;
   unsigned long long timeout_ns;
   int P, G, Hq, Hkv;
+  int lgG;                  // log2(G); G = Hq / Hkv is a power of two
   float scale;              // 1 / sqrt(d)
   float scale_log2;         // log2(e) / sqrt(d)
 };

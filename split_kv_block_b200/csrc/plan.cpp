@@ -276,7 +276,11 @@ void make_lists(const Prob& q, const std::vector<SampleAnchors>& sa, Built& out)
         u.g = it.g;
         u.kbeg = static_cast<int32_t>(kb);
         u.kend = static_cast<int32_t>(std::min<int64_t>(kb + kTileN, it.key_end));
-        u.mt_begin = out.sample_mt[it.b];
+        // first query tile whose largest anchor reaches past the key tile start
+        // (later dead tiles, possible with unsorted anchors, are skipped by the kernel)
+        int32_t first = out.sample_mt[it.b];
+        while (first < out.sample_mt[it.b + 1] && out.mtiles[first].kmax <= kb) ++first;
+        u.mt_begin = first;
         u.mt_end = out.sample_mt[it.b + 1];
         u.item = id;
         u.part = p;
