@@ -75,7 +75,7 @@ def bwd_bytes(prob):
     return 2 * Nq * Hq * d * 2 + 2 * Nq * Hq * 4 + 4 * keys * Hkv * d * 2 + 2 * Nq * Hq * d * 4
 
 
-KERNEL_SOURCES = {"fwd_kernel": ["fwd.cu", "sm100.cuh", "kernels.h", "plan_layout.h"],
+KERNEL_SOURCES = {"fwd_kernel": ["fwd.cu", "fwd2.cu", "sm100.cuh", "kernels.h", "plan_layout.h"],
                   "bwd_kernel": ["bwd.cu", "bwd2.cu", "sm100.cuh", "kernels.h", "plan_layout.h"],
                   "merge_kernel": ["merge.cu", "sm100.cuh", "kernels.h", "plan_layout.h"]}
 

@@ -207,6 +207,8 @@ extern "C" int skv_attn_fwd(const void* plan, const void* q, const void* k, cons
   p.tok_kend = at<int32_t>(dev, h->dev.tok_kend);
   p.units = at<FwdUnit>(dev, h->dev.fwd_units);
   p.part_off = at<int32_t>(dev, h->dev.fwd_part_off);
+  p.pairs = at<FwdPair>(dev, h->dev.fwd_pairs);
+  p.pair_off = at<int32_t>(dev, h->dev.fwd_pair_off);
   p.counters = at<int32_t>(ws, w.counters);
   p.status = at<int>(ws, w.status);
   p.part_o = at<float>(ws, w.fwd_o);
@@ -218,7 +220,7 @@ extern "C" int skv_attn_fwd(const void* plan, const void* q, const void* k, cons
   p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(h->d)));
   int sms = num_sms();
   if (sms <= 0) return cuda_fail(cudaGetLastError());
-  const int grid = static_cast<int>(std::min<int64_t>(sms, h->n_fwd));
+  const int grid = fwd_grid(h->d, sms, h->n_fwd, h->n_fwd_pairs);
   cudaError_t e = mark(SKV_KERNEL_FWD, 0, stream);
   if (e == cudaSuccess) e = launch_fwd(h->d, tq, tk, tv, p, grid, stream);
   if (e == cudaSuccess) e = mark(SKV_KERNEL_FWD, 1, stream);

@@ -342,20 +342,20 @@ __global__ void __launch_bounds__(256, 1)
 
 int fwd_smem_bytes(int d) { return d == 64 ? FwdSmem<64>::kDyn : FwdSmem<128>::kDyn; }
 
+// head_dim 64 runs the one-tile kernel above; head_dim 128 the two-tile kernel of fwd2.cu
 cudaError_t launch_fwd(int d, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                        const FwdParams& p, int grid, cudaStream_t stream) {
-  if (d == 64) {
-    auto k = fwd_kernel<64>;
-    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, FwdSmem<64>::kDyn);
-    if (e != cudaSuccess) return e;
-    k<<<grid, 256, FwdSmem<64>::kDyn, stream>>>(tq, tk, tv, p);
-  } else {
-    auto k = fwd_kernel<128>;
-    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, FwdSmem<128>::kDyn);
-    if (e != cudaSuccess) return e;
-    k<<<grid, 256, FwdSmem<128>::kDyn, stream>>>(tq, tk, tv, p);
-  }
+  if (d == 128) return launch_fwd2(tq, tk, tv, p, grid, stream);
+  auto k = fwd_kernel<64>;
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, FwdSmem<64>::kDyn);
+  if (e != cudaSuccess) return e;
+  k<<<grid, 256, FwdSmem<64>::kDyn, stream>>>(tq, tk, tv, p);
   return cudaGetLastError();
+}
+
+int fwd_grid(int d, int sms, long long n_units, long long n_pairs) {
+  const long long work = d == 128 ? n_pairs : n_units;
+  return static_cast<int>(work < sms ? work : sms);
 }
 
 }  // namespace skv

@@ -14,6 +14,8 @@ struct FwdParams {
   const int32_t* tok_kend;
   const FwdUnit* units;
   const int32_t* part_off;  // [P+1]
+  const FwdPair* pairs;     // head_dim 128 kernel: pairs of units
+  const int32_t* pair_off;  // [P+1]
   int32_t* counters;        // [P] queue heads, zero at launch
   int* status;
   float* part_o;            // [n_fwd][128][d]
@@ -61,6 +63,11 @@ int fwd_smem_bytes(int d);
 int bwd_smem_bytes(int d);
 cudaError_t launch_fwd(int d, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                        const FwdParams& p, int grid, cudaStream_t stream);
+cudaError_t launch_fwd2(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const FwdParams& p,
+                        int grid, cudaStream_t stream);  // head_dim 128: pairs of query tiles
+int fwd2_smem_bytes();
+// CTAs of the forward launch: one per SM, at most one per work unit (pair for head_dim 128)
+int fwd_grid(int d, int sms, long long n_units, long long n_pairs);
 cudaError_t launch_merge(int d, const MergeParams& p, cudaStream_t stream);
 cudaError_t launch_bwd_prep(int d, const __nv_bfloat16* o, const __nv_bfloat16* dout, float* delta, float* dq_acc,
                             long long n_rows, cudaStream_t stream);

@@ -104,6 +104,8 @@ extern "C" int skv_attn_fwd_noalloc(const void* plan, const void* q, const void*
   p.tok_kend = reinterpret_cast<const int32_t*>(dev + h->dev.tok_kend);
   p.units = reinterpret_cast<const FwdUnit*>(dev + h->dev.fwd_units);
   p.part_off = reinterpret_cast<const int32_t*>(dev + h->dev.fwd_part_off);
+  p.pairs = reinterpret_cast<const FwdPair*>(dev + h->dev.fwd_pairs);
+  p.pair_off = reinterpret_cast<const int32_t*>(dev + h->dev.fwd_pair_off);
   p.counters = reinterpret_cast<int32_t*>(base + w.counters);
   p.status = reinterpret_cast<int*>(base + w.status);
   p.part_o = reinterpret_cast<float*>(base + w.fwd_o);
@@ -117,7 +119,7 @@ extern "C" int skv_attn_fwd_noalloc(const void* plan, const void* q, const void*
   e = cudaGetDevice(&dev_id);
   if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev_id);
   if (e != cudaSuccess) return skv_record_cuda_error(static_cast<int>(e));
-  const int grid = static_cast<int>(std::min<int64_t>(sms, h->n_fwd));
+  const int grid = fwd_grid(h->d, sms, h->n_fwd, h->n_fwd_pairs);
   e = launch_fwd(h->d, tq, tk, tv, p, grid, stream);
   if (e != cudaSuccess) return skv_record_cuda_error(static_cast<int>(e));
 

@@ -99,6 +99,8 @@ struct Built {
   std::vector<int32_t> tok_kend;
   std::vector<FwdUnit> fwd;
   std::vector<int32_t> fwd_part_off;
+  std::vector<FwdPair> pairs;
+  std::vector<int32_t> pair_off;
   std::vector<int32_t> merge_off, merge_list;
   std::vector<BwdUnit> bwd;
   std::vector<int32_t> bwd_part_off;
@@ -243,11 +245,14 @@ void make_lists(const Prob& q, const std::vector<SampleAnchors>& sa, Built& out)
 
   out.fwd.clear();
   out.fwd_part_off.assign(q.P + 1, 0);
+  out.pairs.clear();
+  out.pair_off.assign(q.P + 1, 0);
   out.bwd.clear();
   out.bwd_part_off.assign(q.P + 1, 0);
   std::vector<std::pair<int64_t, int32_t>> tiles;
   for (int p = 0; p < q.P; ++p) {
     out.fwd_part_off[p] = static_cast<int32_t>(out.fwd.size());
+    out.pair_off[p] = static_cast<int32_t>(out.pairs.size());
     out.bwd_part_off[p] = static_cast<int32_t>(out.bwd.size());
     for (int32_t id : by_part[p]) {
       const skv_item& it = out.items[id];
@@ -258,7 +263,8 @@ void make_lists(const Prob& q, const std::vector<SampleAnchors>& sa, Built& out)
         if (ke > it.key_begin) tiles.push_back({-(ke - it.key_begin), mt});
       }
       std::sort(tiles.begin(), tiles.end());
-      for (auto& t : tiles) {
+      for (size_t ti = 0; ti < tiles.size(); ++ti) {
+        const auto& t = tiles[ti];
         FwdUnit u{};
         u.mt = t.second;
         u.g = it.g;
@@ -266,6 +272,18 @@ void make_lists(const Prob& q, const std::vector<SampleAnchors>& sa, Built& out)
         u.kend = static_cast<int32_t>(it.key_begin - t.first);
         u.item = id;
         u.part = p;
+        // consecutive tiles (similar key extents) share a pair; the first is the longer
+        if (ti % 2 == 0) {
+          FwdPair pr{};
+          pr.slot[0] = static_cast<int32_t>(out.fwd.size());
+          pr.slot[1] = -1;
+          pr.kbeg = u.kbeg;
+          pr.kend = u.kend;
+          pr.part = p;
+          out.pairs.push_back(pr);
+        } else {
+          out.pairs.back().slot[1] = static_cast<int32_t>(out.fwd.size());
+        }
         out.fwd.push_back(u);
       }
       // backward: key tiles below the sample's largest anchor
@@ -289,6 +307,7 @@ void make_lists(const Prob& q, const std::vector<SampleAnchors>& sa, Built& out)
     }
   }
   out.fwd_part_off[q.P] = static_cast<int32_t>(out.fwd.size());
+  out.pair_off[q.P] = static_cast<int32_t>(out.pairs.size());
   out.bwd_part_off[q.P] = static_cast<int32_t>(out.bwd.size());
 
   // merge lists: per (query tile, kv head), forward units in ascending key order
@@ -348,6 +367,7 @@ PlanHeader layout_of(const Prob& q, int policy, const Built& b) {
   h.n_mtiles = static_cast<int64_t>(b.mtiles.size());
   h.n_fwd = static_cast<int64_t>(b.fwd.size());
   h.n_bwd = static_cast<int64_t>(b.bwd.size());
+  h.n_fwd_pairs = static_cast<int64_t>(b.pairs.size());
   h.imbalance = b.imbalance;
   uint64_t off = align_up(sizeof(PlanHeader), 256);
   h.items_off = off;
@@ -363,6 +383,8 @@ PlanHeader layout_of(const Prob& q, int policy, const Built& b) {
   h.dev.tok_kend = put(b.tok_kend.size() * sizeof(int32_t));
   h.dev.fwd_units = put(b.fwd.size() * sizeof(FwdUnit));
   h.dev.fwd_part_off = put(b.fwd_part_off.size() * sizeof(int32_t));
+  h.dev.fwd_pairs = put(b.pairs.size() * sizeof(FwdPair));
+  h.dev.fwd_pair_off = put(b.pair_off.size() * sizeof(int32_t));
   h.dev.merge_off = put(b.merge_off.size() * sizeof(int32_t));
   h.dev.merge_list = put(b.merge_list.size() * sizeof(int32_t));
   h.dev.bwd_units = put(b.bwd.size() * sizeof(BwdUnit));
@@ -417,6 +439,8 @@ extern "C" int skv_plan(const skv_problem* prob, int policy, void* plan, size_t 
   copy_to(dev, h.dev.tok_kend, b.tok_kend);
   copy_to(dev, h.dev.fwd_units, b.fwd);
   copy_to(dev, h.dev.fwd_part_off, b.fwd_part_off);
+  copy_to(dev, h.dev.fwd_pairs, b.pairs);
+  copy_to(dev, h.dev.fwd_pair_off, b.pair_off);
   copy_to(dev, h.dev.merge_off, b.merge_off);
   copy_to(dev, h.dev.merge_list, b.merge_list);
   copy_to(dev, h.dev.bwd_units, b.bwd);

@@ -34,6 +34,17 @@ struct FwdUnit {
   int32_t pad0, pad1;
 };
 
+// Forward pair: two forward units (slots) of one item, processed together by
+// one CTA that shares every K/V tile between the two query tiles. slot[1] is
+// -1 when the item has an odd number of live query tiles.
+struct FwdPair {
+  int32_t slot[2];
+  int32_t kbeg;  // key range covering both slots
+  int32_t kend;
+  int32_t part;
+  int32_t pad;
+};
+
 // Backward unit: one tile of <= 128 keys of one item, against every query
 // tile of the sample whose kmax exceeds kbeg.
 struct BwdUnit {
@@ -53,6 +64,8 @@ struct DevSection {
   uint64_t tok_kend;      // int32[Nq]: absolute key end of every query token
   uint64_t fwd_units;     // FwdUnit[n_fwd]
   uint64_t fwd_part_off;  // int32[P+1]: units of partition p are [off[p], off[p+1])
+  uint64_t fwd_pairs;     // FwdPair[n_fwd_pairs]
+  uint64_t fwd_pair_off;  // int32[P+1]: pairs of partition p are [off[p], off[p+1])
   uint64_t merge_off;     // int32[n_mtiles * Hkv + 1]
   uint64_t merge_list;    // int32[n_fwd]: fwd unit ids per (tile, kv head), ascending kbeg
   uint64_t bwd_units;     // BwdUnit[n_bwd]
@@ -70,6 +83,7 @@ struct PlanHeader {
   int64_t Nq, Ltot;
   int64_t total_cost;
   int64_t n_items, n_mtiles, n_fwd, n_bwd;
+  int64_t n_fwd_pairs;
   double imbalance;
   uint64_t fingerprint;  // hash of the problem (shapes, offsets, anchors)
   // host-side arrays, offsets from the start of the plan buffer
