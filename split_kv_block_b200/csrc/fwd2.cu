@@ -298,21 +298,24 @@ __global__ void __launch_bounds__(384, 1)
         ++s_cnt;
         tc_fence_after();
         const int lim_c = row_end - (pr.kbeg + j * kTileN);  // valid columns of this row in the tile
-        // pass 1: row maximum of the scaled scores
-        float tmax = -INFINITY;
+        // the whole row of S in registers: four loads in flight, one wait
+        uint32_t sv[128];
 #pragma unroll
-        for (int cc = 0; cc < 128; cc += 32) {
-          uint32_t v[32];
-          tmem_ld32(tS + cc, v);
-          tmem_wait_ld();
-          if (lim_c >= cc + 32) {
+        for (int cc = 0; cc < 128; cc += 32)
+          tmem_ld32(tS + cc, *reinterpret_cast<uint32_t(*)[32]>(&sv[cc]));
+        tmem_wait_ld();
+        if (lim_c < 128) {  // masked keys of this row: -inf
 #pragma unroll
-            for (int i = 0; i < 32; ++i) tmax = fmaxf(tmax, __uint_as_float(v[i]));
-          } else {
-#pragma unroll
-            for (int i = 0; i < 32; ++i) tmax = fmaxf(tmax, (cc + i < lim_c) ? __uint_as_float(v[i]) : -INFINITY);
-          }
+          for (int i = 0; i < 128; ++i)
+            if (i >= lim_c) sv[i] = __float_as_uint(-INFINITY);
         }
+        // row maximum with eight independent partial maxima (a single chain is latency-bound)
+        float mx[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) mx[k] = -INFINITY;
+#pragma unroll
+        for (int i = 0; i < 128; ++i) mx[i & 7] = fmaxf(mx[i & 7], __uint_as_float(sv[i]));
+        float tmax = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])), fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
         tmax *= sl2;  // sl2 > 0: scaling commutes with the maximum
         // lazy reference update: move only when the tile maximum exceeds it by more than 2^8
         const bool move = tmax > m_ref + 8.f;
@@ -334,28 +337,30 @@ __global__ void __launch_bounds__(384, 1)
         }
         m_ref = m_new;
         const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
-        // pass 2: P = 2^(s sl2 - m_ref), packed to bf16 over the columns already read
-        float rs = 0.f;
+        // P = 2^(s sl2 - m_ref) (masked entries are -inf -> 0), bf16 pairs over the first 64 columns of S.
+        // Four independent row sums. The exponentials and the bf16 packing share the special-function
+        // pipe (one warp instruction per 8 cycles per SM quarter), which bounds this loop; moving part
+        // of either to the FMA / integer pipes measured slower here.
+        float rs[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int cc = 0; cc < 128; cc += 32) {
-          uint32_t v[32];
-          tmem_ld32(tS + cc, v);
-          tmem_wait_ld();
           uint32_t pk[16];
 #pragma unroll
-          for (int i = 0; i < 32; i += 2) {
-            float x0 = ex2(fmaf(__uint_as_float(v[i]), sl2, -m_use));
-            float x1 = ex2(fmaf(__uint_as_float(v[i + 1]), sl2, -m_use));
-            if (lim_c < cc + 32) {
-              x0 = (cc + i < lim_c) ? x0 : 0.f;
-              x1 = (cc + i + 1 < lim_c) ? x1 : 0.f;
-            }
-            rs += x0 + x1;
-            pk[i >> 1] = pack_bf16(x0, x1);
+          for (int i = 0; i < 32; i += 4) {
+            const float x0 = ex2(fmaf(__uint_as_float(sv[cc + i]), sl2, -m_use));
+            const float x1 = ex2(fmaf(__uint_as_float(sv[cc + i + 1]), sl2, -m_use));
+            const float x2 = ex2(fmaf(__uint_as_float(sv[cc + i + 2]), sl2, -m_use));
+            const float x3 = ex2(fmaf(__uint_as_float(sv[cc + i + 3]), sl2, -m_use));
+            rs[0] += x0;
+            rs[1] += x1;
+            rs[2] += x2;
+            rs[3] += x3;
+            pk[(i >> 1) + 0] = pack_bf16(x0, x1);
+            pk[(i >> 1) + 1] = pack_bf16(x2, x3);
           }
           tmem_st16(tS + (cc >> 1), pk);
         }
-        l += rs;
+        l += (rs[0] + rs[1]) + (rs[2] + rs[3]);
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(&c.p_full[t]);
