@@ -7,6 +7,7 @@
 #include <cmath>
 #include <cstring>
 #include <mutex>
+#include <vector>
 
 #include "kernels.h"
 #include "plan_layout.h"
@@ -51,6 +52,7 @@ constexpr int kSlots = 4;
 std::mutex g_stage_mu;
 Staging g_stage[kSlots];
 int g_stage_next = 0;
+std::vector<void*> g_retired;  // outgrown staging buffers, released with the process
 
 int upload(const void* src, size_t n, void* dst, cudaStream_t stream) {
   std::lock_guard<std::mutex> lock(g_stage_mu);
@@ -67,12 +69,18 @@ int upload(const void* src, size_t n, void* dst, cudaStream_t stream) {
     if (e != cudaSuccess) return cuda_fail(e);
   }
   if (s.cap < n) {
-    if (s.host) cudaFreeHost(s.host);
-    s.host = nullptr;
-    s.cap = 0;
-    e = cudaHostAlloc(&s.host, n, cudaHostAllocDefault);
+    // Grow geometrically and keep the old buffer until exit: cudaFreeHost
+    // synchronizes the device, which would stall the caller's pipeline
+    // whenever a larger plan arrives (plans change size every step when the
+    // anchors are redrawn).
+    size_t cap = size_t(1) << 20;
+    while (cap < n) cap <<= 1;
+    void* fresh = nullptr;
+    e = cudaHostAlloc(&fresh, cap, cudaHostAllocDefault);
     if (e != cudaSuccess) return cuda_fail(e);
-    s.cap = n;
+    if (s.host) g_retired.push_back(s.host);
+    s.host = fresh;
+    s.cap = cap;
   }
   std::memcpy(s.host, src, n);
   e = cudaMemcpyAsync(dst, s.host, n, cudaMemcpyHostToDevice, stream);

@@ -140,3 +140,38 @@ def test_ctx32k_two_groups():
     """The 32K workload at full size; oracle on 2 of the 8 kv-head groups."""
     prob = synth.make_problem(synth.WORKLOADS["ctx32k"], seed=0)
     _case(prob, groups=(0, 5))
+
+
+def _one_sample(prob, b, q, k, v, do, o, lse, grads):
+    """Sub-problem of sample b alone (its tokens, its context) with the matching
+    slices of inputs and GPU outputs; exact, samples are independent."""
+    S = prob.block_q
+    j0, j1 = int(prob.anchor_offsets[b]), int(prob.anchor_offsets[b + 1])
+    k0, k1 = int(prob.ctx_offsets[b]), int(prob.ctx_offsets[b + 1])
+    t0, t1 = j0 * S, j1 * S
+    sub = prob.replace(ctx_offsets=np.array([0, k1 - k0], dtype=np.int64),
+                       anchor_offsets=np.array([0, j1 - j0], dtype=np.int32), anchors=prob.anchors[j0:j1].copy())
+    dq, dk, dv = grads
+    return (sub, q[t0:t1], k[k0:k1], v[k0:k1], do[t0:t1], o[t0:t1], lse[t0:t1],
+            (dq[t0:t1], dk[k0:k1], dv[k0:k1]))
+
+
+def test_ctx128k_full_size_one_group():
+    """The 128K Beta(5,1) workload at full size with 4 key sub-chunks per chunk
+    (the <= 1% imbalance granularity); oracle on one kv-head group."""
+    prob = synth.make_problem(synth.WORKLOADS["ctx128k"], seed=0, sub_chunks=4)
+    _case(prob, groups=(3,))
+
+
+def test_batch8_full_size_one_sample_one_group():
+    """The batched workload (8 samples, contexts 8K-256K) at full size with
+    fresh anchors; oracle on one sample and one kv-head group."""
+    w = synth.WORKLOADS["batch8_logu"]
+    prob = synth.redraw_anchors(synth.make_problem(w, seed=0), w, seed=11)
+    q, k, v, do = synth.make_tensors(prob, seed=0, backward=True)
+    o, lse, grads, plan = run_gpu(prob, q, k, v, do)
+    lens = np.diff(prob.ctx_offsets)
+    b = int(np.argsort(lens)[len(lens) // 2])  # a mid-sized sample
+    sub, qs, ks, vs, dos, os_, ls, gs = _one_sample(prob, b, q, k, v, do, o, lse, grads)
+    check_forward(sub, qs, ks, vs, os_, ls, groups=(6,))
+    check_backward(sub, qs, ks, vs, dos, gs, groups=(6,))
