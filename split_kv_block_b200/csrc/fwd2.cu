@@ -58,6 +58,54 @@ __device__ __forceinline__ uint64_t kmaj(int ks) {
   return static_cast<uint64_t>(((ks >> 2) * 16384 + (ks & 3) * 32) >> 4);
 }
 
+// Maximum of a 128-column score row: eight independent three-input chains.
+__device__ __forceinline__ float row_max(const uint32_t (&sv)[128]) {
+  float mx[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) mx[k] = -INFINITY;
+#pragma unroll
+  for (int i = 0; i < 128; i += 2) mx[(i >> 1) & 7] = fmax3(mx[(i >> 1) & 7], __uint_as_float(sv[i]), __uint_as_float(sv[i + 1]));
+  return fmaxf(fmax3(mx[0], mx[1], mx[2]), fmax3(fmax3(mx[3], mx[4], mx[5]), mx[6], mx[7]));
+}
+
+// P = 2^(s sl2 - m_use) over one score row (masked entries are -inf -> 0), stored as bf16
+// pairs into the first 64 TMEM columns at tS; returns the row sum (four independent sums).
+// With kMax it also returns, in raw_max, the maximum of the raw scores: the three-input
+// maxima go to the ALU pipe, idle while the exponentials hold the special-function pipe
+// (one warp instruction per 8 cycles per SM quarter, the bound of this loop).
+template <bool kMax>
+__device__ __forceinline__ float exp_row(const uint32_t (&sv)[128], float sl2, float m_use, uint32_t tS,
+                                         float& raw_max) {
+  float rs[4] = {0.f, 0.f, 0.f, 0.f};
+  float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+  for (int cc = 0; cc < 128; cc += 32) {
+    uint32_t pk[16];
+#pragma unroll
+    for (int i = 0; i < 32; i += 4) {
+      const float s0 = __uint_as_float(sv[cc + i]), s1 = __uint_as_float(sv[cc + i + 1]);
+      const float s2 = __uint_as_float(sv[cc + i + 2]), s3 = __uint_as_float(sv[cc + i + 3]);
+      if (kMax) {
+        mx[(i >> 2) & 1] = fmax3(mx[(i >> 2) & 1], s0, s1);
+        mx[2 + ((i >> 2) & 1)] = fmax3(mx[2 + ((i >> 2) & 1)], s2, s3);
+      }
+      const float x0 = ex2(fmaf(s0, sl2, -m_use));
+      const float x1 = ex2(fmaf(s1, sl2, -m_use));
+      const float x2 = ex2(fmaf(s2, sl2, -m_use));
+      const float x3 = ex2(fmaf(s3, sl2, -m_use));
+      rs[0] += x0;
+      rs[1] += x1;
+      rs[2] += x2;
+      rs[3] += x3;
+      pk[(i >> 1) + 0] = pack_bf16(x0, x1);
+      pk[(i >> 1) + 1] = pack_bf16(x2, x3);
+    }
+    tmem_st16(tS + (cc >> 1), pk);
+  }
+  if (kMax) raw_max = fmaxf(fmax3(mx[0], mx[1], mx[2]), mx[3]);
+  return (rs[0] + rs[1]) + (rs[2] + rs[3]);
+}
+
 __global__ void __launch_bounds__(384, 1)
     fwd2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                 const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
@@ -309,58 +357,40 @@ __global__ void __launch_bounds__(384, 1)
           for (int i = 0; i < 128; ++i)
             if (i >= lim_c) sv[i] = __float_as_uint(-INFINITY);
         }
-        // row maximum with eight independent partial maxima (a single chain is latency-bound)
-        float mx[8];
-#pragma unroll
-        for (int k = 0; k < 8; ++k) mx[k] = -INFINITY;
-#pragma unroll
-        for (int i = 0; i < 128; ++i) mx[i & 7] = fmaxf(mx[i & 7], __uint_as_float(sv[i]));
-        float tmax = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])), fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
-        tmax *= sl2;  // sl2 > 0: scaling commutes with the maximum
-        // lazy reference update: move only when the tile maximum exceeds it by more than 2^8
-        const bool move = tmax > m_ref + 8.f;
-        const float m_new = move ? tmax : m_ref;
-        const float alpha = move ? ex2(m_ref - m_new) : 1.f;  // m_ref = -inf -> 0
-        l *= alpha;
-        if (__any_sync(0xffffffffu, move && j > 0)) {
-          // PV of step j-1 completed before this step's S was issued
+        // Lazy reference maximum m_ref (log2 units): it moves only when a tile maximum exceeds it by
+        // more than 8, so every P is at most 2^8 and O is rarely rescaled. sl2 > 0, so scaling
+        // commutes with the maximum.
+        float raw;
+        if (j == 0) {
+          // first tile of the unit: the reference is this tile's maximum (-inf for a row without keys)
+          m_ref = row_max(sv) * sl2;
+          l = exp_row<false>(sv, sl2, m_ref == -INFINITY ? 0.f : m_ref, tS, raw);
+        } else {
+          // later tiles: exponentials against the current reference, the tile maximum alongside;
+          // the pass is redone only for a tile whose maximum moves the reference
+          const float add = exp_row<true>(sv, sl2, m_ref == -INFINITY ? 0.f : m_ref, tS, raw);
+          const float tmax = raw * sl2;
+          const bool move = tmax > m_ref + 8.f;
+          if (__any_sync(0xffffffffu, move)) {
+            const float m_new = move ? tmax : m_ref;
+            const float alpha = move ? ex2(m_ref - m_new) : 1.f;  // m_ref = -inf -> 0
+            // PV of step j-1 completed before this step's S was issued
 #pragma unroll 1
-          for (int cc = 0; cc < kD; cc += 32) {
-            uint32_t v[32];
-            tmem_ld32(tO + cc, v);
-            tmem_wait_ld();
+            for (int cc = 0; cc < kD; cc += 32) {
+              uint32_t v[32];
+              tmem_ld32(tO + cc, v);
+              tmem_wait_ld();
 #pragma unroll
-            for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * alpha);
-            tmem_st32(tO + cc, v);
+              for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * alpha);
+              tmem_st32(tO + cc, v);
+            }
+            tmem_wait_st();  // also orders the first pass's P stores before the rewrite
+            m_ref = m_new;
+            l = l * alpha + exp_row<false>(sv, sl2, m_ref == -INFINITY ? 0.f : m_ref, tS, raw);
+          } else {
+            l += add;
           }
-          tmem_wait_st();
         }
-        m_ref = m_new;
-        const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
-        // P = 2^(s sl2 - m_ref) (masked entries are -inf -> 0), bf16 pairs over the first 64 columns of S.
-        // Four independent row sums. The exponentials and the bf16 packing share the special-function
-        // pipe (one warp instruction per 8 cycles per SM quarter), which bounds this loop; moving part
-        // of either to the FMA / integer pipes measured slower here.
-        float rs[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int cc = 0; cc < 128; cc += 32) {
-          uint32_t pk[16];
-#pragma unroll
-          for (int i = 0; i < 32; i += 4) {
-            const float x0 = ex2(fmaf(__uint_as_float(sv[cc + i]), sl2, -m_use));
-            const float x1 = ex2(fmaf(__uint_as_float(sv[cc + i + 1]), sl2, -m_use));
-            const float x2 = ex2(fmaf(__uint_as_float(sv[cc + i + 2]), sl2, -m_use));
-            const float x3 = ex2(fmaf(__uint_as_float(sv[cc + i + 3]), sl2, -m_use));
-            rs[0] += x0;
-            rs[1] += x1;
-            rs[2] += x2;
-            rs[3] += x3;
-            pk[(i >> 1) + 0] = pack_bf16(x0, x1);
-            pk[(i >> 1) + 1] = pack_bf16(x2, x3);
-          }
-          tmem_st16(tS + (cc >> 1), pk);
-        }
-        l += (rs[0] + rs[1]) + (rs[2] + rs[3]);
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(&c.p_full[t]);
