@@ -181,6 +181,7 @@ def run_gpu(args, rank, world, local_rank):
     Nq, Hq, d = prob.num_tokens_q, prob.num_q_heads, prob.head_dim
     o = torch.empty(Nq, Hq, d, dtype=torch.bfloat16, device=dev)
     lse = torch.empty(Nq, Hq, dtype=torch.float32, device=dev)
+    dq = dk = dv = None
     if backward:
         dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
     flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)  # > 126 MB L2
@@ -272,6 +273,8 @@ def run_gpu(args, rank, world, local_rank):
     lpt = skv.skv_plan(p0, skv.SKV_PLAN_LPT).stats()["imbalance"]
     static = skv.skv_plan(p0, skv.SKV_PLAN_STATIC).stats()["imbalance"]
 
+    realized = realized_busy_imbalance(skv, p0, policy, q, k, v, do, ws, o, lse, dq, dk, dv, stream, dev)
+
     peaks = load_peaks()
     dom = skv.SKV_KERNEL_BWD if backward else skv.SKV_KERNEL_FWD
     dom_t = statistics.mean(t_kern[dom])
@@ -293,6 +296,8 @@ def run_gpu(args, rank, world, local_rank):
         "roofline": {"bound": "tensor", "kernel": "bwd_kernel" if backward else "fwd_kernel",
                      "achieved": round(achieved, 2), "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                      "frac": round(achieved / peaks["bf16_tflops"], 4),
+                     "frac_of_sustained": (round(achieved / peaks["bf16_tflops_sustained"], 4)
+                                           if peaks.get("bf16_tflops_sustained") else None),
                      "traffic": profiled_traffic("bwd_kernel" if backward else "fwd_kernel", args.workload),
                      "peak_source": f"{peaks['source']} bf16 dense (burst)",
                      "step_frac": round(roof_step / (total / K), 4)},
@@ -300,7 +305,7 @@ def run_gpu(args, rank, world, local_rank):
                       "merge": round(statistics.mean(t_kern[skv.SKV_KERNEL_MERGE]) * 1e3, 4),
                       "bwd": round(statistics.mean(t_kern[skv.SKV_KERNEL_BWD]) * 1e3, 4) if backward else None},
         "context_tokens_per_s": round(ctx_tokens / total, 1),
-        "imbalance": {"lpt": lpt, "static": static},
+        "imbalance": {"lpt": lpt, "static": static, "realized": realized},
         "planner_us": round(statistics.median(planner_s) * 1e6, 1),
         "gpu_launches": kernels_per_step * K,
         "clocks": clocks.summary(),
@@ -308,6 +313,48 @@ def run_gpu(args, rank, world, local_rank):
     if not args.no_e2e:
         out["e2e"] = run_e2e(args, prob, step_probs, sizes, policy, q, k, v, do, dev, world)
     return out, prob
+
+
+def realized_busy_imbalance(skv, prob, policy, q, k, v, do, ws, o, lse, dq, dk, dv, stream, dev):
+    """One more (untimed) step with the unit timer on: every work unit's
+    %globaltimer start and end, summed per virtual partition, gives the realized
+    busy time of each partition; its imbalance (max / mean - 1, mean over all P)
+    is the measured counterpart of the plan's LPT imbalance."""
+    backward = do is not None
+    plan = skv.skv_plan(prob, policy)
+    st = plan.stats()
+    n_f, n_b = st["n_fwd_units"], st["n_bwd_units"]
+    fst = torch.zeros(2 * max(n_f, 1), dtype=torch.int64, device=dev)
+    bst = torch.zeros(2 * max(n_b, 1), dtype=torch.int64, device=dev)
+    skv.skv_set_unit_timer(fst, bst if backward else None)
+    try:
+        skv.skv_attn_fwd(plan, q, k, v, ws, stream)
+        skv.skv_lse_merge(plan, ws, o, lse, stream)
+        if backward:
+            skv.skv_attn_bwd(plan, q, k, v, o, lse, do, dq, dk, dv, ws, stream)
+        torch.cuda.synchronize()
+    finally:
+        skv.skv_set_unit_timer(None, None)
+    if skv.skv_status(ws) != 0:
+        raise RuntimeError("device status error in the unit-timer step")
+    fp, bp = plan.unit_partitions()
+    P = prob.num_partitions
+
+    def busy(stamps, parts, n):
+        s = stamps.cpu().numpy()[:2 * n].reshape(n, 2).astype(np.float64)
+        return np.bincount(parts, weights=s[:, 1] - s[:, 0], minlength=P)
+
+    def imb(x):
+        return round(float(x.max() / x.mean() - 1.0), 5) if x.mean() > 0 else None
+
+    bf = busy(fst, fp, n_f)
+    out = {"fwd": imb(bf)}
+    if backward:
+        bb = busy(bst, bp, n_b)
+        out["bwd"] = imb(bb)
+        out["fwd+bwd"] = imb(bf + bb)
+    out["how"] = "sum of work-unit durations (%globaltimer) per virtual partition, one untimed step"
+    return out
 
 
 def run_e2e(args, prob, step_probs, sizes, policy, q, k, v, do, dev, world):
@@ -414,9 +461,20 @@ def cpu_baseline(prob, backward, seed):
     stride = 1 if per_group_all <= 15.0 else int(math.ceil(per_group_all / 15.0))
     groups = tuple(range(n_groups))
     f, dt, sub = time_oracle(prob, q, k, v, do if backward else None, groups, stride)
+    # a sample shorter than ~10 s (the whole workload fits) is run again until it is not
+    reps = 1
+    while dt < 10.0:
+        f1, dt1, _ = time_oracle(prob, q, k, v, do if backward else None, groups, stride)
+        f, dt, reps = f + f1, dt + dt1, reps + 1
+    from oracle import planner as PL
+    t0 = time.perf_counter()
+    PL.lpt_plan(prob)
+    lpt_s = time.perf_counter() - t0
     return {"value": round(f / dt / 1e12, 6), "unit": "TFLOP/s", "cores": torch.get_num_threads(), "kind": "oracle",
             "sample": f"fp64 oracle fwd{'+bwd' if backward else ''} on {n_groups} of {prob.num_kv_heads} kv-head "
-                      f"groups, every {stride}th anchor ({int(sub.anchor_offsets[-1])} anchors), {dt:.1f} s",
+                      f"groups, every {stride}th anchor ({int(sub.anchor_offsets[-1])} anchors), run {reps}x, "
+                      f"{dt:.1f} s",
+            "lpt_planner_us": round(lpt_s * 1e6, 1),
             "cpu": _cpu_name()}
 
 

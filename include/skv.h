@@ -114,6 +114,18 @@ int skv_plan(const skv_problem* prob, int policy, void* plan, size_t plan_bytes,
 /* Items of a plan in (b, c, g, sub) order; *items points into `plan`. */
 int skv_plan_items(const void* plan, const skv_item** items, size_t* n_items);
 
+/* Virtual partition of every work unit of a plan, in the order the unit
+ * timer (skv_set_unit_timer) indexes its stamps: fwd_part receives
+ * [n_fwd_units] and bwd_part [n_bwd_units] int32 values in [0, P) (host
+ * buffers, caller-owned, sized from skv_plan_stats; either may be NULL).
+ * With the stamps, it gives the realized busy time of each partition: the
+ * measured counterpart of the LPT loads ("Split-KV: Breaking the Context
+ * Parallelism Bottleneck in Diffusion Drafter Training", section "LPT
+ * Scheduling: Load Balancing with Real Attention Costs").
+ * Returns SKV_EINVAL for a NULL plan, SKV_EPLAN for a buffer that is not a
+ * plan of this library version. */
+int skv_plan_unit_partitions(const void* plan, int32_t* fwd_part, int32_t* bwd_part);
+
 /* Scalars of a plan: total cost (sum over items), number of forward work
  * units (item x 128-row query tile pairs with unmasked keys), number of
  * backward work units (item x 128-key tiles with unmasked queries),

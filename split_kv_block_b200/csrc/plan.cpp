@@ -458,6 +458,22 @@ extern "C" int skv_plan_items(const void* plan, const skv_item** items, size_t* 
   return SKV_OK;
 }
 
+extern "C" int skv_plan_unit_partitions(const void* plan, int32_t* fwd_part, int32_t* bwd_part) {
+  if (!plan) return SKV_EINVAL;
+  const PlanHeader* h = static_cast<const PlanHeader*>(plan);
+  if (h->magic != kPlanMagic || h->version != kPlanVersion) return SKV_EPLAN;
+  const uint8_t* dev = static_cast<const uint8_t*>(plan) + h->dev_off;
+  if (fwd_part) {
+    const FwdUnit* u = reinterpret_cast<const FwdUnit*>(dev + h->dev.fwd_units);
+    for (int64_t i = 0; i < h->n_fwd; ++i) fwd_part[i] = u[i].part;
+  }
+  if (bwd_part) {
+    const BwdUnit* u = reinterpret_cast<const BwdUnit*>(dev + h->dev.bwd_units);
+    for (int64_t i = 0; i < h->n_bwd; ++i) bwd_part[i] = u[i].part;
+  }
+  return SKV_OK;
+}
+
 extern "C" int skv_plan_stats(const void* plan, int64_t* total_cost, int64_t* n_fwd_units, int64_t* n_bwd_units,
                               double* imbalance) {
   if (!plan) return SKV_EINVAL;

@@ -21,7 +21,8 @@ SKV_PLAN_LPT = 0
 SKV_PLAN_STATIC = 1
 
 # Every function include/skv.h declares.
-EXPORTS = ("skv_plan_size", "skv_plan", "skv_plan_items", "skv_plan_stats", "skv_attn_fwd", "skv_lse_merge",
+EXPORTS = ("skv_plan_size", "skv_plan", "skv_plan_items", "skv_plan_unit_partitions", "skv_plan_stats", "skv_attn_fwd",
+           "skv_lse_merge",
            "skv_attn_bwd", "skv_status", "skv_strerror", "skv_last_cuda_error", "skv_set_unit_timer",
            "skv_set_timing_events", "skv_attn_fwd_noalloc")
 SKV_NOALLOC_SCRATCH_BYTES = 32 << 20
@@ -60,6 +61,7 @@ def lib() -> ctypes.CDLL:
         L.skv_plan.argtypes = [vp, ctypes.c_int, vp, sz, vp]
         L.skv_plan_items.argtypes = [vp, ctypes.POINTER(vp), ctypes.POINTER(sz)]
         L.skv_plan_stats.argtypes = [vp, vp, vp, vp, vp]
+        L.skv_plan_unit_partitions.argtypes = [vp, vp, vp]
         L.skv_attn_fwd.argtypes = [vp, vp, vp, vp, vp, sz, vp]
         L.skv_lse_merge.argtypes = [vp, vp, vp, vp, vp]
         L.skv_attn_bwd.argtypes = [vp] * 11 + [sz, vp]
@@ -154,6 +156,16 @@ class Plan:
             return np.zeros(0, dtype=ITEM_DTYPE)
         raw = (ctypes.c_uint8 * (n.value * ITEM_DTYPE.itemsize)).from_address(p.value)
         return np.frombuffer(raw, dtype=ITEM_DTYPE).copy()
+
+    def unit_partitions(self):
+        """(forward, backward) int32 arrays: the partition of every work unit, in
+        the order the unit timer indexes its stamps."""
+        st = self.stats()
+        fp = np.zeros(st["n_fwd_units"], dtype=np.int32)
+        bp = np.zeros(st["n_bwd_units"], dtype=np.int32)
+        _check("skv_plan_unit_partitions", lib().skv_plan_unit_partitions(self.ptr, ctypes.c_void_p(fp.ctypes.data),
+                                                                          ctypes.c_void_p(bp.ctypes.data)))
+        return fp, bp
 
     def stats(self) -> dict:
         tc, nf, nb = ctypes.c_int64(), ctypes.c_int64(), ctypes.c_int64()

@@ -116,3 +116,55 @@ def test_library_exports_every_declared_symbol():
     L = skv.lib()
     for name in declared:
         assert hasattr(L, name), name
+
+
+def _expected_unit_counts(prob, items):
+    """Forward / backward work units per partition, counted from the items and
+    the anchors alone: a forward unit is an (item, 128-row query tile) whose
+    tile reaches past the item's first key; a backward unit is a 128-key tile
+    of an item below the sample's largest anchor."""
+    P = prob.num_partitions
+    G = prob.num_q_heads // prob.num_kv_heads
+    tok_per_tile = 128 // G
+    fwd, bwd = np.zeros(P, np.int64), np.zeros(P, np.int64)
+    tiles = {}
+    for b in range(prob.num_samples):
+        j0, j1 = int(prob.anchor_offsets[b]), int(prob.anchor_offsets[b + 1])
+        a = [int(x) for x in prob.anchors[j0:j1]]
+        ntok = (j1 - j0) * prob.block_q
+        base = int(prob.ctx_offsets[b])
+        tiles[b] = [base + max(a[t // prob.block_q] for t in range(t0, min(t0 + tok_per_tile, ntok)))
+                    for t0 in range(0, ntok, tok_per_tile)]
+    for it in items:
+        b, kb, ke, p = int(it["b"]), int(it["key_begin"]), int(it["key_end"]), int(it["partition"])
+        fwd[p] += sum(1 for kmax in tiles[b] if min(ke, kmax) > kb)
+        kmax_b = max(tiles[b]) if tiles[b] else int(prob.ctx_offsets[b])
+        bwd[p] += len(range(kb, min(ke, kmax_b), 128))
+    return fwd, bwd
+
+
+@pytest.mark.parametrize("seed", [0, 1, 2])
+def test_unit_partitions_match_item_partitions(seed):
+    rng = np.random.default_rng(500 + seed)
+    prob = synth.random_small_problem(rng, max_len=3000, max_anchors=9, d=128, heads=((8, 2), (16, 4), (4, 1)))
+    plan = skv.skv_plan(prob)
+    fp, bp = plan.unit_partitions()
+    st = plan.stats()
+    assert len(fp) == st["n_fwd_units"] and len(bp) == st["n_bwd_units"]
+    P = prob.num_partitions
+    assert np.all((fp >= 0) & (fp < P)) and np.all((bp >= 0) & (bp < P))
+    # the work lists are grouped by partition
+    assert np.all(np.diff(fp) >= 0) and np.all(np.diff(bp) >= 0)
+    ef, eb = _expected_unit_counts(prob, plan.items())
+    assert np.bincount(fp, minlength=P).tolist() == ef.tolist()
+    assert np.bincount(bp, minlength=P).tolist() == eb.tolist()
+
+
+def test_unit_partitions_of_the_32k_workload():
+    prob = synth.make_problem(synth.WORKLOADS["ctx32k"], seed=0)
+    plan = skv.skv_plan(prob)
+    fp, bp = plan.unit_partitions()
+    ef, eb = _expected_unit_counts(prob, plan.items())
+    P = prob.num_partitions
+    assert np.bincount(fp, minlength=P).tolist() == ef.tolist()
+    assert np.bincount(bp, minlength=P).tolist() == eb.tolist()
