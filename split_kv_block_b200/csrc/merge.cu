@@ -85,21 +85,48 @@ __global__ void __launch_bounds__(256) merge_kernel(const MergeParams p) {
   const int token = M.tok0 + tl;
   const int h = g * p.G + r % p.G;
   const int c0 = p.merge_off[slot], c1 = p.merge_off[slot + 1];
+  // The lanes fetch the partials' indices and LSEs in parallel (lane i: partials c0 + i, c0 + i + 32, ...),
+  // so the only per-partial memory traffic left in the accumulation loop is the partial output row.
   float m = -INFINITY;
-  for (int c = c0; c < c1; ++c) m = fmaxf(m, p.part_lse[static_cast<size_t>(p.merge_list[c]) * kTileM + r]);
+  for (int c = c0 + lane; c < c1; c += 32) m = fmaxf(m, p.part_lse[static_cast<size_t>(p.merge_list[c]) * kTileM + r]);
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
   float acc[Vec<D>::N] = {};
   float den = 0.f;
   if (m != -INFINITY) {
-    for (int c = c0; c < c1; ++c) {
-      const int u = p.merge_list[c];
-      const float lc = p.part_lse[static_cast<size_t>(u) * kTileM + r];
-      if (lc == -INFINITY) continue;
-      const float w = ex2((lc - m) * kLog2e);
-      float x[Vec<D>::N];
-      load_row<D>(p.part_o + (static_cast<size_t>(u) * kTileM + r) * D, lane, x);
+    for (int base = c0; base < c1; base += 32) {
+      const int cnt = min(32, c1 - base);
+      int my_u = 0;
+      float my_w = 0.f;  // weight exp(LSE_c - m); 0 for a dead partial (LSE = -inf)
+      if (lane < cnt) {
+        my_u = p.merge_list[base + lane];
+        my_w = ex2((p.part_lse[static_cast<size_t>(my_u) * kTileM + r] - m) * kLog2e);
+      }
+      float ws = my_w;
 #pragma unroll
-      for (int i = 0; i < Vec<D>::N; ++i) acc[i] += w * x[i];
-      den += w;
+      for (int off = 16; off > 0; off >>= 1) ws += __shfl_xor_sync(0xffffffffu, ws, off);
+      den += ws;
+      // ascending key order; four independent row loads in flight per step
+      for (int j = 0; j < cnt; j += 4) {
+        float x[4][Vec<D>::N];
+        float w[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const int uk = __shfl_sync(0xffffffffu, my_u, (j + k) & 31);
+          w[k] = __shfl_sync(0xffffffffu, my_w, (j + k) & 31);
+          if (j + k < cnt && w[k] != 0.f) {
+            load_row<D>(p.part_o + (static_cast<size_t>(uk) * kTileM + r) * D, lane, x[k]);
+          } else {
+            w[k] = 0.f;
+#pragma unroll
+            for (int i = 0; i < Vec<D>::N; ++i) x[k][i] = 0.f;
+          }
+        }
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+#pragma unroll
+          for (int i = 0; i < Vec<D>::N; ++i) acc[i] += w[k] * x[k][i];
+      }
     }
   }
   const float inv = den > 0.f ? 1.f / den : 0.f;
