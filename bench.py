@@ -57,6 +57,37 @@ def load_peaks():
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
 
 
+def rank_problem(args, rank):
+    """Replicas: every rank runs its own independent problem of the workload,
+    seeded seed + rank (no data is shared between ranks)."""
+    seed = args.seed + rank
+    return seed, synth.make_problem(synth.WORKLOADS[args.workload], seed=seed, sub_chunks=args.sub_chunks)
+
+
+def max_over_ranks(seconds, world, device):
+    """The job's time: the maximum of the ranks' device times (all ranks call it)."""
+    if world <= 1:
+        return seconds
+    t = torch.tensor([seconds], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(x, world, device):
+    """Sum of a per-rank quantity over all ranks (all ranks call it)."""
+    if world <= 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.SUM)
+    return float(t.item())
+
+
+def job_value(flops_all_ranks, seconds):
+    """Whole-job throughput in TFLOP/s: the work all ranks processed (their
+    problems differ, seed + rank) over the max-over-ranks time."""
+    return flops_all_ranks / seconds / 1e12
+
+
 def flops_of(prob, backward=True):
     """Unmasked work: 4 d block_q Hq sum(a) forward, 2.5x that backward."""
     f_fwd = 4.0 * prob.head_dim * prob.block_q * prob.num_q_heads * float(np.sum(prob.anchors))
@@ -161,8 +192,7 @@ def run_gpu(args, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     w = synth.WORKLOADS[args.workload]
-    seed = args.seed + rank
-    prob = synth.make_problem(w, seed=seed, sub_chunks=args.sub_chunks)
+    seed, prob = rank_problem(args, rank)
     backward = w.backward
     q, k, v, do = synth.make_tensors(prob, seed=seed, backward=backward)
     q, k, v = q.to(dev), k.to(dev), v.to(dev)
@@ -252,11 +282,7 @@ def run_gpu(args, rank, world, local_rank):
         raise RuntimeError(f"device status {status} after the timed steps")
     t_steps = [ev[0][0].elapsed_time(ev[0][1]) / 1e3] if stream_mode else [a.elapsed_time(b) / 1e3 for a, b in ev]
     t_kern = {kid: [a.elapsed_time(b) / 1e3 for a, b in lst] for kid, lst in kev.items()}
-    total = sum(t_steps)
-    if world > 1:
-        tt = torch.tensor([total], dtype=torch.float64, device=dev)
-        torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
-        total = float(tt.item())
+    total = max_over_ranks(sum(t_steps), world, dev)
 
     f_fwd_all, f_bwd_all = 0.0, 0.0
     for i in range(K):
@@ -264,9 +290,8 @@ def run_gpu(args, rank, world, local_rank):
         f_fwd_all += a
         f_bwd_all += b
     flops_rank = f_fwd_all + f_bwd_all
-    flops_job = flops_rank * world
-    value = flops_job / total / 1e12
-    ctx_tokens = float(prob.num_tokens_kv) * K * world
+    value = job_value(sum_over_ranks(flops_rank, world, dev), total)
+    ctx_tokens = sum_over_ranks(float(prob.num_tokens_kv) * K, world, dev)
 
     # plan quality (LPT vs static) on this step's problem
     p0 = step_probs[args.warmup]
@@ -404,12 +429,8 @@ def run_e2e(args, prob, step_probs, sizes, policy, q, k, v, do, dev, world):
             times.append(a.elapsed_time(b) / 1e3)
             ff, fb = flops_of(p, backward)
             flops += ff + fb
-    total = sum(times)
-    if world > 1:
-        tt = torch.tensor([total], dtype=torch.float64, device=dev)
-        torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
-        total = float(tt.item())
-    return {"value": round(flops * world / total / 1e12, 4), "unit": "TFLOP/s", "h2d_bytes_per_step": int(h2d),
+    total = max_over_ranks(sum(times), world, dev)
+    return {"value": round(job_value(sum_over_ranks(flops, world, dev), total), 4), "unit": "TFLOP/s", "h2d_bytes_per_step": int(h2d),
             "d2h_bytes_per_step": int(d2h), "steps": n, "ms_per_step": round(total / n * 1e3, 3)}
 
 

@@ -251,32 +251,6 @@ __device__ __forceinline__ float lg2(float x) {
   return y;
 }
 
-// 2^x evaluated on the FMA and integer pipes, leaving the special-function
-// unit to other work. Method: Cody-Waite range reduction (W. J. Cody and
-// W. Waite, "Software Manual for the Elementary Functions", 1980): x = n + f
-// with n = round(x) and |f| <= 1/2; 2^f from a degree-3 polynomial whose
-// coefficients were fitted here for minimal maximum relative error on
-// [-1/2, 1/2] (7.5e-5, evaluated in fp32); 2^n by adding n to the exponent
-// field. n = round(x) comes from adding 1.5 * 2^23, which leaves round(x) in
-// the low mantissa bits. Valid for x <= 0 as used by softmax; inputs below
-// -126 return values below 2^-125 (treated as zero by the callers' bf16 use).
-__device__ __forceinline__ float exp2_poly(float x) {
-  x = fmaxf(x, -126.f);
-  const float t = x + 12582912.f;
-  const float n = t - 12582912.f;
-  const float f = x - n;
-  float p = fmaf(0.0551716685f, f, 0.2426111400f);
-  p = fmaf(p, f, 0.6932609677f);
-  p = fmaf(p, f, 0.9999280572f);
-  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
-}
-
-// Two floats to packed bf16 on the integer pipe: the upper 16 bits after
-// adding half an ulp (ties round away from zero; otherwise round-to-nearest).
-__device__ __forceinline__ uint32_t pack_bf16_alu(float lo, float hi) {
-  return __byte_perm(__float_as_uint(lo) + 0x8000u, __float_as_uint(hi) + 0x8000u, 0x7632);
-}
-
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
