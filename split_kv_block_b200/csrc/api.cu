@@ -7,6 +7,7 @@
 #include <cmath>
 #include <cstring>
 #include <mutex>
+#include <algorithm>
 #include <vector>
 
 #include "kernels.h"
@@ -141,9 +142,8 @@ bool aligned16(const void* p) { return reinterpret_cast<uintptr_t>(p) % 16 == 0;
 
 // Device plan copy + zeroed control block and queue counters.
 int prepare_ws(const PlanHeader& h, const void* plan, void* ws, const WsLayout& w, cudaStream_t stream) {
-  cudaError_t e = cudaMemsetAsync(ws, 0, 256, stream);  // status word
-  if (e != cudaSuccess) return cuda_fail(e);
-  e = cudaMemsetAsync(at<uint8_t>(ws, w.counters), 0, 2 * sizeof(int32_t) * static_cast<size_t>(h.P), stream);
+  // status word and queue counters: one contiguous control block
+  cudaError_t e = cudaMemsetAsync(at<uint8_t>(ws, w.status), 0, w.control, stream);
   if (e != cudaSuccess) return cuda_fail(e);
   if (h.dev.bytes > 0) return upload(static_cast<const uint8_t*>(plan) + h.dev_off, h.dev.bytes, at<uint8_t>(ws, w.dev), stream);
   return SKV_OK;
@@ -277,22 +277,17 @@ extern "C" int skv_attn_bwd(const void* plan, const void* q, const void* k, cons
   int rc = prepare_ws(*h, plan, ws, w, stream);
   if (rc != SKV_OK) return rc;
   cudaError_t e;
-  // keys no query attends to: zero gradients
-  const int64_t* dead = at<int64_t>(plan, h->dead_off);
-  const size_t row_bytes = static_cast<size_t>(h->Hkv) * h->d * 2;
-  for (int b = 0; b < h->B; ++b) {
-    const int64_t k0 = dead[2 * b], k1 = dead[2 * b + 1];
-    if (k1 <= k0) continue;
-    e = cudaMemsetAsync(static_cast<uint8_t*>(dk) + k0 * row_bytes, 0, (k1 - k0) * row_bytes, stream);
-    if (e != cudaSuccess) return cuda_fail(e);
-    e = cudaMemsetAsync(static_cast<uint8_t*>(dv) + k0 * row_bytes, 0, (k1 - k0) * row_bytes, stream);
-    if (e != cudaSuccess) return cuda_fail(e);
-  }
   float* delta = at<float>(ws, w.bwd_delta);
   float* dq_acc = at<float>(ws, w.bwd_dq);
   const long long n_rows = h->Nq * h->Hq;
+  // D, the zeroed dQ accumulator, and zero dK/dV for the keys no query attends to (the plan's
+  // dead ranges, in the device section) in one launch
+  int64_t dead_rows = 0;
+  const int64_t* dead = at<int64_t>(plan, h->dead_off);
+  for (int b = 0; b < h->B; ++b) dead_rows += std::max<int64_t>(0, dead[2 * b + 1] - dead[2 * b]);
   e = launch_bwd_prep(h->d, static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dout), delta,
-                      dq_acc, n_rows, stream);
+                      dq_acc, n_rows, at<int64_t>(at<uint8_t>(ws, w.dev), h->dev.dead), h->B, dead_rows,
+                      static_cast<__nv_bfloat16*>(dk), static_cast<__nv_bfloat16*>(dv), h->Hkv, stream);
   if (e != cudaSuccess) return cuda_fail(e);
   if (h->n_bwd > 0) {
     CUtensorMap tq, tk, tv, tdo;

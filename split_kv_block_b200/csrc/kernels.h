@@ -69,8 +69,11 @@ int fwd2_smem_bytes();
 // CTAs of the forward launch: one per SM, at most one per work unit (pair for head_dim 128)
 int fwd_grid(int d, int sms, long long n_units, long long n_pairs);
 cudaError_t launch_merge(int d, const MergeParams& p, cudaStream_t stream);
+// D = rowsum(dO * O) and the zeroed dQ accumulator per (token, head) row; also zeroes dK/dV of
+// the keys no query attends to (dead[2b] .. dead[2b+1] of every sample, device array).
 cudaError_t launch_bwd_prep(int d, const __nv_bfloat16* o, const __nv_bfloat16* dout, float* delta, float* dq_acc,
-                            long long n_rows, cudaStream_t stream);
+                            long long n_rows, const int64_t* dead, int n_samples, int64_t dead_rows,
+                            __nv_bfloat16* dk, __nv_bfloat16* dv, int hkv, cudaStream_t stream);
 cudaError_t launch_bwd(int d, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                        const CUtensorMap& tdo, const BwdParams& p, int grid, cudaStream_t stream);
 cudaError_t launch_bwd2(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tdo,

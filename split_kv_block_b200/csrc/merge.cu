@@ -138,8 +138,28 @@ __global__ void __launch_bounds__(256) merge_kernel(const MergeParams p) {
 
 // D = rowsum(dO * O) per (token, head); zeroes that row of the dQ accumulator.
 template <int D>
+// Blocks [0, main_blocks): one warp per row. Blocks past them zero the dead key ranges of dK and
+// dV, 16 bytes per thread per step.
 __global__ void __launch_bounds__(256) bwd_prep_kernel(const __nv_bfloat16* o, const __nv_bfloat16* dout,
-                                                       float* delta, float* dq_acc, long long n_rows) {
+                                                       float* delta, float* dq_acc, long long n_rows,
+                                                       unsigned main_blocks, const int64_t* dead, int n_samples,
+                                                       long long row_chunks, uint4* dk, uint4* dv) {
+  if (blockIdx.x >= main_blocks) {
+    const long long zid = static_cast<long long>(blockIdx.x - main_blocks) * blockDim.x + threadIdx.x;
+    const long long zstride = static_cast<long long>(gridDim.x - main_blocks) * blockDim.x;
+    for (int b = 0; b < n_samples; ++b) {
+      const long long k0 = dead[2 * b], k1 = dead[2 * b + 1];
+      if (k1 <= k0) continue;
+      const long long n = (k1 - k0) * row_chunks;
+      uint4* zk = dk + k0 * row_chunks;
+      uint4* zv = dv + k0 * row_chunks;
+      for (long long i = zid; i < n; i += zstride) {
+        zk[i] = make_uint4(0u, 0u, 0u, 0u);
+        zv[i] = make_uint4(0u, 0u, 0u, 0u);
+      }
+    }
+    return;
+  }
   const long long row = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (row >= n_rows) return;
@@ -184,13 +204,22 @@ cudaError_t launch_merge(int d, const MergeParams& p, cudaStream_t stream) {
 }
 
 cudaError_t launch_bwd_prep(int d, const __nv_bfloat16* o, const __nv_bfloat16* dout, float* delta, float* dq_acc,
-                            long long n_rows, cudaStream_t stream) {
-  if (n_rows == 0) return cudaSuccess;
-  const long long blocks = (n_rows * 32 + 255) / 256;
+                            long long n_rows, const int64_t* dead, int n_samples, int64_t dead_rows,
+                            __nv_bfloat16* dk, __nv_bfloat16* dv, int hkv, cudaStream_t stream) {
+  const long long main_blocks = (n_rows * 32 + 255) / 256;
+  const long long row_chunks = static_cast<long long>(hkv) * d * 2 / 16;  // 16-byte chunks per key row
+  long long zero_blocks = (dead_rows * row_chunks + 255) / 256;
+  if (zero_blocks > 148 * 4) zero_blocks = 148 * 4;
+  const long long blocks = main_blocks + zero_blocks;
+  if (blocks == 0) return cudaSuccess;
+  auto* zk = reinterpret_cast<uint4*>(dk);
+  auto* zv = reinterpret_cast<uint4*>(dv);
   if (d == 64)
-    bwd_prep_kernel<64><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(o, dout, delta, dq_acc, n_rows);
+    bwd_prep_kernel<64><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
+        o, dout, delta, dq_acc, n_rows, static_cast<unsigned>(main_blocks), dead, n_samples, row_chunks, zk, zv);
   else
-    bwd_prep_kernel<128><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(o, dout, delta, dq_acc, n_rows);
+    bwd_prep_kernel<128><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
+        o, dout, delta, dq_acc, n_rows, static_cast<unsigned>(main_blocks), dead, n_samples, row_chunks, zk, zv);
   return cudaGetLastError();
 }
 

@@ -85,8 +85,7 @@ extern "C" int skv_attn_fwd_noalloc(const void* plan, const void* q, const void*
   if (e != cudaSuccess) return skv_record_cuda_error(static_cast<int>(e));
   uint8_t* base = static_cast<uint8_t*>(ws);
   // zero what must start at zero: status word and queue counters
-  e = cudaMemsetAsync(base + w.status, 0, 256, stream);
-  if (e == cudaSuccess) e = cudaMemsetAsync(base + w.counters, 0, 2 * sizeof(int32_t) * static_cast<size_t>(h->P), stream);
+  e = cudaMemsetAsync(base + w.status, 0, w.control, stream);  // status word and queue counters
   if (e == cudaSuccess && h->dev.bytes > 0)
     e = cudaMemcpyAsync(base + w.dev, static_cast<const uint8_t*>(plan) + h->dev_off, h->dev.bytes,
                         cudaMemcpyHostToDevice, stream);

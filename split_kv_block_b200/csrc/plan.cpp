@@ -389,6 +389,7 @@ PlanHeader layout_of(const Prob& q, int policy, const Built& b) {
   h.dev.merge_list = put(b.merge_list.size() * sizeof(int32_t));
   h.dev.bwd_units = put(b.bwd.size() * sizeof(BwdUnit));
   h.dev.bwd_part_off = put(b.bwd_part_off.size() * sizeof(int32_t));
+  h.dev.dead = put(b.dead.size() * sizeof(int64_t));
   h.dev.bytes = d;
   h.total_bytes = h.dev_off + d;
   return h;
@@ -445,6 +446,7 @@ extern "C" int skv_plan(const skv_problem* prob, int policy, void* plan, size_t 
   copy_to(dev, h.dev.merge_list, b.merge_list);
   copy_to(dev, h.dev.bwd_units, b.bwd);
   copy_to(dev, h.dev.bwd_part_off, b.bwd_part_off);
+  copy_to(dev, h.dev.dead, b.dead);
   if (partition_load) std::memcpy(partition_load, b.load.data(), b.load.size() * sizeof(int64_t));
   return SKV_OK;
 }

@@ -10,7 +10,7 @@
 namespace skv {
 
 constexpr uint64_t kPlanMagic = 0x31764b5374696c53ull;  // "SlitSKv1"
-constexpr uint32_t kPlanVersion = 1;
+constexpr uint32_t kPlanVersion = 2;
 constexpr int kTileM = 128;  // query rows per tile (TMEM lanes)
 constexpr int kTileN = 128;  // keys per tile
 
@@ -70,6 +70,7 @@ struct DevSection {
   uint64_t merge_list;    // int32[n_fwd]: fwd unit ids per (tile, kv head), ascending kbeg
   uint64_t bwd_units;     // BwdUnit[n_bwd]
   uint64_t bwd_part_off;  // int32[P+1]
+  uint64_t dead;          // int64[2B]: [begin, end) keys of sample b whose dK/dV are zero
   uint64_t bytes;         // total
 };
 
@@ -95,12 +96,13 @@ struct PlanHeader {
   uint64_t total_bytes;
 };
 
-// Workspace layout: control block, device plan section, queue counters, then
-// the pass-specific scratch.
+// Workspace layout: control block (status word and queue counters, cleared by
+// one memset per call), device plan section, then the pass-specific scratch.
 struct WsLayout {
   uint64_t status;    // int32 status word at offset 0
+  uint64_t counters;  // int32[2 * P] queue heads (forward, backward), right after it
+  uint64_t control;   // bytes of the control block
   uint64_t dev;       // device section copy
-  uint64_t counters;  // int32[2 * P] queue heads (forward, backward)
   uint64_t fwd_o;     // fp32 [n_fwd][128][d] partial outputs
   uint64_t fwd_lse;   // fp32 [n_fwd][128] partial LSE
   uint64_t fwd_end;
@@ -114,9 +116,10 @@ inline uint64_t align_up(uint64_t x, uint64_t a) { return (x + a - 1) / a * a; }
 inline WsLayout ws_layout(const PlanHeader& h) {
   WsLayout w{};
   w.status = 0;
-  w.dev = 256;
-  w.counters = align_up(w.dev + h.dev.bytes, 256);
-  uint64_t scratch = align_up(w.counters + 2 * sizeof(int32_t) * static_cast<uint64_t>(h.P), 256);
+  w.counters = 16;
+  w.control = w.counters + 2 * sizeof(int32_t) * static_cast<uint64_t>(h.P);
+  w.dev = align_up(w.control, 256);
+  uint64_t scratch = align_up(w.dev + h.dev.bytes, 256);
   w.fwd_o = scratch;
   w.fwd_lse = align_up(w.fwd_o + static_cast<uint64_t>(h.n_fwd) * kTileM * h.d * 4, 256);
   w.fwd_end = align_up(w.fwd_lse + static_cast<uint64_t>(h.n_fwd) * kTileM * 4, 256);

@@ -175,3 +175,23 @@ def test_batch8_full_size_one_sample_one_group():
     sub, qs, ks, vs, dos, os_, ls, gs = _one_sample(prob, b, q, k, v, do, o, lse, grads)
     check_forward(sub, qs, ks, vs, os_, ls, groups=(6,))
     check_backward(sub, qs, ks, vs, dos, gs, groups=(6,))
+
+
+def test_dead_key_gradients_are_written_zero():
+    """Keys past every anchor of their sample get dK = dV = 0 written by the
+    backward itself (the outputs start as NaN here), in every sample."""
+    prob = synth.small_problem([700, 513, 900], [[300, 2], [513], [64, 450, 10]], block_q=16, chunk_kv=256,
+                               num_partitions=3, hq=8, hkv=2, d=128)
+    q, k, v, do = synth.make_tensors(prob, seed=5, backward=True)
+    plan = skv.skv_plan(prob)
+    qd, kd, vd, dod = _dev(q, k, v, do)
+    ws = skv.alloc_workspace(plan)
+    o, lse = skv.forward(plan, qd, kd, vd, ws)
+    dq = torch.full_like(qd, float("nan"))
+    dk = torch.full_like(kd, float("nan"))
+    dv = torch.full_like(vd, float("nan"))
+    skv.skv_attn_bwd(plan, qd, kd, vd, o, lse, dod, dq, dk, dv, ws)
+    assert skv.skv_status(ws) == 0
+    torch.cuda.synchronize()
+    check_backward(prob, q, k, v, do, (dq.cpu(), dk.cpu(), dv.cpu()))
+    assert not torch.isnan(dk).any() and not torch.isnan(dv).any() and not torch.isnan(dq).any()
