@@ -230,6 +230,24 @@ int skv_set_timing_events(int kernel, void* start_event, void* end_event);
 int skv_attn_fwd_noalloc(const void* plan, const void* q, const void* k, const void* v, void* o, float* lse,
                          skv_stream_t stream);
 
+/*
+ * skv_wait_selftest — exercises, without any fault, the bounded device-side
+ * wait every kernel of this library uses. One CTA waits on a shared-memory
+ * mbarrier phase for at most `limit_ns` nanoseconds of %globaltimer time:
+ *   * arrive != 0: the CTA completes the phase itself first, the wait
+ *     succeeds and the status word stays SKV_OK;
+ *   * arrive == 0: nothing completes the phase, the wait gives up and records
+ *     SKV_ETIMEOUT in the status word, exactly as a stalled pipeline stage of
+ *     the attention kernels would. The device context stays usable.
+ * The outcome is read with skv_status(ws, stream). The pages have no
+ * counterpart of this call; it tests this library's failure detection.
+ * ws: device buffer of at least 256 bytes, 256-byte aligned, caller-owned;
+ * its status word is cleared first. limit_ns: 1 .. 10^10.
+ * Returns SKV_EINVAL for a NULL or misaligned ws or a limit out of range,
+ * SKV_ECUDA when the launch fails, SKV_OK otherwise.
+ */
+int skv_wait_selftest(void* ws, uint64_t limit_ns, int arrive, skv_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -24,7 +24,7 @@ SKV_PLAN_STATIC = 1
 EXPORTS = ("skv_plan_size", "skv_plan", "skv_plan_items", "skv_plan_unit_partitions", "skv_plan_stats", "skv_attn_fwd",
            "skv_lse_merge",
            "skv_attn_bwd", "skv_status", "skv_strerror", "skv_last_cuda_error", "skv_set_unit_timer",
-           "skv_set_timing_events", "skv_attn_fwd_noalloc")
+           "skv_set_timing_events", "skv_attn_fwd_noalloc", "skv_wait_selftest")
 SKV_NOALLOC_SCRATCH_BYTES = 32 << 20
 SKV_KERNEL_FWD, SKV_KERNEL_MERGE, SKV_KERNEL_BWD = 0, 1, 2
 
@@ -71,6 +71,7 @@ def lib() -> ctypes.CDLL:
         L.skv_set_unit_timer.argtypes = [vp, vp]
         L.skv_set_timing_events.argtypes = [ctypes.c_int, vp, vp]
         L.skv_attn_fwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp]
+        L.skv_wait_selftest.argtypes = [vp, ctypes.c_uint64, ctypes.c_int, vp]
         for name in EXPORTS:
             if name not in ("skv_strerror",):
                 getattr(L, name).restype = ctypes.c_int
@@ -205,6 +206,13 @@ def skv_attn_bwd(plan: Plan, q, k, v, o, lse, do, dq, dk, dv, ws, stream=None):
     _check("skv_attn_bwd", lib().skv_attn_bwd(plan.ptr, _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(do),
                                               _ptr(dq), _ptr(dk), _ptr(dv), _ptr(ws), ws.numel(),
                                               _stream_ptr(stream)))
+
+
+def skv_wait_selftest(ws, limit_ns: int, arrive: bool, stream=None):
+    """One bounded device-side wait of `limit_ns`: completed first (arrive) or
+    never (its give-up leaves SKV_ETIMEOUT in ws's status word)."""
+    _check("skv_wait_selftest", lib().skv_wait_selftest(_ptr(ws), int(limit_ns), 1 if arrive else 0,
+                                                        _stream_ptr(stream)))
 
 
 def skv_attn_fwd_noalloc(plan: Plan, q, k, v, o, lse, stream=None):
