@@ -4,13 +4,14 @@
 // from the merged LSE; "Split-KV: Breaking the Context Parallelism Bottleneck
 // in Diffusion Drafter Training", section "Split-KV's Core Mechanism"), laid
 // out so that the tensor core is rarely idle:
-//   * TMEM: two 128-column regions R0/R1 that swap roles every query tile
-//     (S^T of tile i and dQ^T of tile i in R_p, dP^T of tile i and then P^T
-//     (bf16, packed) in R_{1-p}, p = i & 1), plus dV and dK accumulators;
-//     S^T of tile i+1 is computed while tile i's gradient MMAs run.
 //   * Two softmax-gradient warpgroups, each owning 64 of the tile's 128 query
-//     rows (TMEM columns); the gradient MMAs of a half start as soon as that
-//     half is ready.
+//     rows, run two independent half-tile pipelines through the tensor core.
+//     Half h has its own TMEM regions: A_h (64 columns) holds S^T of its rows
+//     and then P^T (bf16, packed), B_h (64 columns) holds dP^T and then dQ^T;
+//     dV and dK accumulate in the last 256 columns for the whole unit. As soon
+//     as half h's gradient MMAs of tile i have consumed A_h and its dQ^T has
+//     been read out of B_h, S^T and dP^T of half h of tile i+1 are computed,
+//     so one half's softmax runs while the other half's MMAs execute.
 //   * P^T stays in TMEM and feeds dV += P^T dO as the A operand; dS^T goes to
 //     shared memory once and serves as the A operand of dK += dS^T Q and the
 //     B operand of dQ^T = K^T dS^T.
@@ -39,9 +40,9 @@ struct Ctl {
   uint64_t sched_full[2], sched_empty[2];
   uint64_t kv_full, kv_empty;
   uint64_t q_full[2], q_empty[2], do_full[2], do_empty[2];
-  uint64_t sdp_full;
-  uint64_t pds_full[2];
-  uint64_t dv_done;
+  uint64_t sdp_full[2];   // per half: S^T and dP^T in TMEM
+  uint64_t pds_full[2];   // per half: P^T in TMEM, dS^T in shared memory
+  uint64_t dv_done[2];    // per half: dV MMA done (A_h free)
   uint64_t dq_full[2], dq_free[2];
   uint64_t acc_full, acc_free;
   uint64_t meta_full[2][2];  // [warpgroup][tile parity]
@@ -59,7 +60,8 @@ constexpr int kCtl = kDS + 128 * 128 * 2;
 constexpr int kSmemBytes = kCtl + static_cast<int>(sizeof(Ctl));
 static_assert(kSmemBytes <= 232448, "shared memory budget");
 
-__device__ __forceinline__ uint32_t col_r(uint32_t i) { return 128u * (i & 1u); }  // region R0 or R1
+__device__ __forceinline__ uint32_t col_a(int h) { return 64u * h; }         // S^T, then P^T, of half h
+__device__ __forceinline__ uint32_t col_b(int h) { return 128u + 64u * h; }  // dP^T, then dQ^T, of half h
 constexpr uint32_t kColDV = 256, kColDK = 384;
 
 // kG: compile-time q-heads per kv-head (0 = runtime value p.G)
@@ -88,6 +90,8 @@ __global__ void __launch_bounds__(384, 1)
       mbar_init(&c.do_full[i], 1);
       mbar_init(&c.do_empty[i], 1);
       mbar_init(&c.pds_full[i], 128);
+      mbar_init(&c.sdp_full[i], 1);
+      mbar_init(&c.dv_done[i], 1);
       mbar_init(&c.dq_full[i], 1);
       mbar_init(&c.dq_free[i], 128);
       mbar_init(&c.meta_full[i][0], 128);
@@ -95,8 +99,6 @@ __global__ void __launch_bounds__(384, 1)
     }
     mbar_init(&c.kv_full, 1);
     mbar_init(&c.kv_empty, 1);
-    mbar_init(&c.sdp_full, 1);
-    mbar_init(&c.dv_done, 1);
     mbar_init(&c.acc_full, 1);
     mbar_init(&c.acc_free, 256);
     mbar_init(&c.final_mma, 1);
@@ -185,13 +187,38 @@ __global__ void __launch_bounds__(384, 1)
   } else if (warp == 1) {
     // ---------------------------------------------------------- MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idS = idesc_bf16(128, 128, false, false);  // S^T = K Q^T, dP^T = V dO^T
-      constexpr uint32_t idKV = idesc_bf16(128, kD, false, true);   // dV += P^T dO, dK += dS^T Q
-      constexpr uint32_t idQ = idesc_bf16(128, 64, true, true);     // dQ^T(half) = K^T dS^T(half)
+      constexpr uint32_t idS = idesc_bf16(128, 64, false, false);   // S^T_h = K Q_h^T, dP^T_h = V dO_h^T
+      constexpr uint32_t idKV = idesc_bf16(128, kD, false, true);   // dV += P^T dO, dK += dS^T Q (half's rows)
+      constexpr uint32_t idQ = idesc_bf16(128, 64, true, true);     // dQ^T_h = K^T dS^T_h
       const uint32_t sK = smem_u32(smem + kK), sV = smem_u32(smem + kV), sQ0 = smem_u32(smem + kQ0),
                      sDO0 = smem_u32(smem + kDO0), sDS = smem_u32(smem + kDS);
       uint32_t n_units = 0, qc = 0, kv_waits = 0;
       bool ok = true;
+      // S^T and dP^T of half h of tile number i: rows 64h..64h+63 of its Q / dO tile, into A_h / B_h once
+      // half h of tile i - 1 has consumed A_h (its dV) and its dQ^T has been read out of B_h
+      auto issue_sdp = [&](uint32_t i, int h) -> bool {
+        const int s = i & 1;
+        const uint32_t use = i >> 1;
+        if (!mbar_wait(&c.q_full[s], use & 1, status, lim)) return false;
+        if (!mbar_wait(&c.do_full[s], use & 1, status, lim)) return false;
+        if (i >= 1 && (!mbar_wait(&c.dv_done[h], (i - 1) & 1, status, lim) ||
+                       !mbar_wait(&c.dq_free[h], (i - 1) & 1, status, lim)))
+          return false;
+        tc_fence_after();
+        const uint32_t sQ = sQ0 + s * kTileBytes + h * 8192, sDO = sDO0 + s * kTileBytes + h * 8192;
+#pragma unroll
+        for (int ks = 0; ks < kD / 16; ++ks) {
+          const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
+          umma_bf16(tmem + col_a(h), sdesc_sw128(sK + off, 16, 1024), sdesc_sw128(sQ + off, 16, 1024), idS, ks > 0);
+        }
+#pragma unroll
+        for (int ks = 0; ks < kD / 16; ++ks) {
+          const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
+          umma_bf16(tmem + col_b(h), sdesc_sw128(sV + off, 16, 1024), sdesc_sw128(sDO + off, 16, 1024), idS, ks > 0);
+        }
+        umma_commit(&c.sdp_full[h]);
+        return true;
+      };
       while (ok) {
         const int slot = n_units & 1;
         if (!mbar_wait(&c.sched_full[slot], (n_units >> 1) & 1, status, lim)) break;
@@ -202,31 +229,14 @@ __global__ void __launch_bounds__(384, 1)
         bool first = true;
         for (int mt = U.mt_begin; mt < U.mt_end; ++mt) {
           if (p.mtiles[mt].kmax <= U.kbeg) continue;
+          int nxt = mt + 1;  // the unit's next live query tile
+          while (nxt < U.mt_end && p.mtiles[nxt].kmax <= U.kbeg) ++nxt;
           const int s = qc & 1;
-          const uint32_t use = qc >> 1;
-          const uint32_t rS = tmem + col_r(qc), rP = tmem + col_r(qc + 1);
           const uint32_t sQ = sQ0 + s * kTileBytes, sDO = sDO0 + s * kTileBytes;
-          if (first && !mbar_wait(&c.kv_full, (kv_waits++) & 1, status, lim)) { ok = false; break; }
-          if (!mbar_wait(&c.q_full[s], use & 1, status, lim)) { ok = false; break; }
-          // S^T -> R_p, where the previous tile's P^T lived: its dV MMA must be done
-          if (qc >= 1 && !mbar_wait(&c.dv_done, (qc - 1) & 1, status, lim)) { ok = false; break; }
-          tc_fence_after();
-#pragma unroll
-          for (int ks = 0; ks < kD / 16; ++ks) {
-            const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
-            umma_bf16(rS, sdesc_sw128(sK + off, 16, 1024), sdesc_sw128(sQ + off, 16, 1024), idS, ks > 0);
+          if (first) {  // a unit's first tile waits for the unit's K/V
+            if (!mbar_wait(&c.kv_full, (kv_waits++) & 1, status, lim)) { ok = false; break; }
+            if (!issue_sdp(qc, 0) || !issue_sdp(qc, 1)) { ok = false; break; }
           }
-          // dP^T -> R_{1-p}, where the previous tile's dQ^T lived: it must be drained
-          if (!mbar_wait(&c.do_full[s], use & 1, status, lim)) { ok = false; break; }
-          if (qc >= 1 && (!mbar_wait(&c.dq_free[0], (qc - 1) & 1, status, lim) ||
-                          !mbar_wait(&c.dq_free[1], (qc - 1) & 1, status, lim))) { ok = false; break; }
-          tc_fence_after();
-#pragma unroll
-          for (int ks = 0; ks < kD / 16; ++ks) {
-            const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
-            umma_bf16(rP, sdesc_sw128(sV + off, 16, 1024), sdesc_sw128(sDO + off, 16, 1024), idS, ks > 0);
-          }
-          umma_commit(&c.sdp_full);
           for (int h = 0; h < 2 && ok; ++h) {
             if (!mbar_wait(&c.pds_full[h], qc & 1, status, lim)) { ok = false; break; }
             if (first && h == 0 && n_units >= 1 && !mbar_wait(&c.acc_free, (n_units - 1) & 1, status, lim)) {
@@ -234,17 +244,15 @@ __global__ void __launch_bounds__(384, 1)
               break;
             }
             tc_fence_after();
-            // dV += P^T dO over the half's 64 rows (A = P^T from TMEM)
+            // dV += P^T dO over the half's 64 rows (A = P^T_h from TMEM)
 #pragma unroll
             for (int k4 = 0; k4 < 4; ++k4) {
               const uint32_t acc = (first && h == 0 && k4 == 0) ? 0u : 1u;
-              umma_bf16_ts(tmem + kColDV, rP + 64 * h + 8 * k4,
+              umma_bf16_ts(tmem + kColDV, tmem + col_a(h) + 8 * k4,
                            sdesc_sw128(sDO + (64 * h + 16 * k4) * 128, 16384, 1024), idKV, acc);
             }
-            if (h == 1) {
-              umma_commit(&c.dv_done);
-              umma_commit(&c.do_empty[s]);
-            }
+            umma_commit(&c.dv_done[h]);
+            if (h == 1) umma_commit(&c.do_empty[s]);
             // dK += dS^T Q over the half's rows
 #pragma unroll
             for (int k4 = 0; k4 < 4; ++k4) {
@@ -253,12 +261,14 @@ __global__ void __launch_bounds__(384, 1)
                         sdesc_sw128(sQ + (64 * h + 16 * k4) * 128, 16384, 1024), idKV, acc);
             }
             if (h == 1) umma_commit(&c.q_empty[s]);
-            // dQ^T of the half's rows = K^T dS^T -> R_p columns [64h, 64h + 64)
+            // dQ^T of the half's rows = K^T dS^T -> B_h
 #pragma unroll
             for (int ks = 0; ks < 128 / 16; ++ks)
-              umma_bf16(rS + 64 * h, sdesc_sw128(sK + ks * 2048, 16384, 1024),
+              umma_bf16(tmem + col_b(h), sdesc_sw128(sK + ks * 2048, 16384, 1024),
                         sdesc_sw128(sDS + h * 16384 + ks * 2048, 16384, 1024), idQ, ks > 0);
             umma_commit(&c.dq_full[h]);
+            // this half of the unit's next tile, as soon as A_h and B_h are free
+            if (nxt < U.mt_end && !issue_sdp(qc + 1, h)) { ok = false; break; }
           }
           if (!ok) break;
           first = false;
@@ -318,7 +328,7 @@ __global__ void __launch_bounds__(384, 1)
       while (mt < U.mt_end) {
         had_tiles = true;
         const int par = qc & 1;
-        const uint32_t rS = tmem + lane_off + col_r(par), rP = tmem + lane_off + col_r(par + 1);
+        const uint32_t tA = tmem + lane_off + col_a(wg), tB = tmem + lane_off + col_b(wg);
         // stage this tile's metadata, then fetch the next live tile's
         if (t < 64) {
           const int r = 64 * wg + t;
@@ -339,7 +349,7 @@ __global__ void __launch_bounds__(384, 1)
         if (!mbar_wait_warp(&c.meta_full[wg][par], (qc >> 1) & 1, status, lim)) { ok = false; break; }
         // every row of this half attends key t of every lane of the warp: no per-element mask
         const bool unmasked = __all_sync(0xffffffffu, t < min(c.kmin[wg][par][0], c.kmin[wg][par][1]));
-        if (!mbar_wait_warp(&c.sdp_full, qc & 1, status, lim)) { ok = false; break; }
+        if (!mbar_wait_warp(&c.sdp_full[wg], qc & 1, status, lim)) { ok = false; break; }
         tc_fence_after();
         uint8_t* dsrow = smem + kDS + wg * 16384;
         const float sl2 = p.scale_log2;
@@ -347,8 +357,8 @@ __global__ void __launch_bounds__(384, 1)
         for (int ch = 0; ch < 2; ++ch) {
           const int col = 64 * wg + 32 * ch;  // first tile row of this chunk
           uint32_t vs[32], vd[32];
-          tmem_ld32(rS + col, vs);
-          tmem_ld32(rP + col, vd);
+          tmem_ld32(tA + 32 * ch, vs);
+          tmem_ld32(tB + 32 * ch, vd);
           tmem_wait_ld();
           uint32_t pk[16];
           uint32_t dk[16];
@@ -372,8 +382,8 @@ __global__ void __launch_bounds__(384, 1)
             dk[(i >> 1) + 0] = pack_bf16(x0 * (__uint_as_float(vd[i + 0]) - D4.x), x1 * (__uint_as_float(vd[i + 1]) - D4.y));
             dk[(i >> 1) + 1] = pack_bf16(x2 * (__uint_as_float(vd[i + 2]) - D4.z), x3 * (__uint_as_float(vd[i + 3]) - D4.w));
           }
-          // P^T (bf16 pairs) over the dP^T columns already read
-          tmem_st16(rP + 64 * wg + 16 * ch, pk);
+          // P^T (bf16 pairs) over the S^T columns of this half already read
+          tmem_st16(tA + 16 * ch, pk);
           // dS^T row t of this warpgroup's 64-row block: 16-byte chunks 4 ch .. 4 ch + 3
 #pragma unroll
           for (int q = 0; q < 4; ++q)
@@ -388,8 +398,8 @@ __global__ void __launch_bounds__(384, 1)
         if (!mbar_wait_warp(&c.dq_full[wg], qc & 1, status, lim)) { ok = false; break; }
         tc_fence_after();
         uint32_t q0[32], q1[32];
-        tmem_ld32(rS + 64 * wg, q0);
-        tmem_ld32(rS + 64 * wg + 32, q1);
+        tmem_ld32(tB, q0);
+        tmem_ld32(tB + 32, q1);
         tmem_wait_ld();
         tc_fence_before();
         mbar_arrive(&c.dq_free[wg]);
