@@ -250,19 +250,28 @@ void make_lists(const Prob& q, const std::vector<SampleAnchors>& sa, Built& out)
   out.bwd.clear();
   out.bwd_part_off.assign(q.P + 1, 0);
   std::vector<std::pair<int64_t, int32_t>> tiles;
+  std::vector<std::pair<int32_t, int32_t>> item_fwd(out.items.size(), {0, 0});  // [first forward unit, count]
   for (int p = 0; p < q.P; ++p) {
     out.fwd_part_off[p] = static_cast<int32_t>(out.fwd.size());
     out.pair_off[p] = static_cast<int32_t>(out.pairs.size());
     out.bwd_part_off[p] = static_cast<int32_t>(out.bwd.size());
     for (int32_t id : by_part[p]) {
       const skv_item& it = out.items[id];
-      // forward: live query tiles, longest key range first
+      // forward: live query tiles, longest key range first (ties by tile index). Tiles reaching past
+      // the item's end all have its full range and come first in index order; only the others,
+      // few per item, need sorting.
       tiles.clear();
+      size_t n_full = 0;
       for (int32_t mt = out.sample_mt[it.b]; mt < out.sample_mt[it.b + 1]; ++mt) {
-        const int64_t ke = std::min<int64_t>(it.key_end, out.mtiles[mt].kmax);
-        if (ke > it.key_begin) tiles.push_back({-(ke - it.key_begin), mt});
+        const int64_t kmax = out.mtiles[mt].kmax;
+        if (kmax >= it.key_end) {
+          tiles.insert(tiles.begin() + static_cast<std::ptrdiff_t>(n_full++), {-(it.key_end - it.key_begin), mt});
+        } else if (kmax > it.key_begin) {
+          tiles.push_back({-(kmax - it.key_begin), mt});
+        }
       }
-      std::sort(tiles.begin(), tiles.end());
+      std::sort(tiles.begin() + static_cast<std::ptrdiff_t>(n_full), tiles.end());
+      item_fwd[id] = {static_cast<int32_t>(out.fwd.size()), static_cast<int32_t>(tiles.size())};
       for (size_t ti = 0; ti < tiles.size(); ++ti) {
         const auto& t = tiles[ti];
         FwdUnit u{};
@@ -288,15 +297,16 @@ void make_lists(const Prob& q, const std::vector<SampleAnchors>& sa, Built& out)
       }
       // backward: key tiles below the sample's largest anchor
       const int64_t kmax_b = q.ctx[it.b] + sa[it.b].max_a;
+      // first query tile whose largest anchor reaches past the key tile start (later dead tiles,
+      // possible with unsorted anchors, are skipped by the kernel); a tile dead for one key tile is
+      // dead for every later one, so the index only moves forward
+      int32_t first = out.sample_mt[it.b];
       for (int64_t kb = it.key_begin; kb < it.key_end && kb < kmax_b; kb += kTileN) {
         BwdUnit u{};
         u.b = it.b;
         u.g = it.g;
         u.kbeg = static_cast<int32_t>(kb);
         u.kend = static_cast<int32_t>(std::min<int64_t>(kb + kTileN, it.key_end));
-        // first query tile whose largest anchor reaches past the key tile start
-        // (later dead tiles, possible with unsorted anchors, are skipped by the kernel)
-        int32_t first = out.sample_mt[it.b];
         while (first < out.sample_mt[it.b + 1] && out.mtiles[first].kmax <= kb) ++first;
         u.mt_begin = first;
         u.mt_end = out.sample_mt[it.b + 1];
@@ -317,13 +327,13 @@ void make_lists(const Prob& q, const std::vector<SampleAnchors>& sa, Built& out)
   for (size_t i = 0; i < nslots; ++i) out.merge_off[i + 1] += out.merge_off[i];
   out.merge_list.assign(out.fwd.size(), 0);
   std::vector<int32_t> fill(out.merge_off.begin(), out.merge_off.end() - 1);
-  for (size_t i = 0; i < out.fwd.size(); ++i) {
-    const auto& u = out.fwd[i];
-    out.merge_list[fill[static_cast<size_t>(u.mt) * q.Hkv + u.g]++] = static_cast<int32_t>(i);
-  }
-  for (size_t sidx = 0; sidx < nslots; ++sidx)
-    std::sort(out.merge_list.begin() + out.merge_off[sidx], out.merge_list.begin() + out.merge_off[sidx + 1],
-              [&](int32_t x, int32_t y) { return out.fwd[x].kbeg < out.fwd[y].kbeg; });
+  // Items are in (b, c, g, s) order: walking them fills every (tile, kv head) slot in ascending key
+  // order (an item has at most one unit per tile, and its key range starts after the previous item's).
+  for (size_t id = 0; id < out.items.size(); ++id)
+    for (int32_t i = item_fwd[id].first; i < item_fwd[id].first + item_fwd[id].second; ++i) {
+      const auto& u = out.fwd[i];
+      out.merge_list[fill[static_cast<size_t>(u.mt) * q.Hkv + u.g]++] = i;
+    }
 
   // keys whose gradients are zero: past the last backward tile of the sample
   out.dead.assign(2 * static_cast<size_t>(q.B), 0);
@@ -405,9 +415,16 @@ void copy_to(uint8_t* base, uint64_t off, const std::vector<T>& v) {
 
 using namespace skv;
 
+// Planner working set of the calling thread: its vectors keep their capacity from call to call,
+// so replanning every step (new anchors) does not reallocate and re-fault megabytes of lists.
+Built& scratch() {
+  thread_local Built b;
+  return b;
+}
+
 extern "C" int skv_plan_size(const skv_problem* prob, int policy, size_t* n_items, size_t* plan_bytes,
                              size_t* ws_fwd_bytes, size_t* ws_bwd_bytes) {
-  Built b;
+  Built& b = scratch();
   Prob q;
   int rc = build(prob, policy, b, q);
   if (rc != SKV_OK) return rc;
@@ -423,7 +440,7 @@ extern "C" int skv_plan_size(const skv_problem* prob, int policy, size_t* n_item
 extern "C" int skv_plan(const skv_problem* prob, int policy, void* plan, size_t plan_bytes,
                         int64_t* partition_load) {
   if (!plan) return SKV_EINVAL;
-  Built b;
+  Built& b = scratch();
   Prob q;
   int rc = build(prob, policy, b, q);
   if (rc != SKV_OK) return rc;
