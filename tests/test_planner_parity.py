@@ -168,3 +168,19 @@ def test_unit_partitions_of_the_32k_workload():
     P = prob.num_partitions
     assert np.bincount(fp, minlength=P).tolist() == ef.tolist()
     assert np.bincount(bp, minlength=P).tolist() == eb.tolist()
+
+
+def test_plans_do_not_depend_on_earlier_calls():
+    """The planner reuses its working memory between calls on a thread: a plan
+    must come out byte-identical whatever was planned before it (larger,
+    smaller, other policy)."""
+    rng = np.random.default_rng(77)
+    big = synth.make_problem(synth.WORKLOADS["ctx128k"], seed=1, sub_chunks=4)
+    small = synth.random_small_problem(rng, max_len=900, max_anchors=5, d=64, heads=((4, 1),))
+    other = synth.make_problem(synth.WORKLOADS["ctx32k"], seed=2)
+    ref = {name: {pol: skv.skv_plan(p, pol).buf.tobytes() for pol in (skv.SKV_PLAN_LPT, skv.SKV_PLAN_STATIC)}
+           for name, p in (("big", big), ("small", small), ("other", other))}
+    order = [("small", small), ("big", big), ("other", other), ("small", small), ("big", big), ("small", small)]
+    for name, p in order:
+        for pol in (skv.SKV_PLAN_STATIC, skv.SKV_PLAN_LPT):
+            assert skv.skv_plan(p, pol).buf.tobytes() == ref[name][pol], (name, pol)
