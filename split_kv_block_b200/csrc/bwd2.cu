@@ -186,70 +186,84 @@ __global__ void __launch_bounds__(384, 1)
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------- MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t idS = idesc_bf16(128, 64, false, false);   // S^T_h = K Q_h^T, dP^T_h = V dO_h^T
-      constexpr uint32_t idKV = idesc_bf16(128, kD, false, true);   // dV += P^T dO, dK += dS^T Q (half's rows)
-      constexpr uint32_t idQ = idesc_bf16(128, 64, true, true);     // dQ^T_h = K^T dS^T_h
-      const uint32_t sK = smem_u32(smem + kK), sV = smem_u32(smem + kV), sQ0 = smem_u32(smem + kQ0),
-                     sDO0 = smem_u32(smem + kDO0), sDS = smem_u32(smem + kDS);
-      uint32_t n_units = 0, qc = 0, kv_waits = 0;
-      bool ok = true;
-      // S^T and dP^T of half h of tile number i: rows 64h..64h+63 of its Q / dO tile, into A_h / B_h once
-      // half h of tile i - 1 has consumed A_h (its dV) and its dQ^T has been read out of B_h
-      auto issue_sdp = [&](uint32_t i, int h) -> bool {
-        const int s = i & 1;
-        const uint32_t use = i >> 1;
-        if (!mbar_wait(&c.q_full[s], use & 1, status, lim)) return false;
-        if (!mbar_wait(&c.do_full[s], use & 1, status, lim)) return false;
-        if (i >= 1 && (!mbar_wait(&c.dv_done[h], (i - 1) & 1, status, lim) ||
-                       !mbar_wait(&c.dq_free[h], (i - 1) & 1, status, lim)))
-          return false;
-        tc_fence_after();
-        const uint32_t sQ = sQ0 + s * kTileBytes + h * 8192, sDO = sDO0 + s * kTileBytes + h * 8192;
+    // All 32 lanes run the loop (stage indices and descriptors stay warp-uniform); one elected lane issues
+    // the MMAs and their commits.
+    const bool leader = elect_one();
+    constexpr uint32_t idS = idesc_bf16(128, 64, false, false);   // S^T_h = K Q_h^T, dP^T_h = V dO_h^T
+    constexpr uint32_t idKV = idesc_bf16(128, kD, false, true);   // dV += P^T dO, dK += dS^T Q (half's rows)
+    constexpr uint32_t idQ = idesc_bf16(128, 64, true, true);     // dQ^T_h = K^T dS^T_h
+    // operand descriptors at their buffers' starts; K steps, row blocks and stages are byte offsets
+    const uint64_t dK_k = sdesc_sw128(smem_u32(smem + kK), 16, 1024);          // K as A of S^T (K-major)
+    const uint64_t dV_k = sdesc_sw128(smem_u32(smem + kV), 16, 1024);          // V as A of dP^T
+    const uint64_t dK_mn = sdesc_sw128(smem_u32(smem + kK), 16384, 1024);      // K^T as A of dQ^T (MN-major)
+    const uint64_t dQ_k = sdesc_sw128(smem_u32(smem + kQ0), 16, 1024);         // Q_h as B of S^T
+    const uint64_t dDO_k = sdesc_sw128(smem_u32(smem + kDO0), 16, 1024);       // dO_h as B of dP^T
+    const uint64_t dQ_mn = sdesc_sw128(smem_u32(smem + kQ0), 16384, 1024);     // Q as B of dK
+    const uint64_t dDO_mn = sdesc_sw128(smem_u32(smem + kDO0), 16384, 1024);   // dO as B of dV
+    const uint64_t dS_k = sdesc_sw128(smem_u32(smem + kDS), 16, 1024);         // dS^T as A of dK
+    const uint64_t dS_mn = sdesc_sw128(smem_u32(smem + kDS), 16384, 1024);     // dS^T as B of dQ^T
+    uint32_t n_units = 0, qc = 0, kv_waits = 0;
+    bool ok = true;
+    // S^T and dP^T of half h of tile number i: rows 64h..64h+63 of its Q / dO tile, into A_h / B_h once
+    // half h of tile i - 1 has consumed A_h (its dV) and its dQ^T has been read out of B_h
+    auto issue_sdp = [&](uint32_t i, int h) -> bool {
+      const int s = i & 1;
+      const uint32_t use = i >> 1;
+      if (!mbar_wait_warp(&c.q_full[s], use & 1, status, lim)) return false;
+      if (!mbar_wait_warp(&c.do_full[s], use & 1, status, lim)) return false;
+      if (i >= 1 && (!mbar_wait_warp(&c.dv_done[h], (i - 1) & 1, status, lim) ||
+                     !mbar_wait_warp(&c.dq_free[h], (i - 1) & 1, status, lim)))
+        return false;
+      tc_fence_after();
+      const uint32_t rows = s * kTileBytes + h * 8192;
+      if (leader) {
 #pragma unroll
         for (int ks = 0; ks < kD / 16; ++ks) {
           const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
-          umma_bf16(tmem + col_a(h), sdesc_sw128(sK + off, 16, 1024), sdesc_sw128(sQ + off, 16, 1024), idS, ks > 0);
+          umma_bf16(tmem + col_a(h), sdesc_add(dK_k, off), sdesc_add(dQ_k, rows + off), idS, ks > 0);
         }
 #pragma unroll
         for (int ks = 0; ks < kD / 16; ++ks) {
           const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
-          umma_bf16(tmem + col_b(h), sdesc_sw128(sV + off, 16, 1024), sdesc_sw128(sDO + off, 16, 1024), idS, ks > 0);
+          umma_bf16(tmem + col_b(h), sdesc_add(dV_k, off), sdesc_add(dDO_k, rows + off), idS, ks > 0);
         }
         umma_commit(&c.sdp_full[h]);
-        return true;
-      };
-      while (ok) {
-        const int slot = n_units & 1;
-        if (!mbar_wait(&c.sched_full[slot], (n_units >> 1) & 1, status, lim)) break;
-        const int u = c.sched[slot];
-        mbar_arrive(&c.sched_empty[slot]);
-        if (u < 0) break;
-        const BwdUnit U = p.units[u];
-        bool first = true;
-        for (int mt = U.mt_begin; mt < U.mt_end; ++mt) {
-          if (p.mtiles[mt].kmax <= U.kbeg) continue;
-          int nxt = mt + 1;  // the unit's next live query tile
-          while (nxt < U.mt_end && p.mtiles[nxt].kmax <= U.kbeg) ++nxt;
-          const int s = qc & 1;
-          const uint32_t sQ = sQ0 + s * kTileBytes, sDO = sDO0 + s * kTileBytes;
-          if (first) {  // a unit's first tile waits for the unit's K/V
-            if (!mbar_wait(&c.kv_full, (kv_waits++) & 1, status, lim)) { ok = false; break; }
-            if (!issue_sdp(qc, 0) || !issue_sdp(qc, 1)) { ok = false; break; }
+      }
+      __syncwarp();
+      return true;
+    };
+    while (ok) {
+      const int slot = n_units & 1;
+      if (!mbar_wait_warp(&c.sched_full[slot], (n_units >> 1) & 1, status, lim)) break;
+      const int u = c.sched[slot];
+      __syncwarp();
+      if (leader) mbar_arrive(&c.sched_empty[slot]);
+      if (u < 0) break;
+      const BwdUnit U = p.units[u];
+      bool first = true;
+      for (int mt = U.mt_begin; mt < U.mt_end; ++mt) {
+        if (p.mtiles[mt].kmax <= U.kbeg) continue;
+        int nxt = mt + 1;  // the unit's next live query tile
+        while (nxt < U.mt_end && p.mtiles[nxt].kmax <= U.kbeg) ++nxt;
+        const int s = qc & 1;
+        if (first) {  // a unit's first tile waits for the unit's K/V
+          if (!mbar_wait_warp(&c.kv_full, (kv_waits++) & 1, status, lim)) { ok = false; break; }
+          if (!issue_sdp(qc, 0) || !issue_sdp(qc, 1)) { ok = false; break; }
+        }
+        for (int h = 0; h < 2 && ok; ++h) {
+          if (!mbar_wait_warp(&c.pds_full[h], qc & 1, status, lim)) { ok = false; break; }
+          if (first && h == 0 && n_units >= 1 && !mbar_wait_warp(&c.acc_free, (n_units - 1) & 1, status, lim)) {
+            ok = false;
+            break;
           }
-          for (int h = 0; h < 2 && ok; ++h) {
-            if (!mbar_wait(&c.pds_full[h], qc & 1, status, lim)) { ok = false; break; }
-            if (first && h == 0 && n_units >= 1 && !mbar_wait(&c.acc_free, (n_units - 1) & 1, status, lim)) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
+          tc_fence_after();
+          if (leader) {
             // dV += P^T dO over the half's 64 rows (A = P^T_h from TMEM)
 #pragma unroll
             for (int k4 = 0; k4 < 4; ++k4) {
               const uint32_t acc = (first && h == 0 && k4 == 0) ? 0u : 1u;
               umma_bf16_ts(tmem + kColDV, tmem + col_a(h) + 8 * k4,
-                           sdesc_sw128(sDO + (64 * h + 16 * k4) * 128, 16384, 1024), idKV, acc);
+                           sdesc_add(dDO_mn, s * kTileBytes + (64 * h + 16 * k4) * 128), idKV, acc);
             }
             umma_commit(&c.dv_done[h]);
             if (h == 1) umma_commit(&c.do_empty[s]);
@@ -257,31 +271,36 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
             for (int k4 = 0; k4 < 4; ++k4) {
               const uint32_t acc = (first && h == 0 && k4 == 0) ? 0u : 1u;
-              umma_bf16(tmem + kColDK, sdesc_sw128(sDS + h * 16384 + k4 * 32, 16, 1024),
-                        sdesc_sw128(sQ + (64 * h + 16 * k4) * 128, 16384, 1024), idKV, acc);
+              umma_bf16(tmem + kColDK, sdesc_add(dS_k, h * 16384 + k4 * 32),
+                        sdesc_add(dQ_mn, s * kTileBytes + (64 * h + 16 * k4) * 128), idKV, acc);
             }
             if (h == 1) umma_commit(&c.q_empty[s]);
             // dQ^T of the half's rows = K^T dS^T -> B_h
 #pragma unroll
             for (int ks = 0; ks < 128 / 16; ++ks)
-              umma_bf16(tmem + col_b(h), sdesc_sw128(sK + ks * 2048, 16384, 1024),
-                        sdesc_sw128(sDS + h * 16384 + ks * 2048, 16384, 1024), idQ, ks > 0);
+              umma_bf16(tmem + col_b(h), sdesc_add(dK_mn, ks * 2048), sdesc_add(dS_mn, h * 16384 + ks * 2048), idQ,
+                        ks > 0);
             umma_commit(&c.dq_full[h]);
-            // this half of the unit's next tile, as soon as A_h and B_h are free
-            if (nxt < U.mt_end && !issue_sdp(qc + 1, h)) { ok = false; break; }
           }
-          if (!ok) break;
-          first = false;
-          ++qc;
+          __syncwarp();
+          // this half of the unit's next tile, as soon as A_h and B_h are free
+          if (nxt < U.mt_end && !issue_sdp(qc + 1, h)) { ok = false; break; }
         }
         if (!ok) break;
+        first = false;
+        ++qc;
+      }
+      if (!ok) break;
+      if (leader) {
         if (!first) umma_commit(&c.kv_empty);  // K/V were loaded for this unit
         umma_commit(&c.acc_full);
-        ++n_units;
       }
-      umma_commit(&c.final_mma);
-      mbar_wait(&c.final_mma, 0, nullptr, lim);
+      __syncwarp();
+      ++n_units;
     }
+    if (leader) umma_commit(&c.final_mma);
+    __syncwarp();
+    mbar_wait_warp(&c.final_mma, 0, nullptr, lim);
   } else if (warp >= 4) {
     // ------------------------- softmax gradient, dQ drain, dK/dV epilogue
     const int wg = (warp - 4) >> 2;          // warpgroup: rows [64 wg, 64 wg + 64) of the tile

@@ -153,6 +153,17 @@ __device__ __forceinline__ void umma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, u
       : "memory");
 }
 
+// True on one lane of the converged warp (elect.sync). An MMA-issuing warp runs
+// its loop on all 32 lanes, so that stage indices and descriptors are
+// warp-uniform values, and issues the MMAs from the elected lane: the same
+// instruction stream issued from a single-lane branch costs 20 to 45 % more
+// cycles per N=64 MMA on the tensor pipe.
+__device__ __forceinline__ bool elect_one() {
+  uint32_t pred = 0;
+  asm volatile("{\n\t.reg .pred P;\n\telect.sync _|P, 0xffffffff;\n\tselp.b32 %0, 1, 0, P;\n\t}" : "=r"(pred));
+  return pred != 0;
+}
+
 // Arrives once on `bar` when every tcgen05.mma issued so far by this thread
 // has completed.
 __device__ __forceinline__ void umma_commit(uint64_t* bar) {
@@ -187,6 +198,11 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo, ui
   d |= static_cast<uint64_t>(2) << 61;  // SWIZZLE_128B
   return d;
 }
+
+// The descriptor of the same operand `bytes` further on (a K step, a row block,
+// a pipeline stage): the start-address field holds address >> 4 in 14 bits,
+// and every shared-memory address is below 2^18, so the field never carries.
+__device__ __forceinline__ uint64_t sdesc_add(uint64_t desc, uint32_t bytes) { return desc + (bytes >> 4); }
 
 // 32 lanes x 32 consecutive fp32 columns: thread t of the warp gets TMEM lane
 // (32 * (warp % 4) + t), register j holds column (col + j).
