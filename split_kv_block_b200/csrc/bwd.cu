@@ -149,69 +149,88 @@ __global__ void __launch_bounds__(256, 1)
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------- MMA issuer
-    if (lane == 0) {
+    // All 32 lanes run the loop (stage indices and descriptors stay warp-uniform); one elected lane issues
+    // the MMAs and their commits.
+    {
+      const bool leader = elect_one();
       constexpr uint32_t idS = idesc_bf16(128, 128, false, false);  // S^T, dP^T
       constexpr uint32_t idKV = idesc_bf16(128, D, false, true);    // dV, dK
       constexpr uint32_t idQ = idesc_bf16(128, D, true, true);      // dQ
-      const uint32_t sK = smem_u32(smem + L::kK), sV = smem_u32(smem + L::kV), sQ = smem_u32(smem + L::kQ),
-                     sDO = smem_u32(smem + L::kDO), sPt = smem_u32(smem + L::kPt), sDSt = smem_u32(smem + L::kDSt);
+      // operand descriptors at their buffers' starts; K steps are byte offsets
+      const uint64_t dK_k = sdesc_sw128(smem_u32(smem + L::kK), 16, 1024);
+      const uint64_t dV_k = sdesc_sw128(smem_u32(smem + L::kV), 16, 1024);
+      const uint64_t dQ_k = sdesc_sw128(smem_u32(smem + L::kQ), 16, 1024);
+      const uint64_t dDO_k = sdesc_sw128(smem_u32(smem + L::kDO), 16, 1024);
+      const uint64_t dPt_k = sdesc_sw128(smem_u32(smem + L::kPt), 16, 1024);
+      const uint64_t dDSt_k = sdesc_sw128(smem_u32(smem + L::kDSt), 16, 1024);
+      const uint64_t dDO_mn = sdesc_sw128(smem_u32(smem + L::kDO), 128 * 128, 1024);
+      const uint64_t dQ_mn = sdesc_sw128(smem_u32(smem + L::kQ), 128 * 128, 1024);
+      const uint64_t dDSt_mn = sdesc_sw128(smem_u32(smem + L::kDSt), 128 * 128, 1024);
+      const uint64_t dK_mn = sdesc_sw128(smem_u32(smem + L::kK), 128 * 128, 1024);
       uint32_t n_units = 0, qc = 0;
       bool ok = true;
       while (ok) {
         const int slot = n_units & 1;
-        if (!mbar_wait(&sh.sched_full[slot], (n_units >> 1) & 1, status, lim)) break;
+        if (!mbar_wait_warp(&sh.sched_full[slot], (n_units >> 1) & 1, status, lim)) break;
         const int u = sh.sched[slot];
-        mbar_arrive(&sh.sched_empty[slot]);
+        __syncwarp();
+        if (leader) mbar_arrive(&sh.sched_empty[slot]);
         if (u < 0) break;
         const BwdUnit U = p.units[u];
-        if (!mbar_wait(&sh.kv_full, n_units & 1, status, lim)) break;
+        if (!mbar_wait_warp(&sh.kv_full, n_units & 1, status, lim)) break;
         tc_fence_after();
         bool first = true;
         for (int mt = U.mt_begin; mt < U.mt_end && ok; ++mt) {
           if (p.mtiles[mt].kmax <= U.kbeg) continue;
-          if (!mbar_wait(&sh.q_full, qc & 1, status, lim)) { ok = false; break; }
+          if (!mbar_wait_warp(&sh.q_full, qc & 1, status, lim)) { ok = false; break; }
           tc_fence_after();
+          if (leader) {
 #pragma unroll
-          for (int ks = 0; ks < D / 16; ++ks) {
-            const uint32_t off = (ks >> 2) * (128 * 128) + (ks & 3) * 32;
-            umma_bf16(tmem + kColS, sdesc_sw128(sK + off, 16, 1024), sdesc_sw128(sQ + off, 16, 1024), idS, ks > 0);
+            for (int ks = 0; ks < D / 16; ++ks) {
+              const uint32_t off = (ks >> 2) * (128 * 128) + (ks & 3) * 32;
+              umma_bf16(tmem + kColS, sdesc_add(dK_k, off), sdesc_add(dQ_k, off), idS, ks > 0);
+            }
           }
-          if (qc >= 1 && !mbar_wait(&sh.dq_free, (qc - 1) & 1, status, lim)) { ok = false; break; }
+          __syncwarp();
+          if (qc >= 1 && !mbar_wait_warp(&sh.dq_free, (qc - 1) & 1, status, lim)) { ok = false; break; }
           tc_fence_after();
+          if (leader) {
 #pragma unroll
-          for (int ks = 0; ks < D / 16; ++ks) {
-            const uint32_t off = (ks >> 2) * (128 * 128) + (ks & 3) * 32;
-            umma_bf16(tmem + kColDP, sdesc_sw128(sV + off, 16, 1024), sdesc_sw128(sDO + off, 16, 1024), idS,
-                      ks > 0);
+            for (int ks = 0; ks < D / 16; ++ks) {
+              const uint32_t off = (ks >> 2) * (128 * 128) + (ks & 3) * 32;
+              umma_bf16(tmem + kColDP, sdesc_add(dV_k, off), sdesc_add(dDO_k, off), idS, ks > 0);
+            }
+            umma_commit(&sh.sdp_full);
           }
-          umma_commit(&sh.sdp_full);
-          if (!mbar_wait(&sh.pds_full, qc & 1, status, lim)) { ok = false; break; }
-          if (first && n_units >= 1 && !mbar_wait(&sh.acc_free, (n_units - 1) & 1, status, lim)) { ok = false; break; }
+          __syncwarp();
+          if (!mbar_wait_warp(&sh.pds_full, qc & 1, status, lim)) { ok = false; break; }
+          if (first && n_units >= 1 && !mbar_wait_warp(&sh.acc_free, (n_units - 1) & 1, status, lim)) { ok = false; break; }
           tc_fence_after();
+          if (leader) {
 #pragma unroll
-          for (int ks = 0; ks < 128 / 16; ++ks) {  // reduction over the tile rows
-            const uint32_t aoff = (ks >> 2) * (128 * 128) + (ks & 3) * 32;
-            const uint32_t acc = (!first || ks > 0) ? 1u : 0u;
-            umma_bf16(tmem + kColDV, sdesc_sw128(sPt + aoff, 16, 1024), sdesc_sw128(sDO + ks * 2048, 128 * 128, 1024),
-                      idKV, acc);
-            umma_bf16(tmem + kColDK, sdesc_sw128(sDSt + aoff, 16, 1024), sdesc_sw128(sQ + ks * 2048, 128 * 128, 1024),
-                      idKV, acc);
-          }
+            for (int ks = 0; ks < 128 / 16; ++ks) {  // reduction over the tile rows
+              const uint32_t aoff = (ks >> 2) * (128 * 128) + (ks & 3) * 32;
+              const uint32_t acc = (!first || ks > 0) ? 1u : 0u;
+              umma_bf16(tmem + kColDV, sdesc_add(dPt_k, aoff), sdesc_add(dDO_mn, ks * 2048), idKV, acc);
+              umma_bf16(tmem + kColDK, sdesc_add(dDSt_k, aoff), sdesc_add(dQ_mn, ks * 2048), idKV, acc);
+            }
 #pragma unroll
-          for (int ks = 0; ks < 128 / 16; ++ks) {  // reduction over the tile keys
-            umma_bf16(tmem + kColDQ, sdesc_sw128(sDSt + ks * 2048, 128 * 128, 1024),
-                      sdesc_sw128(sK + ks * 2048, 128 * 128, 1024), idQ, ks > 0);
+            for (int ks = 0; ks < 128 / 16; ++ks)  // reduction over the tile keys
+              umma_bf16(tmem + kColDQ, sdesc_add(dDSt_mn, ks * 2048), sdesc_add(dK_mn, ks * 2048), idQ, ks > 0);
+            umma_commit(&sh.q_empty);
+            umma_commit(&sh.dq_full);
           }
-          umma_commit(&sh.q_empty);
-          umma_commit(&sh.dq_full);
+          __syncwarp();
           first = false;
           ++qc;
         }
-        umma_commit(&sh.kv_empty);
+        if (leader) umma_commit(&sh.kv_empty);
+        __syncwarp();
         ++n_units;
       }
-      umma_commit(&sh.final_mma);
-      mbar_wait(&sh.final_mma, 0, nullptr, lim);
+      if (leader) umma_commit(&sh.final_mma);
+      __syncwarp();
+      mbar_wait_warp(&sh.final_mma, 0, nullptr, lim);
     }
   } else if (warp >= 4) {
     // ------------------------------- softmax gradient, dQ drain, dK/dV epilogue

@@ -156,36 +156,45 @@ __global__ void __launch_bounds__(256, 1)
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------- MMA issuer
-    if (lane == 0) {
+    // All 32 lanes run the loop (stage indices and descriptors stay warp-uniform); one elected lane issues
+    // the MMAs and their commits.
+    {
+      const bool leader = elect_one();
       constexpr uint32_t idS = idesc_bf16(kTileM, kTileN, false, false);
       constexpr uint32_t idO = idesc_bf16(kTileM, D, false, true);
-      const uint32_t sQ = smem_u32(smem + L::kQ), sK = smem_u32(smem + L::kK0), sV = smem_u32(smem + L::kV0),
-                     sP = smem_u32(smem + L::kP);
+      // operand descriptors at their buffers' starts; K steps and stages are byte offsets
+      const uint64_t dQ_k = sdesc_sw128(smem_u32(smem + L::kQ), 16, 1024);
+      const uint64_t dK_k = sdesc_sw128(smem_u32(smem + L::kK0), 16, 1024);
+      const uint64_t dP_k = sdesc_sw128(smem_u32(smem + L::kP), 16, 1024);
+      const uint64_t dV_mn = sdesc_sw128(smem_u32(smem + L::kV0), kTileN * 128, 1024);
       uint32_t n_units = 0, kv = 0, tcount = 0, pcount = 0;
       bool ok = true;
       while (ok) {
         const int slot = n_units & 1;
-        if (!mbar_wait(&bars.sched_full[slot], (n_units >> 1) & 1, status, lim)) break;
+        if (!mbar_wait_warp(&bars.sched_full[slot], (n_units >> 1) & 1, status, lim)) break;
         const int u = bars.sched[slot];
-        mbar_arrive(&bars.sched_empty[slot]);
+        __syncwarp();
+        if (leader) mbar_arrive(&bars.sched_empty[slot]);
         if (u < 0) break;
         const FwdUnit U = p.units[u];
         const int nt = (U.kend - U.kbeg + kTileN - 1) / kTileN;
-        if (!mbar_wait(&bars.q_full, n_units & 1, status, lim)) break;
+        if (!mbar_wait_warp(&bars.q_full, n_units & 1, status, lim)) break;
         tc_fence_after();
         auto issue_s = [&](uint32_t t_index, uint32_t kv_index) -> bool {
           const int st = kv_index & 1;
-          if (!mbar_wait(&bars.k_full[st], (kv_index >> 1) & 1, status, lim)) return false;
+          if (!mbar_wait_warp(&bars.k_full[st], (kv_index >> 1) & 1, status, lim)) return false;
           tc_fence_after();
           const uint32_t dS = tmem + ((t_index & 1) ? kColS1 : kColS0);
-          const uint32_t kbase = sK + st * L::kKVBytes;
+          if (leader) {
 #pragma unroll
-          for (int ks = 0; ks < D / 16; ++ks) {
-            const uint32_t off = (ks >> 2) * (kTileM * 128) + (ks & 3) * 32;
-            umma_bf16(dS, sdesc_sw128(sQ + off, 16, 1024), sdesc_sw128(kbase + off, 16, 1024), idS, ks > 0);
+            for (int ks = 0; ks < D / 16; ++ks) {
+              const uint32_t off = (ks >> 2) * (kTileM * 128) + (ks & 3) * 32;
+              umma_bf16(dS, sdesc_add(dQ_k, off), sdesc_add(dK_k, st * L::kKVBytes + off), idS, ks > 0);
+            }
+            umma_commit(&bars.k_empty[st]);
+            umma_commit(&bars.s_full[t_index & 1]);
           }
-          umma_commit(&bars.k_empty[st]);
-          umma_commit(&bars.s_full[t_index & 1]);
+          __syncwarp();
           return true;
         };
         if (!issue_s(tcount, kv)) break;
@@ -194,30 +203,34 @@ __global__ void __launch_bounds__(256, 1)
           if (j + 1 < nt) {
             if (!issue_s(tj + 1, kvj + 1)) { ok = false; break; }
           }
-          if (j + 1 == nt) umma_commit(&bars.q_empty);
-          if (!mbar_wait(&bars.p_full, pcount & 1, status, lim)) { ok = false; break; }
+          if (leader && j + 1 == nt) umma_commit(&bars.q_empty);
+          __syncwarp();
+          if (!mbar_wait_warp(&bars.p_full, pcount & 1, status, lim)) { ok = false; break; }
           ++pcount;
           const int st = kvj & 1;
-          if (!mbar_wait(&bars.v_full[st], (kvj >> 1) & 1, status, lim)) { ok = false; break; }
-          if (j == 0 && n_units >= 1 && !mbar_wait(&bars.o_free, (n_units - 1) & 1, status, lim)) { ok = false; break; }
+          if (!mbar_wait_warp(&bars.v_full[st], (kvj >> 1) & 1, status, lim)) { ok = false; break; }
+          if (j == 0 && n_units >= 1 && !mbar_wait_warp(&bars.o_free, (n_units - 1) & 1, status, lim)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t vbase = sV + st * L::kKVBytes;
+          if (leader) {
 #pragma unroll
-          for (int ks = 0; ks < kTileN / 16; ++ks) {
-            const uint32_t aoff = (ks >> 2) * (kTileM * 128) + (ks & 3) * 32;
-            umma_bf16(tmem + kColO, sdesc_sw128(sP + aoff, 16, 1024),
-                      sdesc_sw128(vbase + ks * 2048, kTileN * 128, 1024), idO, (j > 0 || ks > 0) ? 1u : 0u);
+            for (int ks = 0; ks < kTileN / 16; ++ks) {
+              const uint32_t aoff = (ks >> 2) * (kTileM * 128) + (ks & 3) * 32;
+              umma_bf16(tmem + kColO, sdesc_add(dP_k, aoff), sdesc_add(dV_mn, st * L::kKVBytes + ks * 2048), idO,
+                        (j > 0 || ks > 0) ? 1u : 0u);
+            }
+            umma_commit(&bars.v_empty[st]);
+            umma_commit(&bars.o_done);
           }
-          umma_commit(&bars.v_empty[st]);
-          umma_commit(&bars.o_done);
+          __syncwarp();
         }
         tcount += nt;
         kv += nt;
         ++n_units;
       }
       // every MMA issued by this thread completes before TMEM is released
-      umma_commit(&bars.final_mma);
-      mbar_wait(&bars.final_mma, 0, nullptr, lim);
+      if (leader) umma_commit(&bars.final_mma);
+      __syncwarp();
+      mbar_wait_warp(&bars.final_mma, 0, nullptr, lim);
     }
   } else if (warp >= 4) {
     // ------------------------------------------- softmax / correction / epilogue

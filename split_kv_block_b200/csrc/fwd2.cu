@@ -211,7 +211,10 @@ __global__ void __launch_bounds__(384, 1)
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------- MMA issuer
-    if (lane == 0) {
+    {
+      // All 32 lanes run the loop (stage indices and counters stay warp-uniform); one elected lane issues
+      // the MMAs and their commits.
+      const bool leader = elect_one();
       constexpr uint32_t idS = idesc_bf16(128, 128, false, false);  // S = Q K^T
       constexpr uint32_t idO = idesc_bf16(128, kD, false, true);    // O += P V (P from TMEM)
       const uint64_t dQ0 = sdesc_sw128(smem_u32(smem + kQ0), 16, 1024);
@@ -224,43 +227,50 @@ __global__ void __launch_bounds__(384, 1)
       // S of tile t for key step with K stage st
       auto issue_s = [&](int t, int st) {
         const uint64_t dq = dQ0 + t * kTileDesc, dk = dK0 + st * kTileDesc;
+        if (leader) {
 #pragma unroll
-        for (int ks = 0; ks < kD / 16; ++ks) umma_bf16(tmem + col_s(t), dq + kmaj(ks), dk + kmaj(ks), idS, ks > 0);
-        umma_commit(&c.s_full[t]);
+          for (int ks = 0; ks < kD / 16; ++ks) umma_bf16(tmem + col_s(t), dq + kmaj(ks), dk + kmaj(ks), idS, ks > 0);
+          umma_commit(&c.s_full[t]);
+        }
+        __syncwarp();
         ++s_cnt[t];
       };
       // O of tile t += P V with V stage st
       auto issue_pv = [&](int t, int st, bool accumulate) {
         const uint64_t dv = dV0 + st * kTileDesc;
+        if (leader) {
 #pragma unroll
-        for (int ks = 0; ks < 128 / 16; ++ks)
-          umma_bf16_ts(tmem + col_o(t), tmem + col_s(t) + 8 * ks, dv + ((ks * 2048) >> 4), idO,
-                       (accumulate || ks > 0) ? 1u : 0u);
-        umma_commit(&c.pv_done[t]);
+          for (int ks = 0; ks < 128 / 16; ++ks)
+            umma_bf16_ts(tmem + col_o(t), tmem + col_s(t) + 8 * ks, dv + ((ks * 2048) >> 4), idO,
+                         (accumulate || ks > 0) ? 1u : 0u);
+          umma_commit(&c.pv_done[t]);
+        }
+        __syncwarp();
         ++pv_cnt[t];
       };
       // S of tile t overwrites the P that the tile's last PV read: wait for that PV
       auto wait_pv = [&](int t) -> bool {
-        return pv_cnt[t] == 0 || mbar_wait(&c.pv_done[t], (pv_cnt[t] - 1) & 1, status, lim);
+        return pv_cnt[t] == 0 || mbar_wait_warp(&c.pv_done[t], (pv_cnt[t] - 1) & 1, status, lim);
       };
       while (ok) {
         const int slot = n_units & 1;
-        if (!mbar_wait(&c.sched_full[slot], (n_units >> 1) & 1, status, lim)) break;
+        if (!mbar_wait_warp(&c.sched_full[slot], (n_units >> 1) & 1, status, lim)) break;
         const int u = c.sched[slot];
-        mbar_arrive(&c.sched_empty[slot]);
+        __syncwarp();
+        if (leader) mbar_arrive(&c.sched_empty[slot]);
         if (u < 0) break;
         const FwdPair pr = p.pairs[u];
         const bool has[2] = {pr.slot[0] >= 0, pr.slot[1] >= 0};
         const int nt = (pr.kend - pr.kbeg + kTileN - 1) / kTileN;
         for (int t = 0; t < 2 && ok; ++t) {
           if (!has[t]) continue;
-          if (!mbar_wait(&c.q_full[t], q_use[t] & 1, status, lim)) { ok = false; break; }
+          if (!mbar_wait_warp(&c.q_full[t], q_use[t] & 1, status, lim)) { ok = false; break; }
         }
         if (!ok) break;
         // key step 0: S of both tiles
         {
           const int st = kv & 1;
-          if (!mbar_wait(&c.k_full[st], (kv >> 1) & 1, status, lim)) break;
+          if (!mbar_wait_warp(&c.k_full[st], (kv >> 1) & 1, status, lim)) break;
           for (int t = 0; t < 2 && ok; ++t) {
             if (!has[t]) continue;
             if (!wait_pv(t)) { ok = false; break; }
@@ -268,22 +278,25 @@ __global__ void __launch_bounds__(384, 1)
             issue_s(t, st);
           }
           if (!ok) break;
-          umma_commit(&c.k_empty[st]);
-          if (nt == 1)
-            for (int t = 0; t < 2; ++t)
-              if (has[t]) umma_commit(&c.q_empty[t]);
+          if (leader) {
+            umma_commit(&c.k_empty[st]);
+            if (nt == 1)
+              for (int t = 0; t < 2; ++t)
+                if (has[t]) umma_commit(&c.q_empty[t]);
+          }
+          __syncwarp();
         }
         for (int j = 0; j < nt && ok; ++j) {
           const int st = (kv + j) & 1, st1 = (kv + j + 1) & 1;
           const uint32_t use = (kv + j) >> 1, use1 = (kv + j + 1) >> 1;
-          if (!mbar_wait(&c.v_full[st], use & 1, status, lim)) { ok = false; break; }
-          if (j + 1 < nt && !mbar_wait(&c.k_full[st1], use1 & 1, status, lim)) { ok = false; break; }
+          if (!mbar_wait_warp(&c.v_full[st], use & 1, status, lim)) { ok = false; break; }
+          if (j + 1 < nt && !mbar_wait_warp(&c.k_full[st1], use1 & 1, status, lim)) { ok = false; break; }
           for (int t = 0; t < 2 && ok; ++t) {
             if (!has[t]) continue;
             // O_t += P_t V: P from the tile's softmax warpgroup
-            if (!mbar_wait(&c.p_full[t], p_cnt[t] & 1, status, lim)) { ok = false; break; }
+            if (!mbar_wait_warp(&c.p_full[t], p_cnt[t] & 1, status, lim)) { ok = false; break; }
             ++p_cnt[t];
-            if (j == 0 && unit_cnt[t] >= 1 && !mbar_wait(&c.o_free[t], (unit_cnt[t] - 1) & 1, status, lim)) {
+            if (j == 0 && unit_cnt[t] >= 1 && !mbar_wait_warp(&c.o_free[t], (unit_cnt[t] - 1) & 1, status, lim)) {
               ok = false;
               break;
             }
@@ -294,12 +307,16 @@ __global__ void __launch_bounds__(384, 1)
               if (!wait_pv(t)) { ok = false; break; }
               tc_fence_after();
               issue_s(t, st1);
-              if (j + 2 == nt) umma_commit(&c.q_empty[t]);
+              if (leader && j + 2 == nt) umma_commit(&c.q_empty[t]);
+              __syncwarp();
             }
           }
           if (!ok) break;
-          umma_commit(&c.v_empty[st]);
-          if (j + 1 < nt) umma_commit(&c.k_empty[st1]);
+          if (leader) {
+            umma_commit(&c.v_empty[st]);
+            if (j + 1 < nt) umma_commit(&c.k_empty[st1]);
+          }
+          __syncwarp();
         }
         if (!ok) break;
         for (int t = 0; t < 2; ++t)
@@ -310,8 +327,9 @@ __global__ void __launch_bounds__(384, 1)
         kv += nt;
         ++n_units;
       }
-      umma_commit(&c.final_mma);
-      mbar_wait(&c.final_mma, 0, nullptr, lim);
+      if (leader) umma_commit(&c.final_mma);
+      __syncwarp();
+      mbar_wait_warp(&c.final_mma, 0, nullptr, lim);
     }
   } else if (warp >= 4) {
     // ---------------------------------------------- softmax + epilogue of tile t
