@@ -241,10 +241,16 @@ __global__ void __launch_bounds__(384, 1)
       if (u < 0) break;
       const BwdUnit U = p.units[u];
       bool first = true;
-      for (int mt = U.mt_begin; mt < U.mt_end; ++mt) {
-        if (p.mtiles[mt].kmax <= U.kbeg) continue;
-        int nxt = mt + 1;  // the unit's next live query tile
-        while (nxt < U.mt_end && p.mtiles[nxt].kmax <= U.kbeg) ++nxt;
+      // live query tiles in order (mt, then nxt); the liveness of the tile after nxt is loaded at the top of
+      // a tile and read at its end, so no load stalls the issue of a tile's MMAs
+      auto live_from = [&](int i) -> int {
+        while (i < U.mt_end && p.mtiles[i].kmax <= U.kbeg) ++i;
+        return i;
+      };
+      int mt = live_from(U.mt_begin);
+      int nxt = mt < U.mt_end ? live_from(mt + 1) : U.mt_end;
+      while (mt < U.mt_end) {
+        const int kmax_c = (nxt < U.mt_end && nxt + 1 < U.mt_end) ? p.mtiles[nxt + 1].kmax : 0;
         const int s = qc & 1;
         if (first) {  // a unit's first tile waits for the unit's K/V
           if (!mbar_wait_warp(&c.kv_full, (kv_waits++) & 1, status, lim)) { ok = false; break; }
@@ -289,6 +295,13 @@ __global__ void __launch_bounds__(384, 1)
         if (!ok) break;
         first = false;
         ++qc;
+        int nn = U.mt_end;
+        if (nxt < U.mt_end) {
+          nn = nxt + 1;
+          if (nn < U.mt_end && kmax_c <= U.kbeg) nn = live_from(nn + 1);
+        }
+        mt = nxt;
+        nxt = nn;
       }
       if (!ok) break;
       if (leader) {
@@ -312,19 +325,28 @@ __global__ void __launch_bounds__(384, 1)
     const size_t tok_stride = static_cast<size_t>(p.Hq) * kD;
     uint32_t n_units = 0, qc = 0;
     bool ok = true;
-    // metadata of the next live query tile, fetched one tile ahead (threads t < 64: row 64 wg + t)
-    float pf_lse = INFINITY, pf_del = 0.f;
-    int pf_ke = 0;
-    auto fetch = [&](const MTile& M, const BwdUnit& U, int nkeys) {
+    // Row metadata (LSE, D, key end) of the next live query tile, loaded one tile ahead by threads t < 64
+    // (row 64 wg + t) and used only when staged for that tile: the loads never stall the current tile.
+    // Rows past the tile's tokens read token tok0 (a valid address) and are masked when staged.
+    float rw_lse = 0.f, rw_del = 0.f;
+    int rw_ke = 0;
+    bool rw_valid = false;
+    auto fetch = [&](const MTile& Mx, int g) {
       if (t < 64) {
         const int r = 64 * wg + t;
         const int tl = r >> lgG;
-        const bool valid = tl < M.ntok;
-        const int token = M.tok0 + tl, head = U.g * G + (r & (G - 1));
-        pf_lse = valid ? p.lse[static_cast<size_t>(token) * p.Hq + head] * kLog2e : INFINITY;
-        pf_del = valid ? p.delta[static_cast<size_t>(token) * p.Hq + head] : 0.f;
-        pf_ke = valid ? max(0, min(min(p.tok_kend[token], U.kend) - U.kbeg, nkeys)) : 0;
+        rw_valid = tl < Mx.ntok;
+        const int token = Mx.tok0 + (rw_valid ? tl : 0), head = g * G + (r & (G - 1));
+        rw_lse = p.lse[static_cast<size_t>(token) * p.Hq + head];
+        rw_del = p.delta[static_cast<size_t>(token) * p.Hq + head];
+        rw_ke = p.tok_kend[token];
       }
+    };
+    // the next live query tile of unit U at or after index i (the scan loads only at unit starts and when
+    // a prefetched candidate is dead)
+    auto live_from = [&](const BwdUnit& U, int i) -> int {
+      while (i < U.mt_end && p.mtiles[i].kmax <= U.kbeg) ++i;
+      return i;
     };
     while (ok) {
       const int slot = n_units & 1;
@@ -336,12 +358,19 @@ __global__ void __launch_bounds__(384, 1)
       const BwdUnit U = p.units[u];
       if (p.stamps && tid == 128) p.stamps[2 * u] = static_cast<long long>(globaltimer_ns());
       const int nkeys = U.kend - U.kbeg;
-      int mt = U.mt_begin;
-      while (mt < U.mt_end && p.mtiles[mt].kmax <= U.kbeg) ++mt;
-      MTile M{};
+      // live tiles in order: mt (M), then nxt (Mn); cand is the tile after nxt, loaded one tile ahead (Mc)
+      int mt = live_from(U, U.mt_begin);
+      MTile M{}, Mn{}, Mc{};
+      int nxt = U.mt_end, cand = U.mt_end;
       if (mt < U.mt_end) {
         M = p.mtiles[mt];
-        fetch(M, U, nkeys);
+        fetch(M, U.g);
+        nxt = live_from(U, mt + 1);
+        if (nxt < U.mt_end) {
+          Mn = p.mtiles[nxt];
+          cand = nxt + 1;
+          if (cand < U.mt_end) Mc = p.mtiles[cand];
+        }
       }
       bool had_tiles = false;
       while (mt < U.mt_end) {
@@ -351,18 +380,29 @@ __global__ void __launch_bounds__(384, 1)
         // stage this tile's metadata, then fetch the next live tile's
         if (t < 64) {
           const int r = 64 * wg + t;
-          c.lse2[par][r] = pf_lse;
-          c.delta[par][r] = pf_del;
-          c.kend[par][r] = static_cast<uint8_t>(pf_ke);
-          const int wmin = __reduce_min_sync(0xffffffffu, pf_ke);
+          const int ke = rw_valid ? max(0, min(min(rw_ke, U.kend) - U.kbeg, nkeys)) : 0;
+          c.lse2[par][r] = rw_valid ? rw_lse * kLog2e : INFINITY;
+          c.delta[par][r] = rw_valid ? rw_del : 0.f;
+          c.kend[par][r] = static_cast<uint8_t>(ke);
+          const int wmin = __reduce_min_sync(0xffffffffu, ke);
           if (lane == 0) c.kmin[wg][par][warp & 1] = wmin;
         }
-        int nxt = mt + 1;
-        while (nxt < U.mt_end && p.mtiles[nxt].kmax <= U.kbeg) ++nxt;
-        MTile Mn = M;
+        // prefetch: the next tile's row metadata (from Mn, already in registers), then the tile after it from
+        // the candidate loaded one tile ago, and the candidate after that
+        int nn = U.mt_end;
+        MTile Mnn = Mn;
         if (nxt < U.mt_end) {
-          Mn = p.mtiles[nxt];
-          fetch(Mn, U, nkeys);
+          fetch(Mn, U.g);
+          nn = cand;
+          if (nn < U.mt_end) {
+            if (Mc.kmax > U.kbeg) {
+              Mnn = Mc;
+            } else {
+              nn = live_from(U, nn + 1);
+              if (nn < U.mt_end) Mnn = p.mtiles[nn];
+            }
+          }
+          if (nn < U.mt_end && nn + 1 < U.mt_end) Mc = p.mtiles[nn + 1];
         }
         mbar_arrive(&c.meta_full[wg][par]);
         if (!mbar_wait_warp(&c.meta_full[wg][par], (qc >> 1) & 1, status, lim)) { ok = false; break; }
@@ -455,6 +495,9 @@ __global__ void __launch_bounds__(384, 1)
         ++qc;
         M = Mn;
         mt = nxt;
+        Mn = Mnn;
+        nxt = nn;
+        cand = nn + 1;
       }
       if (!ok) break;
       // dV (warpgroup 0) / dK (warpgroup 1) of the unit's keys
