@@ -67,12 +67,18 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* s
                                           uint64_t limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
+  uint64_t next_check = t0 + 20000;
   while (true) {
     for (int i = 0; i < 64; ++i)
       if (mbar_try_wait(bar, parity)) return true;
+    // the status word is a global load: read it (and the limit) only once the wait has lasted 20 us, so that
+    // a phase completing during that load's latency is not noticed late in ordinary waits
+    const uint64_t now = globaltimer_ns();
+    if (now < next_check) continue;
+    next_check = now + 20000;
     // another role already gave up: leave too
     if (status && *reinterpret_cast<volatile int*>(status) != 0) return false;
-    if (globaltimer_ns() - t0 > limit_ns) {
+    if (now - t0 > limit_ns) {
       if (status) atomicCAS(status, 0, kStatusTimeout);
       return false;
     }
