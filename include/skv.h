@@ -242,7 +242,9 @@ int skv_attn_fwd_noalloc(const void* plan, const void* q, const void* k, const v
  * The outcome is read with skv_status(ws, stream). The pages have no
  * counterpart of this call; it tests this library's failure detection.
  * ws: device buffer of at least 256 bytes, 256-byte aligned, caller-owned;
- * its status word is cleared first. limit_ns: 1 .. 10^10.
+ * its status word is cleared first. limit_ns: 1 .. 10^10. A wait checks its
+ * limit (and the status word) only once it has lasted 20 us, and every 20 us
+ * after that, so it gives up between limit_ns and max(limit_ns, 20 us) + 20 us.
  * Returns SKV_EINVAL for a NULL or misaligned ws or a limit out of range,
  * SKV_ECUDA when the launch fails, SKV_OK otherwise.
  */
