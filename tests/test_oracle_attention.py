@@ -173,3 +173,26 @@ def test_merge_of_two_halves_by_hand():
     O, L = A.lse_merge([(o1, l1), dead, (o2, l2)])
     assert abs(float(L) - math.log(4.0)) < 1e-15
     assert torch.allclose(O, torch.tensor([[[0.75, 0.5]]], dtype=F64), atol=1e-15)
+
+
+def test_flops_fwd_hand_instance_and_mask_count():
+    """Forward FLOPs = 4 d per unmasked (query token, key, q-head) triple.
+    Hand instance: one 10-key sample, anchors 3 and 7, block_q 2, 4 q-heads,
+    d 8: 2 tokens x (3 + 7) keys x 4 heads = 80 triples, 4 * 8 * 80 = 2560.
+    Random ragged problems: the triples counted one by one from the explicit
+    boolean mask of every sample."""
+    prob = synth.small_problem([10], [[3, 7]], block_q=2, hq=4, hkv=2, d=8)
+    assert A.flops_fwd(prob) == 2560
+    rng = np.random.default_rng(21)
+    for _ in range(20):
+        prob = synth.random_small_problem(rng)
+        S = prob.block_q
+        triples = 0
+        for b in range(prob.num_samples):
+            k0, k1 = int(prob.ctx_offsets[b]), int(prob.ctx_offsets[b + 1])
+            for j in range(int(prob.anchor_offsets[b]), int(prob.anchor_offsets[b + 1])):
+                for _t in range(S):
+                    for kk in range(k1 - k0):
+                        if kk < int(prob.anchors[j]):
+                            triples += prob.num_q_heads
+        assert A.flops_fwd(prob) == 4 * prob.head_dim * triples
