@@ -134,35 +134,61 @@ int skv_plan_stats(const void* plan, int64_t* total_cost, int64_t* n_fwd_units, 
                    double* imbalance);
 
 /*
- * skv_attn_fwd — split-KV forward ("Split-KV's Core Mechanism": every KV
- * chunk's local attention for the global query set). For every forward work
- * unit, writes the chunk's normalized partial output (fp32) and LSE into the
- * workspace. Copies the device part of `plan` into `ws` first (the caller may
- * reuse `plan` once the call returns). q, k, v: device bf16 in the layouts
- * above. Enqueued on `stream`.
+ * Plan and problem. Every call that runs kernels takes the plan together
+ * with `prob`, the problem the caller's tensors are shaped for (host, read
+ * during the call only). The plan must have been written by skv_plan for that
+ * same problem: same scalars, context offsets, anchor offsets and anchors
+ * (skv_plan stores a 64-bit hash of them in the plan). Otherwise the call
+ * returns SKV_EPLAN before it enqueues anything, so a plan never drives the
+ * kernels over tensors of another problem's sizes. NULL plan or prob:
+ * SKV_EINVAL.
  */
-int skv_attn_fwd(const void* plan, const void* q, const void* k, const void* v, void* ws, size_t ws_bytes,
-                 skv_stream_t stream);
+
+/*
+ * skv_attn_fwd — split-KV forward ("Split-KV: Breaking the Context
+ * Parallelism Bottleneck in Diffusion Drafter Training", section "Split-KV's
+ * Core Mechanism": every KV chunk's local attention for the global query
+ * set). For every forward work unit, writes the chunk's normalized partial
+ * output (fp32) and LSE into the workspace. Copies the device part of `plan`
+ * into `ws` first (the caller may reuse `plan` once the call returns).
+ * q, k, v: device bf16 in the layouts above. Enqueued on `stream`.
+ */
+int skv_attn_fwd(const void* plan, const skv_problem* prob, const void* q, const void* k, const void* v, void* ws,
+                 size_t ws_bytes, skv_stream_t stream);
 
 /*
  * skv_lse_merge — exact query-sized combine of the partials left in `ws` by
- * skv_attn_fwd (same plan, same stream order): per (token, q-head)
+ * skv_attn_fwd (same plan, same stream order). Source: "Split-KV: Breaking
+ * the Context Parallelism Bottleneck in Diffusion Drafter Training", section
+ * "Split-KV's Core Mechanism" (the partial results of every KV shard are
+ * aggregated through query-sized tensors, with results strictly consistent
+ * with the unsharded computation) and "Split-KV: Efficient Context
+ * Parallelism for Training Diffusion Drafters", Abstract (exact). Per
+ * (token, q-head):
  *   m = max_c LSE_c, LSE = m + ln sum_c exp(LSE_c - m),
  *   O = sum_c exp(LSE_c - LSE) O_c, chunks taken in ascending key order.
  * Writes o (device bf16 [Nq][Hq][d]) and lse (device fp32 [Nq][Hq]).
  */
-int skv_lse_merge(const void* plan, const void* ws, void* o, float* lse, skv_stream_t stream);
+int skv_lse_merge(const void* plan, const skv_problem* prob, const void* ws, void* o, float* lse,
+                  skv_stream_t stream);
 
 /*
- * skv_attn_bwd — gradients of the attention through the split: per KV item,
- * probabilities recomputed with the merged LSE; dK/dV of every key written
- * by the one item that owns it (zero for keys no query attends to); dQ summed
- * over items in fp32 inside the workspace, then rounded to bf16.
+ * skv_attn_bwd — gradients of the attention through the split. Source:
+ * "Split-KV: Breaking the Context Parallelism Bottleneck in Diffusion Drafter
+ * Training", section "Split-KV's Core Mechanism" (the split is exact, which
+ * gradient correctness relies on; key/value shards stay where they are and
+ * only query-sized tensors are combined) and "Split-KV: Efficient Context
+ * Parallelism for Training Diffusion Drafters", Abstract. Per KV item,
+ * probabilities are recomputed with the merged LSE and D = rowsum(dO * O);
+ * dK/dV of every key are written by the one item that owns it (zero for keys
+ * no query attends to); dQ is summed over items in fp32 inside the workspace,
+ * then rounded to bf16.
  * Inputs: q, k, v, o (bf16), lse (fp32, from skv_lse_merge), dout (bf16).
  * Outputs: dq, dk, dv (bf16, fully overwritten). Enqueued on `stream`.
  */
-int skv_attn_bwd(const void* plan, const void* q, const void* k, const void* v, const void* o, const float* lse,
-                 const void* dout, void* dq, void* dk, void* dv, void* ws, size_t ws_bytes, skv_stream_t stream);
+int skv_attn_bwd(const void* plan, const skv_problem* prob, const void* q, const void* k, const void* v,
+                 const void* o, const float* lse, const void* dout, void* dq, void* dk, void* dv, void* ws,
+                 size_t ws_bytes, skv_stream_t stream);
 
 /*
  * skv_status — synchronizes `stream`, reads the status word in `ws` and
@@ -212,10 +238,14 @@ int skv_set_timing_events(int kernel, void* start_event, void* end_event);
  * cudaMalloc, cudaFree, pinned staging or library allocator. The caller
  * passes the plan (host, from skv_plan), q, k, v (device bf16) and the outputs
  * o (device bf16 [Nq][Hq][d]) and lse (device fp32 [Nq][Hq]), as for
- * skv_attn_fwd + skv_lse_merge. The plan's device section is copied from
- * `plan` with cudaMemcpyAsync: from pageable memory the copy is staged before
- * the call returns; if `plan` is pinned, keep it unchanged until `stream`
- * has passed this call.
+ * skv_attn_fwd + skv_lse_merge, and `prob`, the problem the plan was made for
+ * (SKV_EPLAN otherwise, before anything is enqueued). The plan's device
+ * section is copied from `plan` with one cudaMemcpyAsync, with no staging of
+ * the library's own. From pageable host memory that copy may block the
+ * calling thread until earlier work on `stream` has drained, and it cannot be
+ * recorded inside a stream capture. Keep the plan in pinned memory instead
+ * (page-locked by the caller's framework) and leave it unchanged until
+ * `stream` has passed this call.
  *
  * The first call on a device looks up the array's device address (this may
  * load the library's device code); make it before any stream capture.
@@ -224,11 +254,24 @@ int skv_set_timing_events(int kernel, void* start_event, void* end_event);
  * streams or threads) race on the array. Returns SKV_ESCRATCH, before
  * enqueuing anything, when the problem's forward workspace (ws_fwd_bytes of
  * skv_plan_size) exceeds SKV_NOALLOC_SCRATCH_BYTES. A device-side wait that
- * gives up ends the kernels early but is not reported here; use skv_attn_fwd
- * and skv_status when that report is needed.
+ * gives up ends the kernels early and leaves SKV_ETIMEOUT in the status word
+ * inside the array; read it with skv_noalloc_status.
  */
-int skv_attn_fwd_noalloc(const void* plan, const void* q, const void* k, const void* v, void* o, float* lse,
-                         skv_stream_t stream);
+int skv_attn_fwd_noalloc(const void* plan, const skv_problem* prob, const void* q, const void* k, const void* v,
+                         void* o, float* lse, skv_stream_t stream);
+
+/*
+ * skv_noalloc_status — the status word left in the library's scratch array
+ * (on the current device) by the last skv_attn_fwd_noalloc call: SKV_OK, or
+ * the error a kernel of that call recorded (SKV_ETIMEOUT, SKV_EDEVICE), in
+ * which case o and lse of that call are invalid. Synchronizes `stream` and
+ * copies the 4-byte word to host memory; allocates nothing. Returns
+ * SKV_ECUDA if the copy or the synchronize failed. Like the scratch array,
+ * the word is shared by every call on the device: read it before the next
+ * skv_attn_fwd_noalloc call clears it. The pages have no counterpart of this
+ * call.
+ */
+int skv_noalloc_status(skv_stream_t stream);
 
 /*
  * skv_wait_selftest — exercises, without any fault, the bounded device-side

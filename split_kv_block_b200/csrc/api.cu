@@ -31,13 +31,6 @@ int cuda_fail(cudaError_t e) {
   return SKV_ECUDA;
 }
 
-const PlanHeader* header_of(const void* plan) {
-  if (!plan) return nullptr;
-  const PlanHeader* h = static_cast<const PlanHeader*>(plan);
-  if (h->magic != kPlanMagic || h->version != kPlanVersion) return nullptr;
-  return h;
-}
-
 // ------------------------------------------------------------ plan upload
 // The plan's device section is copied into the workspace from a pinned
 // staging slot owned by the library; each slot is reused only after the copy
@@ -192,17 +185,18 @@ extern "C" int skv_set_timing_events(int kernel, void* start_event, void* end_ev
   return SKV_OK;
 }
 
-extern "C" int skv_attn_fwd(const void* plan, const void* q, const void* k, const void* v, void* ws,
-                            size_t ws_bytes, skv_stream_t stream_) {
-  const PlanHeader* h = header_of(plan);
-  if (!h) return SKV_EPLAN;
+extern "C" int skv_attn_fwd(const void* plan, const skv_problem* prob, const void* q, const void* k,
+                            const void* v, void* ws, size_t ws_bytes, skv_stream_t stream_) {
+  int rc = SKV_OK;
+  const PlanHeader* h = checked_plan(plan, prob, &rc);
+  if (!h) return rc;
   if (!q || !k || !v || !ws) return SKV_EINVAL;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || reinterpret_cast<uintptr_t>(ws) % 256 != 0)
     return SKV_EINVAL;
   const WsLayout w = ws_layout(*h);
   if (ws_bytes < w.fwd_end) return SKV_EWORKSPACE;
   cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
-  int rc = prepare_ws(*h, plan, ws, w, stream);
+  rc = prepare_ws(*h, plan, ws, w, stream);
   if (rc != SKV_OK) return rc;
   if (h->n_fwd == 0) return SKV_OK;
   CUtensorMap tq, tk, tv;
@@ -236,9 +230,11 @@ extern "C" int skv_attn_fwd(const void* plan, const void* q, const void* k, cons
   return SKV_OK;
 }
 
-extern "C" int skv_lse_merge(const void* plan, const void* ws, void* o, float* lse, skv_stream_t stream_) {
-  const PlanHeader* h = header_of(plan);
-  if (!h) return SKV_EPLAN;
+extern "C" int skv_lse_merge(const void* plan, const skv_problem* prob, const void* ws, void* o, float* lse,
+                             skv_stream_t stream_) {
+  int rc = SKV_OK;
+  const PlanHeader* h = checked_plan(plan, prob, &rc);
+  if (!h) return rc;
   if (!ws || !o || !lse || !aligned16(o) || !aligned16(lse)) return SKV_EINVAL;
   const WsLayout w = ws_layout(*h);
   const uint8_t* dev = at<uint8_t>(ws, w.dev);
@@ -262,11 +258,12 @@ extern "C" int skv_lse_merge(const void* plan, const void* ws, void* o, float* l
   return SKV_OK;
 }
 
-extern "C" int skv_attn_bwd(const void* plan, const void* q, const void* k, const void* v, const void* o,
-                            const float* lse, const void* dout, void* dq, void* dk, void* dv, void* ws,
-                            size_t ws_bytes, skv_stream_t stream_) {
-  const PlanHeader* h = header_of(plan);
-  if (!h) return SKV_EPLAN;
+extern "C" int skv_attn_bwd(const void* plan, const skv_problem* prob, const void* q, const void* k,
+                            const void* v, const void* o, const float* lse, const void* dout, void* dq, void* dk,
+                            void* dv, void* ws, size_t ws_bytes, skv_stream_t stream_) {
+  int rc = SKV_OK;
+  const PlanHeader* h = checked_plan(plan, prob, &rc);
+  if (!h) return rc;
   if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv || !ws) return SKV_EINVAL;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse) || !aligned16(dout) ||
       !aligned16(dq) || !aligned16(dk) || !aligned16(dv) || reinterpret_cast<uintptr_t>(ws) % 256 != 0)
@@ -274,7 +271,7 @@ extern "C" int skv_attn_bwd(const void* plan, const void* q, const void* k, cons
   const WsLayout w = ws_layout(*h);
   if (ws_bytes < w.bwd_end) return SKV_EWORKSPACE;
   cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
-  int rc = prepare_ws(*h, plan, ws, w, stream);
+  rc = prepare_ws(*h, plan, ws, w, stream);
   if (rc != SKV_OK) return rc;
   cudaError_t e;
   float* delta = at<float>(ws, w.bwd_delta);

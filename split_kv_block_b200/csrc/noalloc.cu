@@ -24,8 +24,8 @@
 // per device, so calls whose work overlaps on the GPU (other streams, other
 // host threads) race on it. Problems whose workspace exceeds the array are
 // rejected with SKV_ESCRATCH before anything is enqueued. A device-side wait
-// that gives up ends the kernels early, but its status word stays inside the
-// array: use skv_attn_fwd with skv_status when that report is needed.
+// that gives up ends the kernels early and leaves its error in the status
+// word at the start of the array, which skv_noalloc_status reads back.
 #include <cuda_runtime.h>
 
 #include <cmath>
@@ -69,11 +69,11 @@ cudaError_t scratch_address(void** out) {
 
 using namespace skv;
 
-extern "C" int skv_attn_fwd_noalloc(const void* plan, const void* q, const void* k, const void* v, void* o,
-                                    float* lse, skv_stream_t stream_) {
-  if (!plan) return SKV_EPLAN;
-  const PlanHeader* h = static_cast<const PlanHeader*>(plan);
-  if (h->magic != kPlanMagic || h->version != kPlanVersion) return SKV_EPLAN;
+extern "C" int skv_attn_fwd_noalloc(const void* plan, const skv_problem* prob, const void* q, const void* k,
+                                    const void* v, void* o, float* lse, skv_stream_t stream_) {
+  int rc = SKV_OK;
+  const PlanHeader* h = checked_plan(plan, prob, &rc);
+  if (!h) return rc;
   if (!q || !k || !v || !o || !lse) return SKV_EINVAL;
   for (const void* ptr : {q, k, v, static_cast<const void*>(o), static_cast<const void*>(lse)})
     if (reinterpret_cast<uintptr_t>(ptr) % 16 != 0) return SKV_EINVAL;
@@ -93,7 +93,7 @@ extern "C" int skv_attn_fwd_noalloc(const void* plan, const void* q, const void*
   if (h->n_fwd == 0) return SKV_OK;
 
   CUtensorMap tq, tk, tv;
-  int rc = skv_make_tile_map(&tq, q, h->Nq, h->Hq, h->d, h->G, h->tile_tokens);
+  rc = skv_make_tile_map(&tq, q, h->Nq, h->Hq, h->d, h->G, h->tile_tokens);
   if (rc == SKV_OK) rc = skv_make_tile_map(&tk, k, h->Ltot, h->Hkv, h->d, 1, kTileN);
   if (rc == SKV_OK) rc = skv_make_tile_map(&tv, v, h->Ltot, h->Hkv, h->d, 1, kTileN);
   if (rc != SKV_OK) return rc;
@@ -137,4 +137,16 @@ extern "C" int skv_attn_fwd_noalloc(const void* plan, const void* q, const void*
   e = launch_merge(h->d, m, stream);
   if (e != cudaSuccess) return skv_record_cuda_error(static_cast<int>(e));
   return SKV_OK;
+}
+
+extern "C" int skv_noalloc_status(skv_stream_t stream_) {
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  void* ws = nullptr;
+  cudaError_t e = scratch_address(&ws);
+  if (e != cudaSuccess) return skv_record_cuda_error(static_cast<int>(e));
+  int st = 0;
+  e = cudaMemcpyAsync(&st, ws, sizeof(int), cudaMemcpyDeviceToHost, stream);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+  if (e != cudaSuccess) return skv_record_cuda_error(static_cast<int>(e));
+  return st;
 }

@@ -364,6 +364,16 @@ int build(const skv_problem* prob, int policy, Built& out, Prob& q) {
   return SKV_OK;
 }
 
+// FNV-1a over the bytes of each value in turn.
+struct Fnv {
+  uint64_t h = 0xcbf29ce484222325ull;
+  template <class T>
+  void add(const T& v) {
+    const auto* c = reinterpret_cast<const uint8_t*>(&v);
+    for (size_t i = 0; i < sizeof(T); ++i) h = (h ^ c[i]) * 0x100000001b3ull;
+  }
+};
+
 PlanHeader layout_of(const Prob& q, int policy, const Built& b) {
   PlanHeader h{};
   h.magic = kPlanMagic;
@@ -379,6 +389,7 @@ PlanHeader layout_of(const Prob& q, int policy, const Built& b) {
   h.n_bwd = static_cast<int64_t>(b.bwd.size());
   h.n_fwd_pairs = static_cast<int64_t>(b.pairs.size());
   h.imbalance = b.imbalance;
+  h.fingerprint = 0;  // set by skv_plan from the caller's problem
   uint64_t off = align_up(sizeof(PlanHeader), 256);
   h.items_off = off;
   off = align_up(off + b.items.size() * sizeof(skv_item), 64);
@@ -411,6 +422,46 @@ void copy_to(uint8_t* base, uint64_t off, const std::vector<T>& v) {
 }
 
 }  // namespace
+
+uint64_t problem_fingerprint(const skv_problem* p) {
+  Fnv f;
+  f.add(p->num_samples);
+  f.add(p->block_q);
+  f.add(p->chunk_kv);
+  f.add(p->sub_chunks);
+  f.add(p->num_partitions);
+  f.add(p->num_q_heads);
+  f.add(p->num_kv_heads);
+  f.add(p->head_dim);
+  for (int b = 0; b <= p->num_samples; ++b) {
+    f.add(p->ctx_offsets[b]);
+    f.add(p->anchor_offsets[b]);
+  }
+  const int32_t A = p->anchor_offsets[p->num_samples];
+  for (int32_t j = 0; j < A; ++j) f.add(p->anchors[j]);
+  return f.h;
+}
+
+const PlanHeader* checked_plan(const void* plan, const skv_problem* prob, int* rc) {
+  *rc = SKV_EINVAL;
+  if (!plan || !prob || prob->num_samples < 1 || !prob->ctx_offsets || !prob->anchor_offsets) return nullptr;
+  const PlanHeader* h = static_cast<const PlanHeader*>(plan);
+  *rc = SKV_EPLAN;
+  if (h->magic != kPlanMagic || h->version != kPlanVersion) return nullptr;
+  // scalars first: a wrong sample count must not drive the reads of the problem's arrays
+  if (h->B != prob->num_samples || h->Hq != prob->num_q_heads || h->Hkv != prob->num_kv_heads ||
+      h->d != prob->head_dim || h->block_q != prob->block_q || h->chunk_kv != prob->chunk_kv ||
+      h->sub_chunks != prob->sub_chunks || h->P != prob->num_partitions)
+    return nullptr;
+  if (prob->anchor_offsets[prob->num_samples] > 0 && !prob->anchors) return nullptr;
+  if (h->Ltot != prob->ctx_offsets[prob->num_samples] ||
+      h->Nq != static_cast<int64_t>(prob->anchor_offsets[prob->num_samples]) * prob->block_q)
+    return nullptr;
+  if (h->fingerprint != problem_fingerprint(prob)) return nullptr;
+  *rc = SKV_OK;
+  return h;
+}
+
 }  // namespace skv
 
 using namespace skv;
@@ -448,6 +499,7 @@ extern "C" int skv_plan(const skv_problem* prob, int policy, void* plan, size_t 
   if (plan_bytes < h.total_bytes) return SKV_EWORKSPACE;
   uint8_t* base = static_cast<uint8_t*>(plan);
   std::memset(base, 0, h.total_bytes);
+  h.fingerprint = problem_fingerprint(prob);
   std::memcpy(base, &h, sizeof(h));
   copy_to(base, h.items_off, b.items);
   copy_to(base, h.load_off, b.load);

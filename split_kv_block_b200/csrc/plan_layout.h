@@ -10,7 +10,7 @@
 namespace skv {
 
 constexpr uint64_t kPlanMagic = 0x31764b5374696c53ull;  // "SlitSKv1"
-constexpr uint32_t kPlanVersion = 2;
+constexpr uint32_t kPlanVersion = 3;
 constexpr int kTileM = 128;  // query rows per tile (TMEM lanes)
 constexpr int kTileN = 128;  // keys per tile
 
@@ -112,6 +112,16 @@ struct WsLayout {
 };
 
 inline uint64_t align_up(uint64_t x, uint64_t a) { return (x + a - 1) / a * a; }
+
+// 64-bit FNV-1a hash of a problem: its scalars, context offsets, anchor
+// offsets and anchors (plan.cpp). Stored in every plan by skv_plan.
+uint64_t problem_fingerprint(const skv_problem* p);
+
+// The plan's header when `plan` is a plan of this library version written
+// for `prob` (same scalars and the same fingerprint); otherwise nullptr with
+// *rc = SKV_EINVAL (NULL pointers) or SKV_EPLAN. Host only: it reads the
+// problem's arrays and touches no device state (plan.cpp).
+const struct PlanHeader* checked_plan(const void* plan, const skv_problem* prob, int* rc);
 
 inline WsLayout ws_layout(const PlanHeader& h) {
   WsLayout w{};

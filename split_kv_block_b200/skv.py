@@ -24,7 +24,7 @@ SKV_PLAN_STATIC = 1
 EXPORTS = ("skv_plan_size", "skv_plan", "skv_plan_items", "skv_plan_unit_partitions", "skv_plan_stats", "skv_attn_fwd",
            "skv_lse_merge",
            "skv_attn_bwd", "skv_status", "skv_strerror", "skv_last_cuda_error", "skv_set_unit_timer",
-           "skv_set_timing_events", "skv_attn_fwd_noalloc", "skv_wait_selftest")
+           "skv_set_timing_events", "skv_attn_fwd_noalloc", "skv_noalloc_status", "skv_wait_selftest")
 SKV_NOALLOC_SCRATCH_BYTES = 32 << 20
 SKV_KERNEL_FWD, SKV_KERNEL_MERGE, SKV_KERNEL_BWD = 0, 1, 2
 
@@ -62,15 +62,16 @@ def lib() -> ctypes.CDLL:
         L.skv_plan_items.argtypes = [vp, ctypes.POINTER(vp), ctypes.POINTER(sz)]
         L.skv_plan_stats.argtypes = [vp, vp, vp, vp, vp]
         L.skv_plan_unit_partitions.argtypes = [vp, vp, vp]
-        L.skv_attn_fwd.argtypes = [vp, vp, vp, vp, vp, sz, vp]
-        L.skv_lse_merge.argtypes = [vp, vp, vp, vp, vp]
-        L.skv_attn_bwd.argtypes = [vp] * 11 + [sz, vp]
+        L.skv_attn_fwd.argtypes = [vp, vp, vp, vp, vp, vp, sz, vp]
+        L.skv_lse_merge.argtypes = [vp, vp, vp, vp, vp, vp]
+        L.skv_attn_bwd.argtypes = [vp] * 12 + [sz, vp]
         L.skv_status.argtypes = [vp, vp]
         L.skv_strerror.argtypes = [ctypes.c_int]
         L.skv_strerror.restype = ctypes.c_char_p
         L.skv_set_unit_timer.argtypes = [vp, vp]
         L.skv_set_timing_events.argtypes = [ctypes.c_int, vp, vp]
-        L.skv_attn_fwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp]
+        L.skv_attn_fwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp]
+        L.skv_noalloc_status.argtypes = [vp]
         L.skv_wait_selftest.argtypes = [vp, ctypes.c_uint64, ctypes.c_int, vp]
         for name in EXPORTS:
             if name not in ("skv_strerror",):
@@ -145,10 +146,17 @@ class Plan:
         self.sizes = sizes
         self.policy = policy
         self.problem = prob
+        self._pargs = _ProblemArgs(prob)
 
     @property
     def ptr(self):
         return ctypes.c_void_p(self.buf.ctypes.data)
+
+    @property
+    def prob_ref(self):
+        """The skv_problem the plan was made for (passed with the plan to every
+        call that runs kernels; the library checks that they match)."""
+        return self._pargs.ref()
 
     def items(self) -> np.ndarray:
         p, n = ctypes.c_void_p(), ctypes.c_size_t()
@@ -194,18 +202,19 @@ def alloc_workspace(plan: Plan, device="cuda"):
 
 
 def skv_attn_fwd(plan: Plan, q, k, v, ws, stream=None):
-    _check("skv_attn_fwd", lib().skv_attn_fwd(plan.ptr, _ptr(q), _ptr(k), _ptr(v), _ptr(ws), ws.numel(),
-                                              _stream_ptr(stream)))
+    _check("skv_attn_fwd", lib().skv_attn_fwd(plan.ptr, plan.prob_ref, _ptr(q), _ptr(k), _ptr(v), _ptr(ws),
+                                              ws.numel(), _stream_ptr(stream)))
 
 
 def skv_lse_merge(plan: Plan, ws, o, lse, stream=None):
-    _check("skv_lse_merge", lib().skv_lse_merge(plan.ptr, _ptr(ws), _ptr(o), _ptr(lse), _stream_ptr(stream)))
+    _check("skv_lse_merge", lib().skv_lse_merge(plan.ptr, plan.prob_ref, _ptr(ws), _ptr(o), _ptr(lse),
+                                                _stream_ptr(stream)))
 
 
 def skv_attn_bwd(plan: Plan, q, k, v, o, lse, do, dq, dk, dv, ws, stream=None):
-    _check("skv_attn_bwd", lib().skv_attn_bwd(plan.ptr, _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(do),
-                                              _ptr(dq), _ptr(dk), _ptr(dv), _ptr(ws), ws.numel(),
-                                              _stream_ptr(stream)))
+    _check("skv_attn_bwd", lib().skv_attn_bwd(plan.ptr, plan.prob_ref, _ptr(q), _ptr(k), _ptr(v), _ptr(o),
+                                              _ptr(lse), _ptr(do), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(ws),
+                                              ws.numel(), _stream_ptr(stream)))
 
 
 def skv_wait_selftest(ws, limit_ns: int, arrive: bool, stream=None):
@@ -218,8 +227,14 @@ def skv_wait_selftest(ws, limit_ns: int, arrive: bool, stream=None):
 def skv_attn_fwd_noalloc(plan: Plan, q, k, v, o, lse, stream=None):
     """Forward + merge with the library's static scratch: for callers that
     cannot allocate device memory (see include/skv.h)."""
-    _check("skv_attn_fwd_noalloc", lib().skv_attn_fwd_noalloc(plan.ptr, _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse),
-                                                              _stream_ptr(stream)))
+    _check("skv_attn_fwd_noalloc", lib().skv_attn_fwd_noalloc(plan.ptr, plan.prob_ref, _ptr(q), _ptr(k), _ptr(v),
+                                                              _ptr(o), _ptr(lse), _stream_ptr(stream)))
+
+
+def skv_noalloc_status(stream=None) -> int:
+    """Status word of the last skv_attn_fwd_noalloc call on the current device
+    (synchronizes the stream; allocates nothing)."""
+    return lib().skv_noalloc_status(_stream_ptr(stream))
 
 
 def skv_status(ws, stream=None) -> int:

@@ -2,6 +2,8 @@
 items, realized costs, partitions and partition loads must be bit-exact
 ("Split-KV: Breaking the Context Parallelism Bottleneck ...", section "LPT
 Scheduling"). Host-only: runs without a GPU."""
+import ctypes
+
 import numpy as np
 import pytest
 
@@ -184,3 +186,39 @@ def test_plans_do_not_depend_on_earlier_calls():
     for name, p in order:
         for pol in (skv.SKV_PLAN_STATIC, skv.SKV_PLAN_LPT):
             assert skv.skv_plan(p, pol).buf.tobytes() == ref[name][pol], (name, pol)
+
+
+def _fake_dev(n=8):
+    """Non-NULL, 256-byte aligned addresses that no call may dereference: every
+    call below is refused on the host before it enqueues anything."""
+    return [ctypes.c_void_p(0x100000 + 0x1000 * i) for i in range(n)]
+
+
+def test_plan_for_another_problem_is_refused_before_any_launch():
+    """A plan is bound to the problem it was made for (the library stores a
+    hash of the problem in it). Every call that runs kernels takes the
+    problem too and returns SKV_EPLAN, on the host, when they differ: other
+    anchors with the same sizes, more anchors (a larger Nq), a longer context,
+    another head count. With the matching problem the same calls pass the
+    check (here they would then need a GPU, so only refusals run on CPU)."""
+    L = skv.lib()
+    base = synth.small_problem([700, 300], [[5, 600, 41], [300]], block_q=16, chunk_kv=256, hq=8, hkv=2, d=128)
+    plan = skv.skv_plan(base)
+    others = [base.replace(anchors=np.array([5, 601, 41, 300], dtype=np.int64)),
+              synth.small_problem([700, 300], [[5, 600, 41, 7], [300]], block_q=16, chunk_kv=256, hq=8, hkv=2,
+                                  d=128),
+              synth.small_problem([701, 300], [[5, 600, 41], [300]], block_q=16, chunk_kv=256, hq=8, hkv=2, d=128),
+              base.replace(num_q_heads=16),
+              base.replace(num_partitions=5)]
+    f = _fake_dev()
+    for other in others:
+        pr = skv._ProblemArgs(other).ref()
+        assert L.skv_attn_fwd(plan.ptr, pr, f[0], f[1], f[2], f[3], 1 << 30, None) == 5
+        assert L.skv_lse_merge(plan.ptr, pr, f[3], f[4], f[5], None) == 5
+        assert L.skv_attn_bwd(plan.ptr, pr, *f[:7], f[7], f[0], f[1], 1 << 30, None) == 5
+        assert L.skv_attn_fwd_noalloc(plan.ptr, pr, f[0], f[1], f[2], f[3], f[4], None) == 5
+    # NULL problem: invalid argument; a buffer that is not a plan: SKV_EPLAN
+    assert L.skv_attn_fwd(plan.ptr, None, f[0], f[1], f[2], f[3], 1 << 30, None) == 1
+    junk = np.zeros(plan.buf.nbytes, dtype=np.uint8)
+    assert L.skv_attn_fwd(ctypes.c_void_p(junk.ctypes.data), plan.prob_ref, f[0], f[1], f[2], f[3], 1 << 30,
+                          None) == 5
