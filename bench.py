@@ -47,6 +47,16 @@ METRIC = "split-KV attn fwd+bwd effective TFLOP/s"
 L2_BYTES = 126 * 1000 * 1000
 
 
+def check_world(gpus, world):
+    """--gpus N must match the number of ranks: N > 1 runs one process per GPU
+    under torchrun (WORLD_SIZE = N), N = 1 a single process."""
+    if gpus < 1:
+        raise SystemExit(f"--gpus {gpus}: need at least one GPU")
+    if gpus != world:
+        raise SystemExit(f"--gpus {gpus} but WORLD_SIZE={world}: launch N > 1 with "
+                         "torch.distributed.run --nproc-per-node N (one rank per GPU)")
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -107,9 +117,10 @@ def bwd_bytes(prob):
     return 2 * Nq * Hq * d * 2 + 2 * Nq * Hq * 4 + 4 * keys * Hkv * d * 2 + 2 * Nq * Hq * d * 4
 
 
-KERNEL_SOURCES = {"fwd_kernel": ["fwd.cu", "fwd2.cu", "sm100.cuh", "kernels.h", "plan_layout.h"],
+KERNEL_SOURCES = {"fwd_kernel": ["fwd.cu", "fwd2.cu", "sm100.cuh", "kernels.h", "plan_layout.h", "merge_row.cuh",
+                                  "tail_merge.cuh"],
                   "bwd_kernel": ["bwd.cu", "bwd2.cu", "sm100.cuh", "kernels.h", "plan_layout.h"],
-                  "merge_kernel": ["merge.cu", "sm100.cuh", "kernels.h", "plan_layout.h"]}
+                  "merge_kernel": ["merge.cu", "sm100.cuh", "kernels.h", "plan_layout.h", "merge_row.cuh"]}
 
 
 def kernel_digest(kernel):
@@ -186,23 +197,39 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------- GPU arm
-def run_gpu(args, rank, world, local_rank):
+EXTRA_WORKLOADS = ("ctx128k", "batch8_logu")  # measured beside the headline workload on one GPU
+
+
+def merge_bytes(prob, n_fwd_units):
+    """Algorithmic bytes of the LSE merge kernel: every partial read once (fp32
+    output row and LSE per query-tile row), merged O (bf16) and LSE (fp32)
+    written once."""
+    rows = prob.num_tokens_q * prob.num_q_heads
+    return n_fwd_units * 128 * (prob.head_dim + 1) * 4 + rows * prob.head_dim * 2 + rows * 4
+
+
+def run_workload(args, name, steps, warmup, rank, world, local_rank, e2e):
+    """Time `steps` whole steps of workload `name` (after `warmup` untimed ones)
+    on this rank's GPU and return its record."""
     from split_kv_block_b200 import skv
 
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
-    w = synth.WORKLOADS[args.workload]
-    seed, prob = rank_problem(args, rank)
+    w = synth.WORKLOADS[name]
+    seed = args.seed + rank
+    prob = synth.make_problem(w, seed=seed, sub_chunks=args.sub_chunks if name == args.workload else None)
     backward = w.backward
     q, k, v, do = synth.make_tensors(prob, seed=seed, backward=backward)
     q, k, v = q.to(dev), k.to(dev), v.to(dev)
     do = do.to(dev) if backward else None
     policy = skv.SKV_PLAN_STATIC if args.policy == "static" else skv.SKV_PLAN_LPT
-    redraw = args.workload == "batch8_logu"
+    if args.partials == "bf16":
+        policy |= skv.SKV_PLAN_PARTIALS_BF16
+    redraw = name == "batch8_logu"
+    fused = args.fused_merge  # the merge in the forward kernel's tail, or its own launch (default: faster here)
 
     # anchors of every step (the batched workload redraws them each step)
-    step_probs = [synth.redraw_anchors(prob, w, seed * 1000 + i) if redraw else prob
-                  for i in range(args.warmup + args.steps)]
+    step_probs = [synth.redraw_anchors(prob, w, seed * 1000 + i) if redraw else prob for i in range(warmup + steps)]
     sizes = [skv.skv_plan_size(p, policy) for p in step_probs]
     ws_bytes = max(s.ws_bytes for s in sizes)
     plan_bytes = max(s.plan_bytes for s in sizes)
@@ -216,6 +243,11 @@ def run_gpu(args, rank, world, local_rank):
         dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
     flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)  # > 126 MB L2
     stream = torch.cuda.current_stream()
+    # Every forward and backward call clears the workspace's status word before it runs, so the word is
+    # copied (4 bytes, device to device, on the launch stream) after the merge and after the backward of
+    # every step, warm-up and timed; a wait that gave up in any call is then seen after the loop.
+    ws_status = ws[:4].view(torch.int32)
+    status_log = torch.zeros(2 * (warmup + steps), dtype=torch.int32, device=dev)
 
     planner_s = []
 
@@ -224,10 +256,15 @@ def run_gpu(args, rank, world, local_rank):
         t0 = time.perf_counter()
         plan = skv.skv_plan(p, policy, sizes=sizes[i], buf=plan_buf)
         planner_s.append(time.perf_counter() - t0)
-        skv.skv_attn_fwd(plan, q, k, v, ws, stream)
-        skv.skv_lse_merge(plan, ws, o, lse, stream)
+        if fused:
+            skv.skv_attn_fwd_merged(plan, q, k, v, o, lse, ws, stream)
+        else:
+            skv.skv_attn_fwd(plan, q, k, v, ws, stream)
+            skv.skv_lse_merge(plan, ws, o, lse, stream)
+        status_log[2 * i:2 * i + 1].copy_(ws_status)
         if backward:
             skv.skv_attn_bwd(plan, q, k, v, o, lse, do, dq, dk, dv, ws, stream)
+            status_log[2 * i + 1:2 * i + 2].copy_(ws_status)
         return plan
 
     def mk_event():
@@ -235,16 +272,16 @@ def run_gpu(args, rank, world, local_rank):
         e.record(stream)
         return e
 
-    for i in range(args.warmup):
+    for i in range(warmup):
         step(i)
     torch.cuda.synchronize()
-    assert skv.skv_status(ws) == 0, "device status error during warm-up"
     planner_s.clear()
 
-    K = args.steps
+    K = steps
     ev = [(mk_event(), mk_event()) for _ in range(K)]
-    kev = {kid: [(mk_event(), mk_event()) for _ in range(K)] for kid in (skv.SKV_KERNEL_FWD, skv.SKV_KERNEL_MERGE,
-                                                                          skv.SKV_KERNEL_BWD)}
+    kids = ((skv.SKV_KERNEL_FWD,) + (() if fused else (skv.SKV_KERNEL_MERGE,)) +
+            ((skv.SKV_KERNEL_BWD,) if backward else ()))
+    kev = {kid: [(mk_event(), mk_event()) for _ in range(K)] for kid in kids}
     torch.cuda.synchronize()
     if world > 1:
         torch.distributed.barrier()
@@ -261,7 +298,7 @@ def run_gpu(args, rank, world, local_rank):
             for i in range(K):
                 for kid, lst in kev.items():
                     skv.skv_set_timing_events(kid, lst[i][0], lst[i][1])
-                step(args.warmup + i)
+                step(warmup + i)
             ev[0][1].record(stream)
         else:
             for i in range(K):
@@ -269,7 +306,7 @@ def run_gpu(args, rank, world, local_rank):
                 for kid, lst in kev.items():
                     skv.skv_set_timing_events(kid, lst[i][0], lst[i][1])
                 ev[i][0].record(stream)
-                step(args.warmup + i)
+                step(warmup + i)
                 ev[i][1].record(stream)
         torch.cuda.synchronize()
     for kid in kev:
@@ -277,70 +314,112 @@ def run_gpu(args, rank, world, local_rank):
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
-    status = skv.skv_status(ws)
-    if status != 0:
-        raise RuntimeError(f"device status {status} after the timed steps")
+    bad = status_log.nonzero().flatten().tolist()
+    if bad:
+        codes = sorted(set(status_log.cpu().tolist()) - {0})
+        raise RuntimeError(f"{name}: device status {codes} in step calls {bad} (warm-up and timed)")
     t_steps = [ev[0][0].elapsed_time(ev[0][1]) / 1e3] if stream_mode else [a.elapsed_time(b) / 1e3 for a, b in ev]
     t_kern = {kid: [a.elapsed_time(b) / 1e3 for a, b in lst] for kid, lst in kev.items()}
     total = max_over_ranks(sum(t_steps), world, dev)
 
-    f_fwd_all, f_bwd_all = 0.0, 0.0
+    f_fwd_all, f_bwd_all, mbytes_all = 0.0, 0.0, 0.0
     for i in range(K):
-        a, b = flops_of(step_probs[args.warmup + i], backward)
+        p = step_probs[warmup + i]
+        a, b = flops_of(p, backward)
         f_fwd_all += a
         f_bwd_all += b
+        if not fused:
+            mbytes_all += merge_bytes(p, skv.skv_plan(p, policy, sizes=sizes[warmup + i]).stats()["n_fwd_units"])
     flops_rank = f_fwd_all + f_bwd_all
     value = job_value(sum_over_ranks(flops_rank, world, dev), total)
     ctx_tokens = sum_over_ranks(float(prob.num_tokens_kv) * K, world, dev)
 
     # plan quality (LPT vs static) on this step's problem
-    p0 = step_probs[args.warmup]
+    p0 = step_probs[warmup]
     lpt = skv.skv_plan(p0, skv.SKV_PLAN_LPT).stats()["imbalance"]
     static = skv.skv_plan(p0, skv.SKV_PLAN_STATIC).stats()["imbalance"]
 
-    realized = realized_busy_imbalance(skv, p0, policy, q, k, v, do, ws, o, lse, dq, dk, dv, stream, dev)
+    realized = realized_busy_imbalance(skv, p0, policy, q, k, v, do, ws, o, lse, dq, dk, dv, stream, dev, fused)
 
     peaks = load_peaks()
-    dom = skv.SKV_KERNEL_BWD if backward else skv.SKV_KERNEL_FWD
-    dom_t = statistics.mean(t_kern[dom])
-    dom_flops = (f_bwd_all if backward else f_fwd_all) / K
-    achieved = dom_flops / dom_t / 1e12
-    roof_step = max(flops_rank / K / (peaks["bf16_tflops"] * 1e12), 0.0)
-    kernels_per_step = 2 + (3 if backward else 0)
+    kms = {kid: statistics.mean(t) for kid, t in t_kern.items()}
 
-    out = {
-        "metric": METRIC, "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world, "steps": K,
-        "warmup": args.warmup, "ms_per_step": round(total / K * 1e3, 4), "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": f"{args.workload}: {WORKLOAD_TEXT[args.workload]}", "seed": args.seed,
-                   "policy": args.policy, "sub_chunks": prob.sub_chunks,
-                   "l2": (f"inputs larger than L2 (K+V {kv_bytes / 2**20:.0f} MiB > 126 MB): no flush, {K} steps back "
-                          "to back between two events, host planning of the next step overlapping the GPU")
-                         if stream_mode else "flushed before every step (256 MiB write outside the step's event window)",
-                   "parallelism": f"replicas x{world}" if world > 1 else "1 GPU, P virtual partitions"},
-        "roofline": {"bound": "tensor", "kernel": "bwd_kernel" if backward else "fwd_kernel",
-                     "achieved": round(achieved, 2), "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                     "frac": round(achieved / peaks["bf16_tflops"], 4),
-                     "frac_of_sustained": (round(achieved / peaks["bf16_tflops_sustained"], 4)
-                                           if peaks.get("bf16_tflops_sustained") else None),
-                     "traffic": profiled_traffic("bwd_kernel" if backward else "fwd_kernel", args.workload),
-                     "peak_source": f"{peaks['source']} bf16 dense (burst)",
-                     "step_frac": round(roof_step / (total / K), 4)},
-        "kernel_ms": {"fwd": round(statistics.mean(t_kern[skv.SKV_KERNEL_FWD]) * 1e3, 4),
-                      "merge": round(statistics.mean(t_kern[skv.SKV_KERNEL_MERGE]) * 1e3, 4),
-                      "bwd": round(statistics.mean(t_kern[skv.SKV_KERNEL_BWD]) * 1e3, 4) if backward else None},
+    def tensor_roof(kernel, flops_per_launch, t):
+        a = flops_per_launch / t / 1e12
+        return {"bound": "tensor", "kernel": kernel, "achieved": round(a, 2), "peak": peaks["bf16_tflops"],
+                "unit": "TFLOP/s", "frac": round(a / peaks["bf16_tflops"], 4),
+                "frac_of_sustained": (round(a / peaks["bf16_tflops_sustained"], 4)
+                                      if peaks.get("bf16_tflops_sustained") else None),
+                "traffic": profiled_traffic(kernel, name),
+                "peak_source": f"{peaks['source']} bf16 dense (burst)"}
+
+    kernels = {"fwd": tensor_roof("fwd_kernel", f_fwd_all / K, kms[skv.SKV_KERNEL_FWD])}
+    if fused:
+        kernels["fwd"]["note"] = "forward with the LSE merge in its tail (one launch)"
+    else:
+        m_gbs = mbytes_all / K / kms[skv.SKV_KERNEL_MERGE] / 1e9
+        kernels["merge"] = {"bound": "hbm", "kernel": "merge_kernel", "achieved": round(m_gbs, 1),
+                            "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(m_gbs / peaks["hbm_gbs"], 4),
+                            "traffic": profiled_traffic("merge_kernel", name),
+                            "peak_source": f"{peaks['source']} HBM copy"}
+    if backward:
+        kernels["bwd"] = tensor_roof("bwd_kernel", f_bwd_all / K, kms[skv.SKV_KERNEL_BWD])
+    roofline = dict(kernels["bwd" if backward else "fwd"])
+    roofline["step_frac"] = round(flops_rank / K / (peaks["bf16_tflops"] * 1e12) / (total / K), 4)
+    kernels_per_step = (1 if fused else 2) + (3 if backward else 0)
+
+    rec = {
+        "workload": f"{name}: {WORKLOAD_TEXT[name]}", "value": round(value, 3), "unit": "TFLOP/s", "steps": K,
+        "warmup": warmup, "ms_per_step": round(total / K * 1e3, 4), "seed": args.seed, "policy": args.policy,
+        "sub_chunks": prob.sub_chunks, "partials": args.partials,
+        "l2": (f"inputs larger than L2 (K+V {kv_bytes / 2**20:.0f} MiB > 126 MB): no flush, {K} steps back "
+               "to back between two events, host planning of the next step overlapping the GPU")
+              if stream_mode else "flushed before every step (256 MiB write outside the step's event window)",
+        "roofline": roofline, "kernels": kernels,
+        "kernel_ms": {"fwd": round(kms[skv.SKV_KERNEL_FWD] * 1e3, 4),
+                      "merge": None if fused else round(kms[skv.SKV_KERNEL_MERGE] * 1e3, 4),
+                      "bwd": round(kms[skv.SKV_KERNEL_BWD] * 1e3, 4) if backward else None},
+        "merge": "in the forward kernel's tail" if fused else "separate launch",
         "context_tokens_per_s": round(ctx_tokens / total, 1),
         "imbalance": {"lpt": lpt, "static": static, "realized": realized},
         "planner_us": round(statistics.median(planner_s) * 1e6, 1),
         "gpu_launches": kernels_per_step * K,
         "clocks": clocks.summary(),
     }
-    if not args.no_e2e:
-        out["e2e"] = run_e2e(args, prob, step_probs, sizes, policy, q, k, v, do, dev, world)
+    if e2e:
+        rec["e2e"] = run_e2e(args, prob, step_probs, sizes, policy, q, k, v, do, dev, world)
+    del ws, flush, q, k, v, do, o, lse, dq, dk, dv
+    torch.cuda.empty_cache()
+    return rec, prob
+
+
+def run_gpu(args, rank, world, local_rank):
+    rec, prob = run_workload(args, args.workload, args.steps, args.warmup, rank, world, local_rank, not args.no_e2e)
+    out = {
+        "metric": METRIC, "value": rec["value"], "unit": "TFLOP/s", "n_gpus": world, "steps": rec["steps"],
+        "warmup": rec["warmup"], "ms_per_step": rec["ms_per_step"], "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": rec["workload"], "seed": args.seed, "policy": args.policy,
+                   "sub_chunks": rec["sub_chunks"], "partials": rec["partials"], "l2": rec["l2"],
+                   "parallelism": f"replicas x{world}" if world > 1 else "1 GPU, P virtual partitions"},
+    }
+    for key in ("roofline", "kernels", "kernel_ms", "merge", "context_tokens_per_s", "imbalance", "planner_us",
+                "gpu_launches", "clocks", "e2e"):
+        if key in rec:
+            out[key] = rec[key]
+    if world == 1 and not args.no_extra:
+        # the other target workloads, each timed on its own (same contract: warm-up, then steps timed with
+        # CUDA events, clocks sampled during its timed region)
+        out["workloads"] = {}
+        for name in EXTRA_WORKLOADS:
+            if name == args.workload:
+                continue
+            r, _ = run_workload(args, name, min(args.steps, 20), args.warmup, rank, world, local_rank, False)
+            out["workloads"][name] = r
     return out, prob
 
 
-def realized_busy_imbalance(skv, prob, policy, q, k, v, do, ws, o, lse, dq, dk, dv, stream, dev):
+def realized_busy_imbalance(skv, prob, policy, q, k, v, do, ws, o, lse, dq, dk, dv, stream, dev, fused=True):
     """One more (untimed) step with the unit timer on: every work unit's
     %globaltimer start and end, summed per virtual partition, gives the realized
     busy time of each partition; its imbalance (max / mean - 1, mean over all P)
@@ -353,8 +432,11 @@ def realized_busy_imbalance(skv, prob, policy, q, k, v, do, ws, o, lse, dq, dk, 
     bst = torch.zeros(2 * max(n_b, 1), dtype=torch.int64, device=dev)
     skv.skv_set_unit_timer(fst, bst if backward else None)
     try:
-        skv.skv_attn_fwd(plan, q, k, v, ws, stream)
-        skv.skv_lse_merge(plan, ws, o, lse, stream)
+        if fused:
+            skv.skv_attn_fwd_merged(plan, q, k, v, o, lse, ws, stream)
+        else:
+            skv.skv_attn_fwd(plan, q, k, v, ws, stream)
+            skv.skv_lse_merge(plan, ws, o, lse, stream)
         if backward:
             skv.skv_attn_bwd(plan, q, k, v, o, lse, do, dq, dk, dv, ws, stream)
         torch.cuda.synchronize()
@@ -420,8 +502,11 @@ def run_e2e(args, prob, step_probs, sizes, policy, q, k, v, do, dev, world):
         p = step_probs[i % len(step_probs)]
         plan = skv.skv_plan(p, policy, sizes=sizes[i % len(sizes)])
         x, y = din[b], dout[b]
-        skv.skv_attn_fwd(plan, x["q"], x["k"], x["v"], ws, stream)
-        skv.skv_lse_merge(plan, ws, y["o"], y["lse"], stream)
+        if args.fused_merge:
+            skv.skv_attn_fwd_merged(plan, x["q"], x["k"], x["v"], y["o"], y["lse"], ws, stream)
+        else:
+            skv.skv_attn_fwd(plan, x["q"], x["k"], x["v"], ws, stream)
+            skv.skv_lse_merge(plan, ws, y["o"], y["lse"], stream)
         if backward:
             skv.skv_attn_bwd(plan, x["q"], x["k"], x["v"], y["o"], y["lse"], x["do"], y["dq"], y["dk"], y["dv"],
                              ws, stream)
@@ -583,7 +668,7 @@ def run_reference(args):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(total / args.steps * 1e3, 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": f"{args.workload}: {WORKLOAD_TEXT[args.workload]}", "seed": args.seed,
-                   "parallelism": "CPU host cores"},
+                   "policy": args.policy, "sub_chunks": prob.sub_chunks, "parallelism": "CPU host cores"},
         "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": torch.get_num_threads(),
                          "kind": "oracle", "sample": sample, "cpu": _cpu_name()},
         "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -604,12 +689,19 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extra", action="store_true", help="time the headline workload only")
+    ap.add_argument("--partials", default="fp32", choices=["fp32", "bf16"],
+                    help="storage of the per-chunk partial outputs between the forward and the merge")
+    ap.add_argument("--fused-merge", action="store_true",
+                    help="run the LSE merge in the forward kernel's tail (skv_attn_fwd_merged) instead of as its own "
+                         "launch")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    check_world(args.gpus, world)
 
     if args.impl == "reference":
         if rank == 0:

@@ -64,7 +64,15 @@ enum skv_status_code {
 
 enum skv_plan_policy {
   SKV_PLAN_LPT = 0,    /* cost-aware LPT over (b, c, g, s) items ("LPT Scheduling") */
-  SKV_PLAN_STATIC = 1  /* equal-token contiguous split, the baseline LPT replaces */
+  SKV_PLAN_STATIC = 1, /* equal-token contiguous split, the baseline LPT replaces */
+  /* Flag, OR-ed into either policy: the forward stores each chunk's partial
+   * output in bf16 instead of fp32 (the partial LSE stays fp32), halving the
+   * partials' memory traffic and workspace. A partial output is a convex
+   * combination of bf16 value rows, so rounding it adds at most 2^-9 times
+   * the largest |V| to the merged output (about 1.1e-2 for N(0,1) values)
+   * and nothing to the LSE. skv_plan_size, the forward and the merge read
+   * the format from the plan. */
+  SKV_PLAN_PARTIALS_BF16 = 0x100
 };
 
 /* One split-KV problem. Host pointers; read during the call only. */
@@ -89,6 +97,9 @@ typedef struct {
   int64_t cost;                /* unmasked (query, key) pairs x q-heads of the group */
   int32_t partition;           /* partition the planner placed the item on */
   int32_t order;               /* position in the placement order (LPT: longest first) */
+  int64_t kv_row;              /* row of key_begin in the K/V buffers the kernels read: key_begin for a
+                                  full plan; for a shard plan the item's first row in the shard buffer
+                                  (one kv head per row), or -1 for items of other partitions */
 } skv_item;
 
 /*
@@ -110,6 +121,43 @@ int skv_plan_size(const skv_problem* prob, int policy, size_t* n_items, size_t* 
  * skv_plan_size); `partition_load` (may be NULL) receives [P] int64 loads.
  */
 int skv_plan(const skv_problem* prob, int policy, void* plan, size_t plan_bytes, int64_t* partition_load);
+
+/*
+ * Context parallelism across GPUs ("Split-KV: Breaking the Context
+ * Parallelism Bottleneck in Diffusion Drafter Training", section "Split-KV's
+ * Core Mechanism: Decoupling Communication from Context Length"; "Split-KV:
+ * Efficient Context Parallelism for Training Diffusion Drafters", Abstract):
+ * the P partitions of an LPT plan are the ranks. Each rank keeps the key/
+ * value rows of its own items, sees the whole (small) query set, computes its
+ * partial output and LSE over its items and its share of dQ, and only
+ * query-sized tensors cross ranks: the (O_r, LSE_r) pairs, combined exactly
+ * by skv_lse_combine, and the dQ shares, summed by skv_dq_combine. dK and dV
+ * stay on the rank that owns the keys.
+ *
+ * skv_plan_shard_size / skv_plan_shard — the plan of rank `partition` (0 <=
+ * partition < P): the global plan's items and placement, with only that
+ * partition's items turned into work units, all on one work queue. The
+ * rank's K/V (and dK/dV) buffers hold the rows of its items, one kv head per
+ * row, items in (b, c, g, s) order: item i occupies rows [kv_row, kv_row +
+ * key_end - key_begin) of a bf16 [kv_rows][1][d] buffer (skv_plan_items gives
+ * kv_row; skv_plan_kv_layout gives kv_rows). Queries, outputs, LSE and dO
+ * keep the full problem's layout. Every call below accepts such a plan with
+ * the full problem; skv_attn_fwd + skv_lse_merge then give the rank's
+ * (O_r, LSE_r) (rows without keys on the rank: O_r = 0, LSE_r = -inf), and
+ * skv_attn_bwd_partial its dQ share and its items' dK/dV. Same arguments and
+ * errors as skv_plan_size / skv_plan, plus SKV_EINVAL for a partition out of
+ * range.
+ */
+int skv_plan_shard_size(const skv_problem* prob, int policy, int partition, size_t* n_items, size_t* plan_bytes,
+                        size_t* ws_fwd_bytes, size_t* ws_bwd_bytes);
+int skv_plan_shard(const skv_problem* prob, int policy, int partition, void* plan, size_t plan_bytes,
+                   int64_t* partition_load);
+
+/* Layout of the K/V (and dK/dV) buffers a plan's kernels read: kv_rows rows
+ * of kv_heads heads of head_dim bf16 each (Ltot and Hkv for a full plan;
+ * the shard's key count and 1 for a shard plan), and the plan's shard (-1
+ * for a full plan). Any pointer may be NULL. */
+int skv_plan_kv_layout(const void* plan, int64_t* kv_rows, int32_t* kv_heads, int32_t* shard);
 
 /* Items of a plan in (b, c, g, sub) order; *items points into `plan`. */
 int skv_plan_items(const void* plan, const skv_item** items, size_t* n_items);
@@ -173,6 +221,24 @@ int skv_lse_merge(const void* plan, const skv_problem* prob, const void* ws, voi
                   skv_stream_t stream);
 
 /*
+ * skv_attn_fwd_merged — skv_attn_fwd and skv_lse_merge in one kernel launch
+ * (same passages as those two calls). Every forward work unit writes its
+ * partial into `ws` as skv_attn_fwd does; as soon as all units of a (query
+ * tile, kv head) have written theirs, a CTA of the same launch that has no
+ * forward work left merges that tile's rows into o and lse, with the
+ * arithmetic and ascending key order of skv_lse_merge. So the merge runs in
+ * the forward's scheduling tail, while the partials are recent in L2, and o
+ * and lse are bitwise equal to those of skv_attn_fwd + skv_lse_merge (the
+ * partials stay in `ws` as well). Outputs: o (device bf16 [Nq][Hq][d]), lse
+ * (device fp32 [Nq][Hq]). The workspace is the forward's (ws_fwd_bytes).
+ * Waits across CTAs are bounded like every other wait: a tile whose partials
+ * do not all arrive within the limit records SKV_ETIMEOUT in the status word.
+ * Enqueued on `stream`.
+ */
+int skv_attn_fwd_merged(const void* plan, const skv_problem* prob, const void* q, const void* k, const void* v,
+                        void* o, float* lse, void* ws, size_t ws_bytes, skv_stream_t stream);
+
+/*
  * skv_attn_bwd — gradients of the attention through the split. Source:
  * "Split-KV: Breaking the Context Parallelism Bottleneck in Diffusion Drafter
  * Training", section "Split-KV's Core Mechanism" (the split is exact, which
@@ -189,6 +255,60 @@ int skv_lse_merge(const void* plan, const skv_problem* prob, const void* ws, voi
 int skv_attn_bwd(const void* plan, const skv_problem* prob, const void* q, const void* k, const void* v,
                  const void* o, const float* lse, const void* dout, void* dq, void* dk, void* dv, void* ws,
                  size_t ws_bytes, skv_stream_t stream);
+
+/*
+ * skv_attn_bwd_deterministic — skv_attn_bwd with dQ summed over the key
+ * tiles in one fixed order, so that two runs of the same problem give the
+ * same dQ bits (dK and dV are bitwise reproducible in both calls: every key's
+ * gradient is written by the one unit that owns it). Reading of the pages:
+ * dQ = sum over KV chunks of the chunks' dQ contributions ("Split-KV:
+ * Breaking the Context Parallelism Bottleneck in Diffusion Drafter Training",
+ * section "Split-KV's Core Mechanism"), taken here in ascending key order, in
+ * fp32. skv_attn_bwd adds the contributions with fp32 atomics in whatever
+ * order the work units finish, which is faster but reproducible only to
+ * rounding. Here the units are taken from one queue in (sample, key tile,
+ * kv head) order, and each warp adds its rows of a query tile's dQ once every
+ * unit with a lower key tile of the same sample and kv head has added its
+ * own (a turn counter per query tile, kv head and warp, waited on with the
+ * bounded wait of every kernel). Same arguments, layouts and workspace size
+ * as skv_attn_bwd.
+ */
+int skv_attn_bwd_deterministic(const void* plan, const skv_problem* prob, const void* q, const void* k,
+                               const void* v, const void* o, const float* lse, const void* dout, void* dq,
+                               void* dk, void* dv, void* ws, size_t ws_bytes, skv_stream_t stream);
+
+/*
+ * skv_attn_bwd_partial — skv_attn_bwd with dQ written in fp32 (device
+ * [Nq][Hq][d], scaled): the plan's share of dQ, to be summed over ranks with
+ * skv_dq_combine. For a shard plan it is the rank's share (its keys' part of
+ * every query's gradient); dk and dv are the shard's rows (kv_rows x 1 x d).
+ * Same arguments, layouts and workspace as skv_attn_bwd otherwise.
+ */
+int skv_attn_bwd_partial(const void* plan, const skv_problem* prob, const void* q, const void* k, const void* v,
+                         const void* o, const float* lse, const void* dout, float* dq, void* dk, void* dv, void* ws,
+                         size_t ws_bytes, skv_stream_t stream);
+
+/*
+ * skv_lse_combine — exact combine of the ranks' partial outputs (the
+ * query-sized aggregation of "Split-KV's Core Mechanism"): per row i of
+ * n_rows = Nq * Hq, over ranks r = 0 .. n_parts-1 in order,
+ *   m = max_r LSE_r, LSE = m + ln sum_r exp(LSE_r - m),
+ *   O = sum_r exp(LSE_r - LSE) O_r; ranks with LSE_r = -inf weigh nothing.
+ * o_parts: device bf16 [n_parts][n_rows][head_dim] (the all-gathered rank
+ * outputs of skv_lse_merge), lse_parts: device fp32 [n_parts][n_rows];
+ * writes o (bf16 [n_rows][head_dim]) and lse (fp32 [n_rows]). head_dim 64 or
+ * 128; SKV_EINVAL otherwise or for misaligned pointers. Enqueued on `stream`.
+ */
+int skv_lse_combine(const void* o_parts, const float* lse_parts, int n_parts, int64_t n_rows, int head_dim,
+                    void* o, float* lse, skv_stream_t stream);
+
+/*
+ * skv_dq_combine — dQ = sum over ranks of their fp32 shares (from
+ * skv_attn_bwd_partial), ranks in order r = 0 .. n_parts-1, rounded once to
+ * bf16. dq_parts: device fp32 [n_parts][n]; dq: device bf16 [n]; n a
+ * multiple of 4 (Nq * Hq * head_dim). Enqueued on `stream`.
+ */
+int skv_dq_combine(const float* dq_parts, int n_parts, int64_t n, void* dq, skv_stream_t stream);
 
 /*
  * skv_status — synchronizes `stream`, reads the status word in `ws` and
@@ -214,8 +334,8 @@ enum skv_kernel_id { SKV_KERNEL_FWD = 0, SKV_KERNEL_MERGE = 1, SKV_KERNEL_BWD = 
 /* Kernel timing: while set, the library records the caller-created CUDA
  * events `start` / `end` (cudaEvent_t) on the launch stream immediately
  * before and after every launch of the given kernel (the forward attention
- * kernel, the LSE merge kernel, or the backward attention kernel). NULL
- * disables. Process-wide setting. */
+ * kernel, with its merge for skv_attn_fwd_merged; the LSE merge kernel; or
+ * the backward attention kernel). NULL disables. Process-wide setting. */
 int skv_set_timing_events(int kernel, void* start_event, void* end_event);
 
 /* Size of the library-owned scratch array used by skv_attn_fwd_noalloc. */

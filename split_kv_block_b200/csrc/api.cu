@@ -25,6 +25,7 @@ cudaError_t mark(int kernel, int which, cudaStream_t stream) {
   return g_ev[kernel][which] ? cudaEventRecord(g_ev[kernel][which], stream) : cudaSuccess;
 }
 constexpr unsigned long long kTimeoutNs = 2000000000ull;  // 2 s per device-side wait
+constexpr uint64_t kPartialsL2Bytes = 64ull << 20;          // half of the 126 MB L2
 
 int cuda_fail(cudaError_t e) {
   g_last_cuda = static_cast<int>(e);
@@ -133,12 +134,15 @@ const T* at(const void* base, uint64_t off) {
 
 bool aligned16(const void* p) { return reinterpret_cast<uintptr_t>(p) % 16 == 0; }
 
-// Device plan copy + zeroed control block and queue counters.
-int prepare_ws(const PlanHeader& h, const void* plan, void* ws, const WsLayout& w, cudaStream_t stream) {
-  // status word and queue counters: one contiguous control block
+// Device plan copy + zeroed control block and queue counters. `full` also
+// uploads the arrays only the deterministic backward reads.
+int prepare_ws(const PlanHeader& h, const void* plan, void* ws, const WsLayout& w, cudaStream_t stream,
+               bool full = false) {
+  // status word, queue counters and merge counters: one contiguous control block
   cudaError_t e = cudaMemsetAsync(at<uint8_t>(ws, w.status), 0, w.control, stream);
   if (e != cudaSuccess) return cuda_fail(e);
-  if (h.dev.bytes > 0) return upload(static_cast<const uint8_t*>(plan) + h.dev_off, h.dev.bytes, at<uint8_t>(ws, w.dev), stream);
+  const uint64_t n = full ? h.dev.bytes : h.dev.base_bytes;
+  if (n > 0) return upload(static_cast<const uint8_t*>(plan) + h.dev_off, n, at<uint8_t>(ws, w.dev), stream);
   return SKV_OK;
 }
 
@@ -185,24 +189,26 @@ extern "C" int skv_set_timing_events(int kernel, void* start_event, void* end_ev
   return SKV_OK;
 }
 
-extern "C" int skv_attn_fwd(const void* plan, const skv_problem* prob, const void* q, const void* k,
-                            const void* v, void* ws, size_t ws_bytes, skv_stream_t stream_) {
-  int rc = SKV_OK;
-  const PlanHeader* h = checked_plan(plan, prob, &rc);
-  if (!h) return rc;
-  if (!q || !k || !v || !ws) return SKV_EINVAL;
+namespace {
+
+// Forward launch shared by skv_attn_fwd (partials only, o == nullptr) and
+// skv_attn_fwd_merged (partials merged into o / lse in the same launch).
+int run_fwd(const PlanHeader* h, const void* plan, const void* q, const void* k, const void* v, void* ws,
+            size_t ws_bytes, void* o, float* lse, cudaStream_t stream) {
+  // a shard plan may own no key rows at all (more ranks than items): its K/V buffers may then be empty
+  if (!q || !ws || (h->kv_rows > 0 && (!k || !v))) return SKV_EINVAL;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || reinterpret_cast<uintptr_t>(ws) % 256 != 0)
     return SKV_EINVAL;
+  if (o && (!lse || !aligned16(o) || !aligned16(lse))) return SKV_EINVAL;
   const WsLayout w = ws_layout(*h);
   if (ws_bytes < w.fwd_end) return SKV_EWORKSPACE;
-  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
-  rc = prepare_ws(*h, plan, ws, w, stream);
+  int rc = prepare_ws(*h, plan, ws, w, stream);
   if (rc != SKV_OK) return rc;
   if (h->n_fwd == 0) return SKV_OK;
   CUtensorMap tq, tk, tv;
   if ((rc = make_map(&tq, q, h->Nq, h->Hq, h->d, h->G, h->tile_tokens)) != SKV_OK) return rc;
-  if ((rc = make_map(&tk, k, h->Ltot, h->Hkv, h->d, 1, kTileN)) != SKV_OK) return rc;
-  if ((rc = make_map(&tv, v, h->Ltot, h->Hkv, h->d, 1, kTileN)) != SKV_OK) return rc;
+  if ((rc = make_map(&tk, k, h->kv_rows, h->kv_heads, h->d, 1, kTileN)) != SKV_OK) return rc;
+  if ((rc = make_map(&tv, v, h->kv_rows, h->kv_heads, h->d, 1, kTileN)) != SKV_OK) return rc;
   const uint8_t* dev = at<uint8_t>(ws, w.dev);
   FwdParams p{};
   p.mtiles = at<MTile>(dev, h->dev.mtiles);
@@ -215,11 +221,26 @@ extern "C" int skv_attn_fwd(const void* plan, const skv_problem* prob, const voi
   p.status = at<int>(ws, w.status);
   p.part_o = at<float>(ws, w.fwd_o);
   p.part_lse = at<float>(ws, w.fwd_lse);
+  p.partial_bf16 = (h->policy & SKV_PLAN_PARTIALS_BF16) ? 1 : 0;
   p.stamps = g_fwd_stamps;
   p.timeout_ns = kTimeoutNs;
-  p.P = h->P;
+  p.P = h->n_queues;
   p.G = h->G;
   p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(h->d)));
+  // partials that fit in half of L2 are kept there (evict_last) until the merge reads them
+  p.partials_l2_last = (w.fwd_end - w.fwd_o) <= kPartialsL2Bytes ? 1 : 0;
+  if (o) {
+    p.merge_off = at<int32_t>(dev, h->dev.merge_off);
+    p.merge_list = at<int32_t>(dev, h->dev.merge_list);
+    p.arrive = at<int32_t>(ws, w.arrive);
+    p.ready = at<int32_t>(ws, w.ready);
+    p.merge_ctr = at<int32_t>(ws, w.merge_ctr);
+    p.o = static_cast<__nv_bfloat16*>(o);
+    p.lse = lse;
+    p.n_slots = static_cast<int>(h->n_mtiles * h->Hkv);
+    p.Hkv = h->Hkv;
+    p.Hq = h->Hq;
+  }
   int sms = num_sms();
   if (sms <= 0) return cuda_fail(cudaGetLastError());
   const int grid = fwd_grid(h->d, sms, h->n_fwd, h->n_fwd_pairs);
@@ -228,6 +249,33 @@ extern "C" int skv_attn_fwd(const void* plan, const skv_problem* prob, const voi
   if (e == cudaSuccess) e = mark(SKV_KERNEL_FWD, 1, stream);
   if (e != cudaSuccess) return cuda_fail(e);
   return SKV_OK;
+}
+
+}  // namespace
+
+extern "C" int skv_attn_fwd(const void* plan, const skv_problem* prob, const void* q, const void* k,
+                            const void* v, void* ws, size_t ws_bytes, skv_stream_t stream_) {
+  int rc = SKV_OK;
+  const PlanHeader* h = checked_plan(plan, prob, &rc);
+  if (!h) return rc;
+  return run_fwd(h, plan, q, k, v, ws, ws_bytes, nullptr, nullptr, reinterpret_cast<cudaStream_t>(stream_));
+}
+
+extern "C" int skv_attn_fwd_merged(const void* plan, const skv_problem* prob, const void* q, const void* k,
+                                   const void* v, void* o, float* lse, void* ws, size_t ws_bytes,
+                                   skv_stream_t stream_) {
+  int rc = SKV_OK;
+  const PlanHeader* h = checked_plan(plan, prob, &rc);
+  if (!h) return rc;
+  if (!o || !lse) return SKV_EINVAL;
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  if (h->empty_slots > 0) {
+    // a shard plan whose rank has no unit for some query tiles: those rows are merged (O = 0,
+    // LSE = -inf) by the merge kernel, launched after the forward
+    rc = run_fwd(h, plan, q, k, v, ws, ws_bytes, nullptr, nullptr, stream);
+    return rc != SKV_OK ? rc : skv_lse_merge(plan, prob, ws, o, lse, stream_);
+  }
+  return run_fwd(h, plan, q, k, v, ws, ws_bytes, o, lse, stream);
 }
 
 extern "C" int skv_lse_merge(const void* plan, const skv_problem* prob, const void* ws, void* o, float* lse,
@@ -244,6 +292,7 @@ extern "C" int skv_lse_merge(const void* plan, const skv_problem* prob, const vo
   p.merge_list = at<int32_t>(dev, h->dev.merge_list);
   p.part_o = at<float>(ws, w.fwd_o);
   p.part_lse = at<float>(ws, w.fwd_lse);
+  p.partial_bf16 = (h->policy & SKV_PLAN_PARTIALS_BF16) ? 1 : 0;
   p.o = static_cast<__nv_bfloat16*>(o);
   p.lse = lse;
   p.n_rows = h->n_mtiles * h->Hkv * kTileM;
@@ -258,22 +307,27 @@ extern "C" int skv_lse_merge(const void* plan, const skv_problem* prob, const vo
   return SKV_OK;
 }
 
-extern "C" int skv_attn_bwd(const void* plan, const skv_problem* prob, const void* q, const void* k,
-                            const void* v, const void* o, const float* lse, const void* dout, void* dq, void* dk,
-                            void* dv, void* ws, size_t ws_bytes, skv_stream_t stream_) {
+namespace {
+
+// dq_f32: write dQ as fp32 (this plan's contribution, to be summed over ranks) instead of bf16.
+int run_bwd(const PlanHeader* h, const void* plan, const void* q, const void* k, const void* v, const void* o,
+            const float* lse, const void* dout, void* dq, void* dk, void* dv, void* ws, size_t ws_bytes,
+            cudaStream_t stream, bool det, bool dq_f32 = false) {
   int rc = SKV_OK;
-  const PlanHeader* h = checked_plan(plan, prob, &rc);
-  if (!h) return rc;
-  if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv || !ws) return SKV_EINVAL;
+  if (!q || !o || !lse || !dout || !dq || !ws) return SKV_EINVAL;
+  if (h->kv_rows > 0 && (!k || !v || !dk || !dv)) return SKV_EINVAL;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse) || !aligned16(dout) ||
       !aligned16(dq) || !aligned16(dk) || !aligned16(dv) || reinterpret_cast<uintptr_t>(ws) % 256 != 0)
     return SKV_EINVAL;
   const WsLayout w = ws_layout(*h);
   if (ws_bytes < w.bwd_end) return SKV_EWORKSPACE;
-  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
-  rc = prepare_ws(*h, plan, ws, w, stream);
+  rc = prepare_ws(*h, plan, ws, w, stream, det);
   if (rc != SKV_OK) return rc;
   cudaError_t e;
+  if (det) {
+    e = cudaMemsetAsync(at<uint8_t>(ws, w.bwd_turn), 0, w.bwd_end - w.bwd_turn, stream);
+    if (e != cudaSuccess) return cuda_fail(e);
+  }
   float* delta = at<float>(ws, w.bwd_delta);
   float* dq_acc = at<float>(ws, w.bwd_dq);
   const long long n_rows = h->Nq * h->Hq;
@@ -281,17 +335,17 @@ extern "C" int skv_attn_bwd(const void* plan, const skv_problem* prob, const voi
   // dead ranges, in the device section) in one launch
   int64_t dead_rows = 0;
   const int64_t* dead = at<int64_t>(plan, h->dead_off);
-  for (int b = 0; b < h->B; ++b) dead_rows += std::max<int64_t>(0, dead[2 * b + 1] - dead[2 * b]);
+  for (int i = 0; i < h->n_dead; ++i) dead_rows += std::max<int64_t>(0, dead[2 * i + 1] - dead[2 * i]);
   e = launch_bwd_prep(h->d, static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dout), delta,
-                      dq_acc, n_rows, at<int64_t>(at<uint8_t>(ws, w.dev), h->dev.dead), h->B, dead_rows,
-                      static_cast<__nv_bfloat16*>(dk), static_cast<__nv_bfloat16*>(dv), h->Hkv, stream);
+                      dq_acc, n_rows, at<int64_t>(at<uint8_t>(ws, w.dev), h->dev.dead), h->n_dead, dead_rows,
+                      static_cast<__nv_bfloat16*>(dk), static_cast<__nv_bfloat16*>(dv), h->kv_heads, stream);
   if (e != cudaSuccess) return cuda_fail(e);
   if (h->n_bwd > 0) {
     CUtensorMap tq, tk, tv, tdo;
     if ((rc = make_map(&tq, q, h->Nq, h->Hq, h->d, h->G, h->tile_tokens)) != SKV_OK) return rc;
     if ((rc = make_map(&tdo, dout, h->Nq, h->Hq, h->d, h->G, h->tile_tokens)) != SKV_OK) return rc;
-    if ((rc = make_map(&tk, k, h->Ltot, h->Hkv, h->d, 1, kTileN)) != SKV_OK) return rc;
-    if ((rc = make_map(&tv, v, h->Ltot, h->Hkv, h->d, 1, kTileN)) != SKV_OK) return rc;
+    if ((rc = make_map(&tk, k, h->kv_rows, h->kv_heads, h->d, 1, kTileN)) != SKV_OK) return rc;
+    if ((rc = make_map(&tv, v, h->kv_rows, h->kv_heads, h->d, 1, kTileN)) != SKV_OK) return rc;
     const uint8_t* dev = at<uint8_t>(ws, w.dev);
     BwdParams p{};
     p.mtiles = at<MTile>(dev, h->dev.mtiles);
@@ -305,9 +359,17 @@ extern "C" int skv_attn_bwd(const void* plan, const skv_problem* prob, const voi
     p.dq_acc = dq_acc;
     p.dk = static_cast<__nv_bfloat16*>(dk);
     p.dv = static_cast<__nv_bfloat16*>(dv);
+    p.kv_heads = h->kv_heads;
     p.stamps = g_bwd_stamps;
     p.timeout_ns = kTimeoutNs;
-    p.P = h->P;
+    if (det) {
+      p.rank = at<int32_t>(dev, h->dev.bwd_rank);
+      p.det_order = at<int32_t>(dev, h->dev.bwd_det_order);
+      p.turn = at<int32_t>(ws, w.bwd_turn);
+      p.n_bwd = static_cast<int>(h->n_bwd);
+      p.det = 1;
+    }
+    p.P = h->n_queues;
     p.G = h->G;
     p.Hq = h->Hq;
     p.Hkv = h->Hkv;
@@ -323,10 +385,64 @@ extern "C" int skv_attn_bwd(const void* plan, const skv_problem* prob, const voi
     if (e == cudaSuccess) e = mark(SKV_KERNEL_BWD, 1, stream);
     if (e != cudaSuccess) return cuda_fail(e);
   }
-  e = launch_dq_cast(dq_acc, static_cast<__nv_bfloat16*>(dq),
-                     static_cast<float>(1.0 / std::sqrt(static_cast<double>(h->d))), n_rows * h->d, stream);
+  const float dq_scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(h->d)));
+  e = dq_f32 ? launch_dq_scale(dq_acc, static_cast<float*>(dq), dq_scale, n_rows * h->d, stream)
+             : launch_dq_cast(dq_acc, static_cast<__nv_bfloat16*>(dq), dq_scale, n_rows * h->d, stream);
   if (e != cudaSuccess) return cuda_fail(e);
   return SKV_OK;
+}
+
+}  // namespace
+
+extern "C" int skv_attn_bwd(const void* plan, const skv_problem* prob, const void* q, const void* k,
+                            const void* v, const void* o, const float* lse, const void* dout, void* dq, void* dk,
+                            void* dv, void* ws, size_t ws_bytes, skv_stream_t stream) {
+  int rc = SKV_OK;
+  const PlanHeader* h = checked_plan(plan, prob, &rc);
+  if (!h) return rc;
+  return run_bwd(h, plan, q, k, v, o, lse, dout, dq, dk, dv, ws, ws_bytes, reinterpret_cast<cudaStream_t>(stream),
+                 false);
+}
+
+extern "C" int skv_attn_bwd_deterministic(const void* plan, const skv_problem* prob, const void* q, const void* k,
+                                          const void* v, const void* o, const float* lse, const void* dout,
+                                          void* dq, void* dk, void* dv, void* ws, size_t ws_bytes,
+                                          skv_stream_t stream) {
+  int rc = SKV_OK;
+  const PlanHeader* h = checked_plan(plan, prob, &rc);
+  if (!h) return rc;
+  return run_bwd(h, plan, q, k, v, o, lse, dout, dq, dk, dv, ws, ws_bytes, reinterpret_cast<cudaStream_t>(stream),
+                 true);
+}
+
+extern "C" int skv_attn_bwd_partial(const void* plan, const skv_problem* prob, const void* q, const void* k,
+                                    const void* v, const void* o, const float* lse, const void* dout, float* dq,
+                                    void* dk, void* dv, void* ws, size_t ws_bytes, skv_stream_t stream) {
+  int rc = SKV_OK;
+  const PlanHeader* h = checked_plan(plan, prob, &rc);
+  if (!h) return rc;
+  return run_bwd(h, plan, q, k, v, o, lse, dout, dq, dk, dv, ws, ws_bytes, reinterpret_cast<cudaStream_t>(stream),
+                 false, true);
+}
+
+extern "C" int skv_lse_combine(const void* o_parts, const float* lse_parts, int n_parts, int64_t n_rows,
+                               int head_dim, void* o, float* lse, skv_stream_t stream) {
+  if (n_parts < 1 || n_rows < 0 || (head_dim != 64 && head_dim != 128)) return SKV_EINVAL;
+  if (n_rows > 0 && (!o_parts || !lse_parts || !o || !lse)) return SKV_EINVAL;
+  if (!aligned16(o_parts) || !aligned16(o) || reinterpret_cast<uintptr_t>(lse_parts) % 4 != 0 ||
+      reinterpret_cast<uintptr_t>(lse) % 4 != 0)
+    return SKV_EINVAL;
+  cudaError_t e = launch_lse_combine(head_dim, static_cast<const __nv_bfloat16*>(o_parts), lse_parts, n_parts, n_rows,
+                                     static_cast<__nv_bfloat16*>(o), lse, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? SKV_OK : cuda_fail(e);
+}
+
+extern "C" int skv_dq_combine(const float* dq_parts, int n_parts, int64_t n, void* dq, skv_stream_t stream) {
+  if (n_parts < 1 || n < 0 || n % 4 != 0) return SKV_EINVAL;
+  if (n > 0 && (!dq_parts || !dq || !aligned16(dq_parts) || !aligned16(dq))) return SKV_EINVAL;
+  cudaError_t e = launch_dq_combine(dq_parts, n_parts, n, static_cast<__nv_bfloat16*>(dq),
+                                    reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? SKV_OK : cuda_fail(e);
 }
 
 extern "C" int skv_status(const void* ws, skv_stream_t stream_) {

@@ -53,7 +53,7 @@ struct BwdShared {
   int32_t kend[2][128]; // absolute key end of the tile rows
 };
 
-template <int D>
+template <int D, bool kDet>  // kDet: dQ added in ascending key order under turn counters
 __global__ void __launch_bounds__(256, 1)
     bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
@@ -109,15 +109,21 @@ __global__ void __launch_bounds__(256, 1)
       bool ok = true;
       while (ok) {
         int u = -1;
-        while (visited < p.P) {
-          const int cnt = p.part_off[part + 1] - p.part_off[part];
-          const int idx = atomicAdd(&p.counters[part], 1);
-          if (idx < cnt) {
-            u = p.part_off[part] + idx;
-            break;
+        if constexpr (kDet) {
+          // one queue in (sample, rank, kv head) order: a unit only ever waits for units taken before it
+          const int idx = atomicAdd(&p.counters[0], 1);
+          if (idx < p.n_bwd) u = p.det_order[idx];
+        } else {
+          while (visited < p.P) {
+            const int cnt = p.part_off[part + 1] - p.part_off[part];
+            const int idx = atomicAdd(&p.counters[part], 1);
+            if (idx < cnt) {
+              u = p.part_off[part] + idx;
+              break;
+            }
+            part = (part + 1 == p.P) ? 0 : part + 1;
+            ++visited;
           }
-          part = (part + 1 == p.P) ? 0 : part + 1;
-          ++visited;
         }
         const int slot = n_units & 1;
         if (n_units >= 2 && !mbar_wait(&sh.sched_empty[slot], ((n_units >> 1) - 1) & 1, status, lim)) break;
@@ -128,8 +134,8 @@ __global__ void __launch_bounds__(256, 1)
         if (n_units >= 1 && !mbar_wait(&sh.kv_empty, (n_units - 1) & 1, status, lim)) break;
         mbar_arrive_expect_tx(&sh.kv_full, 2 * L::kTile);
         for (int db = 0; db < kDBlocks; ++db) {
-          tma_load_3d(smem + L::kK + db * (128 * 128), &tmK, &sh.kv_full, db * 64, U.g, U.kbeg);
-          tma_load_3d(smem + L::kV + db * (128 * 128), &tmV, &sh.kv_full, db * 64, U.g, U.kbeg);
+          tma_load_3d(smem + L::kK + db * (128 * 128), &tmK, &sh.kv_full, db * 64, U.kvh, U.kbeg - U.kshift);
+          tma_load_3d(smem + L::kV + db * (128 * 128), &tmV, &sh.kv_full, db * 64, U.kvh, U.kbeg - U.kshift);
         }
         ++n_units;
         for (int mt = U.mt_begin; mt < U.mt_end; ++mt) {
@@ -307,12 +313,17 @@ __global__ void __launch_bounds__(256, 1)
         if (!mbar_wait_warp(&sh.dq_full, qc & 1, status, lim)) { ok = false; break; }
         tc_fence_after();
         float* dst = p.dq_acc + (static_cast<size_t>(token) * p.Hq + h) * D;
+        // deterministic mode: this warp's 32 rows are added after every lower-ranked unit of the sample and
+        // kv head has added its own (ascending key order); the turn fixes the order in which the fp32
+        // reductions reach each address
+        int32_t* turn = kDet ? p.turn + (static_cast<size_t>(mt) * p.Hkv + U.g) * 8 + (warp & 3) : nullptr;
+        const bool my_turn = kDet && turn_wait(turn, p.rank[u], status, lim, lane);
 #pragma unroll 1
         for (int c = 0; c < D; c += 32) {
           uint32_t v[32];
           tmem_ld32(lane_base + kColDQ + c, v);
           tmem_wait_ld();
-          if (row_ok) {
+          if (row_ok && (!kDet || my_turn)) {
 #pragma unroll
             for (int i = 0; i < 32; i += 4)
               atomicAdd(reinterpret_cast<float4*>(dst + c + i),
@@ -320,6 +331,7 @@ __global__ void __launch_bounds__(256, 1)
                                     __uint_as_float(v[i + 3])));
           }
         }
+        if (kDet && my_turn) turn_pass(turn, p.rank[u] + 1, lane);
         tc_fence_before();
         mbar_arrive(&sh.dq_free);
         ++qc;
@@ -327,7 +339,7 @@ __global__ void __launch_bounds__(256, 1)
       if (!ok) break;
       // dK, dV of the unit's keys (every MMA of the unit completed: dq_full above)
       tc_fence_after();
-      const size_t krow = (static_cast<size_t>(my_key) * p.Hkv + U.g) * D;
+      const size_t krow = (static_cast<size_t>(my_key - U.kshift) * p.kv_heads + U.kvh) * D;
 #pragma unroll 1
       for (int c = 0; c < D; c += 32) {
         uint32_t vv[32], vk[32];
@@ -370,7 +382,7 @@ int bwd_smem_bytes(int d) { return d == 64 ? BwdSmem<64>::kDyn : bwd2_smem_bytes
 cudaError_t launch_bwd(int d, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                        const CUtensorMap& tdo, const BwdParams& p, int grid, cudaStream_t stream) {
   if (d == 128) return launch_bwd2(tq, tk, tv, tdo, p, grid, stream);
-  auto k = bwd_kernel<64>;
+  auto k = p.det ? bwd_kernel<64, true> : bwd_kernel<64, false>;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, BwdSmem<64>::kDyn);
   if (e != cudaSuccess) return e;
   k<<<grid, 256, BwdSmem<64>::kDyn, stream>>>(tq, tk, tv, tdo, p);

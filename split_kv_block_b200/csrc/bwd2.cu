@@ -64,8 +64,10 @@ __device__ __forceinline__ uint32_t col_a(int h) { return 64u * h; }         // 
 __device__ __forceinline__ uint32_t col_b(int h) { return 128u + 64u * h; }  // dP^T, then dQ^T, of half h
 constexpr uint32_t kColDV = 256, kColDK = 384;
 
-// kG: compile-time q-heads per kv-head (0 = runtime value p.G)
-template <int kG>
+// kG: compile-time q-heads per kv-head (0 = runtime value p.G). kDet: dQ added
+// in ascending key order under turn counters (deterministic backward) instead
+// of fp32 atomics in any order.
+template <int kG, bool kDet>
 __global__ void __launch_bounds__(384, 1)
     bwd2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                 const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
@@ -140,15 +142,21 @@ __global__ void __launch_bounds__(384, 1)
       };
       while (ok) {
         int u = -1;
-        while (visited < p.P) {
-          const int cnt = p.part_off[part + 1] - p.part_off[part];
-          const int idx = atomicAdd(&p.counters[part], 1);
-          if (idx < cnt) {
-            u = p.part_off[part] + idx;
-            break;
+        if constexpr (kDet) {
+          // one queue in (sample, rank, kv head) order: a unit only ever waits for units taken before it
+          const int idx = atomicAdd(&p.counters[0], 1);
+          if (idx < p.n_bwd) u = p.det_order[idx];
+        } else {
+          while (visited < p.P) {
+            const int cnt = p.part_off[part + 1] - p.part_off[part];
+            const int idx = atomicAdd(&p.counters[part], 1);
+            if (idx < cnt) {
+              u = p.part_off[part] + idx;
+              break;
+            }
+            part = (part + 1 == p.P) ? 0 : part + 1;
+            ++visited;
           }
-          part = (part + 1 == p.P) ? 0 : part + 1;
-          ++visited;
         }
         const int slot = n_units & 1;
         if (n_units >= 2 && !mbar_wait(&c.sched_empty[slot], ((n_units >> 1) - 1) & 1, status, lim)) break;
@@ -165,8 +173,8 @@ __global__ void __launch_bounds__(384, 1)
             if (kv_issued >= 1 && !mbar_wait(&c.kv_empty, (kv_issued - 1) & 1, status, lim)) { ok = false; break; }
             mbar_arrive_expect_tx(&c.kv_full, 2 * kTileBytes);
             for (int db = 0; db < 2; ++db) {
-              tma_load_3d(smem + kK + db * 16384, &tmK, &c.kv_full, db * 64, U.g, U.kbeg);
-              tma_load_3d(smem + kV + db * 16384, &tmV, &c.kv_full, db * 64, U.g, U.kbeg);
+              tma_load_3d(smem + kK + db * 16384, &tmK, &c.kv_full, db * 64, U.kvh, U.kbeg - U.kshift);
+              tma_load_3d(smem + kV + db * 16384, &tmV, &c.kv_full, db * 64, U.kvh, U.kbeg - U.kshift);
             }
             ++kv_issued;
             kv_loaded = true;
@@ -464,7 +472,28 @@ __global__ void __launch_bounds__(384, 1)
         mbar_arrive(&c.dq_free[wg]);
         // fp32 reduction: row r -> dq_acc[(tok0 + r / G) * Hq + g * G + r % G][t]
         float* base = p.dq_acc + (static_cast<size_t>(M.tok0) * p.Hq + static_cast<size_t>(U.g) * G) * kD + t;
-        if constexpr (kG > 0) {
+        if constexpr (kDet) {
+          // in ascending key order: this warp's 32 head-dim columns of the half's rows, after every
+          // lower-ranked unit of the sample and kv head has added its own. Within the turn the adds are
+          // fp32 reductions: the turn fixes the order in which they reach each address, and the fence
+          // of turn_pass waits for them before the next rank may start.
+          int32_t* turn = p.turn + (static_cast<size_t>(mt) * p.Hkv + U.g) * 8 + wg * 4 + (warp & 3);
+          const int my = p.rank[u];
+          if (turn_wait(turn, my, status, lim, lane)) {
+            const int nrows = M.ntok << lgG;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              const int r = 64 * wg + j;
+              if (r < nrows) atomicAdd(base + (r >> lgG) * tok_stride + (r & (G - 1)) * kD, __uint_as_float(q0[j]));
+            }
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              const int r = 64 * wg + 32 + j;
+              if (r < nrows) atomicAdd(base + (r >> lgG) * tok_stride + (r & (G - 1)) * kD, __uint_as_float(q1[j]));
+            }
+            turn_pass(turn, my + 1, lane);
+          }
+        } else if constexpr (kG > 0) {
           static_assert(64 % (kG > 0 ? kG : 1) == 0, "group size must divide 64");
           constexpr int kTok = 64 / (kG > 0 ? kG : 1);  // tokens per half tile
           const int tl0 = (64 * wg) / (kG > 0 ? kG : 1);
@@ -505,7 +534,8 @@ __global__ void __launch_bounds__(384, 1)
       tc_fence_after();
       const uint32_t acc_col = wg == 0 ? kColDV : kColDK;
       const float mul = wg == 0 ? 1.f : p.scale;
-      __nv_bfloat16* dst = (wg == 0 ? p.dv : p.dk) + (static_cast<size_t>(U.kbeg + t) * p.Hkv + U.g) * kD;
+      __nv_bfloat16* dst =
+          (wg == 0 ? p.dv : p.dk) + (static_cast<size_t>(U.kbeg - U.kshift + t) * p.kv_heads + U.kvh) * kD;
 #pragma unroll 1
       for (int cc = 0; cc < kD; cc += 32) {
         uint32_t v[32];
@@ -545,7 +575,8 @@ int bwd2_smem_bytes() { return kSmemBytes; }
 
 cudaError_t launch_bwd2(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tdo,
                         const BwdParams& p, int grid, cudaStream_t stream) {
-  auto kern = p.G == 4 ? bwd2_kernel<4> : bwd2_kernel<0>;
+  auto kern = p.det ? (p.G == 4 ? bwd2_kernel<4, true> : bwd2_kernel<0, true>)
+                    : (p.G == 4 ? bwd2_kernel<4, false> : bwd2_kernel<0, false>);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
   if (e != cudaSuccess) return e;
   kern<<<grid, 384, kSmemBytes, stream>>>(tq, tk, tv, tdo, p);

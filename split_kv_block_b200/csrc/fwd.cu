@@ -25,6 +25,7 @@
 
 #include "kernels.h"
 #include "sm100.cuh"
+#include "tail_merge.cuh"
 
 namespace skv {
 
@@ -50,9 +51,11 @@ struct FwdBarriers {
   uint64_t final_mma;
   int32_t sched[2];
   uint32_t tmem_base;
+  int32_t merge_slot;  // tail merge: slot being merged (broadcast)
 };
 
-template <int D>
+// kMerge: the LSE merge runs in the kernel's tail (skv_attn_fwd_merged).
+template <int D, bool kMerge>
 __global__ void __launch_bounds__(256, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
@@ -135,13 +138,13 @@ __global__ void __launch_bounds__(256, 1)
           mbar_arrive_expect_tx(&bars.k_full[st], L::kKVBytes);
           for (int db = 0; db < kDBlocks; ++db)
             tma_load_3d(smem + L::kK0 + st * L::kKVBytes + db * (kTileN * 128), &tmK, &bars.k_full[st], db * 64,
-                        U.g, kb);
+                        U.kvh, kb - U.kshift);
           ++k_issued;
           if (use >= 1 && !mbar_wait(&bars.v_empty[st], (use - 1) & 1, status, lim)) { ok = false; break; }
           mbar_arrive_expect_tx(&bars.v_full[st], L::kKVBytes);
           for (int db = 0; db < kDBlocks; ++db)
             tma_load_3d(smem + L::kV0 + st * L::kKVBytes + db * (kTileN * 128), &tmV, &bars.v_full[st], db * 64,
-                        U.g, kb);
+                        U.kvh, kb - U.kshift);
           ++v_issued;
         }
         ++n_units;
@@ -325,21 +328,41 @@ __global__ void __launch_bounds__(256, 1)
       tc_fence_after();
       const float inv_l = l > 0.f ? 1.f / l : 0.f;
       float* orow = p.part_o + (static_cast<size_t>(u) * kTileM + r) * D;
+      const uint64_t pol = l2_policy_evict_last();
+      __nv_bfloat16* orow16 = reinterpret_cast<__nv_bfloat16*>(p.part_o) + (static_cast<size_t>(u) * kTileM + r) * D;
 #pragma unroll
       for (int c = 0; c < D; c += 32) {
         uint32_t v[32];
         tmem_ld32(lane_base + kColO + c, v);
         tmem_wait_ld();
+        if (p.partial_bf16) {
 #pragma unroll
-        for (int i = 0; i < 32; i += 4) {
-          float4 o4 = make_float4(__uint_as_float(v[i]) * inv_l, __uint_as_float(v[i + 1]) * inv_l,
-                                  __uint_as_float(v[i + 2]) * inv_l, __uint_as_float(v[i + 3]) * inv_l);
-          *reinterpret_cast<float4*>(orow + c + i) = o4;
+          for (int i = 0; i < 32; i += 8) {
+            const uint4 w = make_uint4(pack_bf16(__uint_as_float(v[i]) * inv_l, __uint_as_float(v[i + 1]) * inv_l),
+                                       pack_bf16(__uint_as_float(v[i + 2]) * inv_l, __uint_as_float(v[i + 3]) * inv_l),
+                                       pack_bf16(__uint_as_float(v[i + 4]) * inv_l, __uint_as_float(v[i + 5]) * inv_l),
+                                       pack_bf16(__uint_as_float(v[i + 6]) * inv_l, __uint_as_float(v[i + 7]) * inv_l));
+            if (p.partials_l2_last)
+              st_global_v4u_hint(orow16 + c + i, w, pol);
+            else
+              *reinterpret_cast<uint4*>(orow16 + c + i) = w;
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; i += 4) {
+            float4 o4 = make_float4(__uint_as_float(v[i]) * inv_l, __uint_as_float(v[i + 1]) * inv_l,
+                                    __uint_as_float(v[i + 2]) * inv_l, __uint_as_float(v[i + 3]) * inv_l);
+            if (p.partials_l2_last)
+              st_global_v4_hint(orow + c + i, o4, pol);
+            else
+              *reinterpret_cast<float4*>(orow + c + i) = o4;
+          }
         }
       }
       tc_fence_before();
       mbar_arrive(&bars.o_free);
       p.part_lse[static_cast<size_t>(u) * kTileM + r] = l > 0.f ? (m + lg2(l)) * 0.69314718055994531f : -INFINITY;
+      if constexpr (kMerge) tail_merge_arrive(p, U.mt * p.Hkv + U.g, lane);
       if (p.stamps && r == 0) p.stamps[2 * u + 1] = static_cast<long long>(globaltimer_ns());
       tcount += nt;
       ++n_units;
@@ -351,6 +374,7 @@ __global__ void __launch_bounds__(256, 1)
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }
+  if constexpr (kMerge) tail_merge<D>(p, &bars.merge_slot);
 }
 
 int fwd_smem_bytes(int d) { return d == 64 ? FwdSmem<64>::kDyn : FwdSmem<128>::kDyn; }
@@ -359,7 +383,7 @@ int fwd_smem_bytes(int d) { return d == 64 ? FwdSmem<64>::kDyn : FwdSmem<128>::k
 cudaError_t launch_fwd(int d, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                        const FwdParams& p, int grid, cudaStream_t stream) {
   if (d == 128) return launch_fwd2(tq, tk, tv, p, grid, stream);
-  auto k = fwd_kernel<64>;
+  auto k = p.o ? fwd_kernel<64, true> : fwd_kernel<64, false>;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, FwdSmem<64>::kDyn);
   if (e != cudaSuccess) return e;
   k<<<grid, 256, FwdSmem<64>::kDyn, stream>>>(tq, tk, tv, p);

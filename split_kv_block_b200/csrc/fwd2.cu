@@ -23,6 +23,7 @@
 
 #include "kernels.h"
 #include "sm100.cuh"
+#include "tail_merge.cuh"
 
 namespace skv {
 namespace {
@@ -46,6 +47,7 @@ struct Ctl {
   uint64_t final_mma;
   int32_t sched[2];
   uint32_t tmem_base;
+  int32_t merge_slot;  // tail merge: slot being merged (broadcast)
 };
 constexpr int kSmemBytes = kCtl + static_cast<int>(sizeof(Ctl));
 static_assert(kSmemBytes <= 232448, "shared memory budget");
@@ -106,6 +108,9 @@ __device__ __forceinline__ float exp_row(const uint32_t (&sv)[128], float sl2, f
   return (rs[0] + rs[1]) + (rs[2] + rs[3]);
 }
 
+// kMerge: the LSE merge runs in the kernel's tail (skv_attn_fwd_merged); the
+// plain forward is compiled without that code.
+template <bool kMerge>
 __global__ void __launch_bounds__(384, 1)
     fwd2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                 const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
@@ -183,19 +188,20 @@ __global__ void __launch_bounds__(384, 1)
             tma_load_3d(smem + kQ0 + t * kTileBytes + db * 16384, &tmQ, &c.q_full[t], db * 64, U.g * p.G, M.tok0);
           ++q_iss[t];
         }
-        const int g = p.units[pr.slot[0]].g;
+        // K/V buffer coordinates of the pair's item: head kvh, key kb at row kb - kshift
+        const int kvh = p.units[pr.slot[0]].kvh, kshift = p.units[pr.slot[0]].kshift;
         for (int kb = pr.kbeg; kb < pr.kend && ok; kb += kTileN, ++kv) {
           const int st = kv & 1;
           const uint32_t use = kv >> 1;
           if (use >= 1 && !mbar_wait(&c.k_empty[st], (use - 1) & 1, status, lim)) { ok = false; break; }
           mbar_arrive_expect_tx(&c.k_full[st], kTileBytes);
           for (int db = 0; db < 2; ++db)
-            tma_load_3d(smem + kK0 + st * kTileBytes + db * 16384, &tmK, &c.k_full[st], db * 64, g, kb);
+            tma_load_3d(smem + kK0 + st * kTileBytes + db * 16384, &tmK, &c.k_full[st], db * 64, kvh, kb - kshift);
           ++k_iss;
           if (use >= 1 && !mbar_wait(&c.v_empty[st], (use - 1) & 1, status, lim)) { ok = false; break; }
           mbar_arrive_expect_tx(&c.v_full[st], kTileBytes);
           for (int db = 0; db < 2; ++db)
-            tma_load_3d(smem + kV0 + st * kTileBytes + db * 16384, &tmV, &c.v_full[st], db * 64, g, kb);
+            tma_load_3d(smem + kV0 + st * kTileBytes + db * 16384, &tmV, &c.v_full[st], db * 64, kvh, kb - kshift);
           ++v_iss;
         }
         ++n_units;
@@ -420,21 +426,42 @@ __global__ void __launch_bounds__(384, 1)
       tc_fence_after();
       const float inv_l = l > 0.f ? 1.f / l : 0.f;
       float* orow = p.part_o + (static_cast<size_t>(sl) * kTileM + r) * kD;
+      const uint64_t pol = l2_policy_evict_last();
+      __nv_bfloat16* orow16 = reinterpret_cast<__nv_bfloat16*>(p.part_o) + (static_cast<size_t>(sl) * kTileM + r) * kD;
 #pragma unroll 1
       for (int cc = 0; cc < kD; cc += 32) {
         uint32_t v[32];
         tmem_ld32(tO + cc, v);
         tmem_wait_ld();
+        if (p.partial_bf16) {
 #pragma unroll
-        for (int i = 0; i < 32; i += 4)
-          *reinterpret_cast<float4*>(orow + cc + i) =
-              make_float4(__uint_as_float(v[i]) * inv_l, __uint_as_float(v[i + 1]) * inv_l,
-                          __uint_as_float(v[i + 2]) * inv_l, __uint_as_float(v[i + 3]) * inv_l);
+          for (int i = 0; i < 32; i += 8) {
+            const uint4 w = make_uint4(pack_bf16(__uint_as_float(v[i]) * inv_l, __uint_as_float(v[i + 1]) * inv_l),
+                                       pack_bf16(__uint_as_float(v[i + 2]) * inv_l, __uint_as_float(v[i + 3]) * inv_l),
+                                       pack_bf16(__uint_as_float(v[i + 4]) * inv_l, __uint_as_float(v[i + 5]) * inv_l),
+                                       pack_bf16(__uint_as_float(v[i + 6]) * inv_l, __uint_as_float(v[i + 7]) * inv_l));
+            if (p.partials_l2_last)
+              st_global_v4u_hint(orow16 + cc + i, w, pol);
+            else
+              *reinterpret_cast<uint4*>(orow16 + cc + i) = w;
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; i += 4) {
+            const float4 o4 = make_float4(__uint_as_float(v[i]) * inv_l, __uint_as_float(v[i + 1]) * inv_l,
+                                          __uint_as_float(v[i + 2]) * inv_l, __uint_as_float(v[i + 3]) * inv_l);
+            if (p.partials_l2_last)
+              st_global_v4_hint(orow + cc + i, o4, pol);
+            else
+              *reinterpret_cast<float4*>(orow + cc + i) = o4;
+          }
+        }
       }
       tc_fence_before();
       mbar_arrive(&c.o_free[t]);
       p.part_lse[static_cast<size_t>(sl) * kTileM + r] =
           l > 0.f ? (m_ref + lg2(l)) * 0.69314718055994531f : -INFINITY;
+      if constexpr (kMerge) tail_merge_arrive(p, U.mt * p.Hkv + U.g, lane);
       if (p.stamps && r == 0) p.stamps[2 * sl + 1] = static_cast<long long>(globaltimer_ns());
     }
   }
@@ -444,6 +471,7 @@ __global__ void __launch_bounds__(384, 1)
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
+  if constexpr (kMerge) tail_merge<kD>(p, &c.merge_slot);
 }
 
 }  // namespace
@@ -452,9 +480,10 @@ int fwd2_smem_bytes() { return kSmemBytes; }
 
 cudaError_t launch_fwd2(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const FwdParams& p,
                         int grid, cudaStream_t stream) {
-  cudaError_t e = cudaFuncSetAttribute(fwd2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  auto kern = p.o ? fwd2_kernel<true> : fwd2_kernel<false>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
   if (e != cudaSuccess) return e;
-  fwd2_kernel<<<grid, 384, kSmemBytes, stream>>>(tq, tk, tv, p);
+  kern<<<grid, 384, kSmemBytes, stream>>>(tq, tk, tv, p);
   return cudaGetLastError();
 }
 

@@ -94,8 +94,8 @@ extern "C" int skv_attn_fwd_noalloc(const void* plan, const skv_problem* prob, c
 
   CUtensorMap tq, tk, tv;
   rc = skv_make_tile_map(&tq, q, h->Nq, h->Hq, h->d, h->G, h->tile_tokens);
-  if (rc == SKV_OK) rc = skv_make_tile_map(&tk, k, h->Ltot, h->Hkv, h->d, 1, kTileN);
-  if (rc == SKV_OK) rc = skv_make_tile_map(&tv, v, h->Ltot, h->Hkv, h->d, 1, kTileN);
+  if (rc == SKV_OK) rc = skv_make_tile_map(&tk, k, h->kv_rows, h->kv_heads, h->d, 1, kTileN);
+  if (rc == SKV_OK) rc = skv_make_tile_map(&tv, v, h->kv_rows, h->kv_heads, h->d, 1, kTileN);
   if (rc != SKV_OK) return rc;
   const uint8_t* dev = base + w.dev;
   FwdParams p{};
@@ -109,9 +109,10 @@ extern "C" int skv_attn_fwd_noalloc(const void* plan, const skv_problem* prob, c
   p.status = reinterpret_cast<int*>(base + w.status);
   p.part_o = reinterpret_cast<float*>(base + w.fwd_o);
   p.part_lse = reinterpret_cast<float*>(base + w.fwd_lse);
+  p.partial_bf16 = (h->policy & SKV_PLAN_PARTIALS_BF16) ? 1 : 0;
   p.stamps = nullptr;
   p.timeout_ns = 2000000000ull;
-  p.P = h->P;
+  p.P = h->n_queues;
   p.G = h->G;
   p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(h->d)));
   int dev_id = 0, sms = 0;
@@ -128,6 +129,7 @@ extern "C" int skv_attn_fwd_noalloc(const void* plan, const skv_problem* prob, c
   m.merge_list = reinterpret_cast<const int32_t*>(dev + h->dev.merge_list);
   m.part_o = p.part_o;
   m.part_lse = p.part_lse;
+  m.partial_bf16 = p.partial_bf16;
   m.o = static_cast<__nv_bfloat16*>(o);
   m.lse = lse;
   m.n_rows = h->n_mtiles * h->Hkv * kTileM;

@@ -104,7 +104,11 @@ struct Built {
   std::vector<int32_t> merge_off, merge_list;
   std::vector<BwdUnit> bwd;
   std::vector<int32_t> bwd_part_off;
-  std::vector<int64_t> dead;  // [2B]
+  std::vector<int32_t> bwd_item, bwd_part;  // host-side: item and partition of every backward unit
+  std::vector<int32_t> bwd_rank, bwd_det_order;
+  std::vector<int64_t> dead;  // [2 n_dead]
+  int shard = -1, n_queues = 1, kv_heads = 1;
+  int64_t kv_rows = 0;
   int64_t total_cost = 0;
   double imbalance = 0.0;
 };
@@ -220,7 +224,12 @@ void place(const Prob& q, int policy, Built& out) {
   out.imbalance = out.total_cost > 0 ? static_cast<double>(mx) * q.P / static_cast<double>(out.total_cost) - 1.0 : 0.0;
 }
 
-void make_lists(const Prob& q, const std::vector<SampleAnchors>& sa, Built& out) {
+// shard < 0: the full plan: every partition's items on P work queues; the
+// K/V buffers are the packed context, all kv heads per row. shard = p: the
+// items of partition p only, on one work queue; the K/V buffers hold those
+// items' keys, one kv head per row, items in (b, c, g, s) order (the layout a
+// context-parallel rank keeps of its own chunks).
+void make_lists(const Prob& q, const std::vector<SampleAnchors>& sa, int shard, Built& out) {
   // query tiles
   out.mtiles.clear();
   out.sample_mt.assign(q.B + 1, 0);
@@ -239,24 +248,51 @@ void make_lists(const Prob& q, const std::vector<SampleAnchors>& sa, Built& out)
   }
   out.sample_mt[q.B] = static_cast<int32_t>(out.mtiles.size());
 
-  // items of every partition in placement order
-  std::vector<std::vector<int32_t>> by_part(q.P);
-  for (int32_t id : out.placement) by_part[out.items[id].partition].push_back(id);
+  // K/V rows of every item, and the items each work queue runs in placement order
+  out.shard = shard;
+  out.n_queues = shard < 0 ? q.P : 1;
+  out.kv_heads = shard < 0 ? q.Hkv : 1;
+  std::vector<char> in_plan(out.items.size(), shard < 0 ? 1 : 0);
+  if (shard < 0) {
+    for (auto& it : out.items) it.kv_row = it.key_begin;
+    out.kv_rows = q.Ltot;
+  } else {
+    int64_t row = 0;
+    for (size_t id = 0; id < out.items.size(); ++id) {
+      skv_item& it = out.items[id];
+      if (it.partition == shard) {
+        in_plan[id] = 1;
+        it.kv_row = row;
+        row += it.key_end - it.key_begin;
+      } else {
+        it.kv_row = -1;
+      }
+    }
+    out.kv_rows = row;
+  }
+  std::vector<std::vector<int32_t>> by_queue(out.n_queues);
+  for (int32_t id : out.placement)
+    if (in_plan[id]) by_queue[shard < 0 ? out.items[id].partition : 0].push_back(id);
 
   out.fwd.clear();
-  out.fwd_part_off.assign(q.P + 1, 0);
+  out.fwd_part_off.assign(out.n_queues + 1, 0);
   out.pairs.clear();
-  out.pair_off.assign(q.P + 1, 0);
+  out.pair_off.assign(out.n_queues + 1, 0);
   out.bwd.clear();
-  out.bwd_part_off.assign(q.P + 1, 0);
+  out.bwd_item.clear();
+  out.bwd_part.clear();
+  out.bwd_part_off.assign(out.n_queues + 1, 0);
   std::vector<std::pair<int64_t, int32_t>> tiles;
   std::vector<std::pair<int32_t, int32_t>> item_fwd(out.items.size(), {0, 0});  // [first forward unit, count]
-  for (int p = 0; p < q.P; ++p) {
+  std::vector<int64_t> item_cov_end(out.items.size(), 0);  // end of the keys the item's backward units cover
+  for (int p = 0; p < out.n_queues; ++p) {
     out.fwd_part_off[p] = static_cast<int32_t>(out.fwd.size());
     out.pair_off[p] = static_cast<int32_t>(out.pairs.size());
     out.bwd_part_off[p] = static_cast<int32_t>(out.bwd.size());
-    for (int32_t id : by_part[p]) {
+    for (int32_t id : by_queue[p]) {
       const skv_item& it = out.items[id];
+      const int32_t kshift = static_cast<int32_t>(it.key_begin - it.kv_row);
+      const int32_t kvh = shard < 0 ? it.g : 0;
       // forward: live query tiles, longest key range first (ties by tile index). Tiles reaching past
       // the item's end all have its full range and come first in index order; only the others,
       // few per item, need sorting.
@@ -280,7 +316,9 @@ void make_lists(const Prob& q, const std::vector<SampleAnchors>& sa, Built& out)
         u.kbeg = static_cast<int32_t>(it.key_begin);
         u.kend = static_cast<int32_t>(it.key_begin - t.first);
         u.item = id;
-        u.part = p;
+        u.part = it.partition;
+        u.kshift = kshift;
+        u.kvh = kvh;
         // consecutive tiles (similar key extents) share a pair; the first is the longer
         if (ti % 2 == 0) {
           FwdPair pr{};
@@ -288,7 +326,7 @@ void make_lists(const Prob& q, const std::vector<SampleAnchors>& sa, Built& out)
           pr.slot[1] = -1;
           pr.kbeg = u.kbeg;
           pr.kend = u.kend;
-          pr.part = p;
+          pr.part = it.partition;
           out.pairs.push_back(pr);
         } else {
           out.pairs.back().slot[1] = static_cast<int32_t>(out.fwd.size());
@@ -301,6 +339,7 @@ void make_lists(const Prob& q, const std::vector<SampleAnchors>& sa, Built& out)
       // possible with unsorted anchors, are skipped by the kernel); a tile dead for one key tile is
       // dead for every later one, so the index only moves forward
       int32_t first = out.sample_mt[it.b];
+      item_cov_end[id] = it.key_begin;
       for (int64_t kb = it.key_begin; kb < it.key_end && kb < kmax_b; kb += kTileN) {
         BwdUnit u{};
         u.b = it.b;
@@ -310,15 +349,66 @@ void make_lists(const Prob& q, const std::vector<SampleAnchors>& sa, Built& out)
         while (first < out.sample_mt[it.b + 1] && out.mtiles[first].kmax <= kb) ++first;
         u.mt_begin = first;
         u.mt_end = out.sample_mt[it.b + 1];
-        u.item = id;
-        u.part = p;
+        u.kshift = kshift;
+        u.kvh = kvh;
+        item_cov_end[id] = u.kend;
         out.bwd.push_back(u);
+        out.bwd_item.push_back(id);
+        out.bwd_part.push_back(it.partition);
       }
     }
   }
-  out.fwd_part_off[q.P] = static_cast<int32_t>(out.fwd.size());
-  out.pair_off[q.P] = static_cast<int32_t>(out.pairs.size());
-  out.bwd_part_off[q.P] = static_cast<int32_t>(out.bwd.size());
+  out.fwd_part_off[out.n_queues] = static_cast<int32_t>(out.fwd.size());
+  out.pair_off[out.n_queues] = static_cast<int32_t>(out.pairs.size());
+  out.bwd_part_off[out.n_queues] = static_cast<int32_t>(out.bwd.size());
+
+  // Deterministic backward: the rank of every unit's key tile among the plan's key tiles of its (sample,
+  // kv head) in ascending key order, and the dispatch order (sample, rank, kv head). Items of one (sample,
+  // kv head) are numbered in ascending key order, so ranks run on from item to item. In a full plan every
+  // kv head has the same key tiles, so (sample, rank, kv head) numbers the units densely; a shard's heads
+  // differ, so its order is sorted.
+  {
+    std::vector<int32_t> first_rank(out.items.size(), 0);
+    std::vector<int32_t> running(static_cast<size_t>(q.Hkv), 0);
+    std::vector<int32_t> tiles_of_sample(q.B, 0);
+    int b_prev = -1;
+    for (size_t id = 0; id < out.items.size(); ++id) {
+      const skv_item& it = out.items[id];
+      if (it.b != b_prev) {
+        std::fill(running.begin(), running.end(), 0);
+        b_prev = it.b;
+      }
+      if (!in_plan[id]) continue;
+      first_rank[id] = running[it.g];
+      const int64_t kmax_b = q.ctx[it.b] + sa[it.b].max_a;
+      const int64_t hi = std::min<int64_t>(it.key_end, kmax_b);
+      const int32_t nt = hi > it.key_begin ? static_cast<int32_t>((hi - it.key_begin + kTileN - 1) / kTileN) : 0;
+      running[it.g] += nt;
+      tiles_of_sample[it.b] = std::max(tiles_of_sample[it.b], running[it.g]);
+    }
+    out.bwd_rank.assign(out.bwd.size(), 0);
+    for (size_t u = 0; u < out.bwd.size(); ++u) {
+      const skv_item& it = out.items[out.bwd_item[u]];
+      out.bwd_rank[u] = first_rank[out.bwd_item[u]] + static_cast<int32_t>((out.bwd[u].kbeg - it.key_begin) / kTileN);
+    }
+    out.bwd_det_order.assign(out.bwd.size(), -1);
+    if (shard < 0) {
+      std::vector<int64_t> base(q.B + 1, 0);
+      for (int b = 0; b < q.B; ++b) base[b + 1] = base[b] + static_cast<int64_t>(tiles_of_sample[b]) * q.Hkv;
+      for (size_t u = 0; u < out.bwd.size(); ++u) {
+        const int64_t pos = base[out.bwd[u].b] + static_cast<int64_t>(out.bwd_rank[u]) * q.Hkv + out.bwd[u].g;
+        if (pos >= 0 && pos < static_cast<int64_t>(out.bwd.size())) out.bwd_det_order[pos] = static_cast<int32_t>(u);
+      }
+    } else {
+      std::iota(out.bwd_det_order.begin(), out.bwd_det_order.end(), 0);
+      std::sort(out.bwd_det_order.begin(), out.bwd_det_order.end(), [&](int32_t x, int32_t y) {
+        const BwdUnit &a = out.bwd[x], &c = out.bwd[y];
+        if (a.b != c.b) return a.b < c.b;
+        if (out.bwd_rank[x] != out.bwd_rank[y]) return out.bwd_rank[x] < out.bwd_rank[y];
+        return a.g < c.g;
+      });
+    }
+  }
 
   // merge lists: per (query tile, kv head), forward units in ascending key order
   const size_t nslots = out.mtiles.size() * static_cast<size_t>(q.Hkv);
@@ -335,19 +425,37 @@ void make_lists(const Prob& q, const std::vector<SampleAnchors>& sa, Built& out)
       out.merge_list[fill[static_cast<size_t>(u.mt) * q.Hkv + u.g]++] = i;
     }
 
-  // keys whose gradients are zero: past the last backward tile of the sample
-  out.dead.assign(2 * static_cast<size_t>(q.B), 0);
-  std::vector<int64_t> live_end(q.B);
-  for (int b = 0; b < q.B; ++b) live_end[b] = q.ctx[b];
-  for (const auto& u : out.bwd) live_end[u.b] = std::max<int64_t>(live_end[u.b], u.kend);
-  for (int b = 0; b < q.B; ++b) {
-    out.dead[2 * b] = live_end[b];
-    out.dead[2 * b + 1] = q.ctx[b + 1];
+  // K/V rows whose gradients are zero (no query attends to them): in a full plan the keys of every
+  // sample past its last backward tile; in a shard, the rows of each item past its last backward tile
+  out.dead.clear();
+  if (shard < 0) {
+    std::vector<int64_t> live_end(q.B);
+    for (int b = 0; b < q.B; ++b) live_end[b] = q.ctx[b];
+    for (const auto& u : out.bwd) live_end[u.b] = std::max<int64_t>(live_end[u.b], u.kend);
+    for (int b = 0; b < q.B; ++b) {
+      out.dead.push_back(live_end[b]);
+      out.dead.push_back(q.ctx[b + 1]);
+    }
+  } else {
+    for (size_t id = 0; id < out.items.size(); ++id) {
+      if (!in_plan[id]) continue;
+      const skv_item& it = out.items[id];
+      if (item_cov_end[id] >= it.key_end) continue;
+      const int64_t lo = item_cov_end[id] - (it.key_begin - it.kv_row), hi = it.kv_row + (it.key_end - it.key_begin);
+      if (!out.dead.empty() && out.dead.back() == lo)
+        out.dead.back() = hi;  // adjacent rows: one range
+      else {
+        out.dead.push_back(lo);
+        out.dead.push_back(hi);
+      }
+    }
   }
 }
 
-int build(const skv_problem* prob, int policy, Built& out, Prob& q) {
-  if (policy != SKV_PLAN_LPT && policy != SKV_PLAN_STATIC) return SKV_EINVAL;
+int build(const skv_problem* prob, int policy, Built& out, Prob& q, int shard = -1) {
+  if ((policy & ~SKV_PLAN_PARTIALS_BF16) != SKV_PLAN_LPT && (policy & ~SKV_PLAN_PARTIALS_BF16) != SKV_PLAN_STATIC)
+    return SKV_EINVAL;
+  policy &= ~SKV_PLAN_PARTIALS_BF16;
   int rc = validate(prob, q);
   if (rc != SKV_OK) return rc;
   std::vector<SampleAnchors> sa(q.B);
@@ -358,9 +466,10 @@ int build(const skv_problem* prob, int policy, Built& out, Prob& q) {
     for (size_t i = 0; i < sa[b].a.size(); ++i) sa[b].prefix[i + 1] = sa[b].prefix[i] + sa[b].a[i];
     sa[b].max_a = sa[b].a.empty() ? 0 : sa[b].a.back();
   }
+  if (shard >= q.P) return SKV_EINVAL;
   make_items(q, policy, sa, out);
   place(q, policy, out);
-  make_lists(q, sa, out);
+  make_lists(q, sa, shard, out);
   return SKV_OK;
 }
 
@@ -390,13 +499,22 @@ PlanHeader layout_of(const Prob& q, int policy, const Built& b) {
   h.n_fwd_pairs = static_cast<int64_t>(b.pairs.size());
   h.imbalance = b.imbalance;
   h.fingerprint = 0;  // set by skv_plan from the caller's problem
+  h.shard = b.shard;
+  h.n_queues = b.n_queues;
+  h.kv_heads = b.kv_heads;
+  h.kv_rows = b.kv_rows;
+  h.n_dead = static_cast<int32_t>(b.dead.size() / 2);
+  h.empty_slots = 0;
+  for (size_t i = 0; i + 1 < b.merge_off.size(); ++i) h.empty_slots += b.merge_off[i + 1] == b.merge_off[i];
   uint64_t off = align_up(sizeof(PlanHeader), 256);
   h.items_off = off;
   off = align_up(off + b.items.size() * sizeof(skv_item), 64);
   h.load_off = off;
   off = align_up(off + static_cast<uint64_t>(q.P) * sizeof(int64_t), 64);
   h.dead_off = off;
-  off = align_up(off + b.dead.size() * sizeof(int64_t), 256);
+  off = align_up(off + b.dead.size() * sizeof(int64_t), 64);
+  h.bwd_part_host_off = off;
+  off = align_up(off + b.bwd_part.size() * sizeof(int32_t), 256);
   h.dev_off = off;
   uint64_t d = 0;
   auto put = [&](uint64_t bytes) { uint64_t at = d; d = align_up(d + bytes, 256); return at; };
@@ -411,6 +529,9 @@ PlanHeader layout_of(const Prob& q, int policy, const Built& b) {
   h.dev.bwd_units = put(b.bwd.size() * sizeof(BwdUnit));
   h.dev.bwd_part_off = put(b.bwd_part_off.size() * sizeof(int32_t));
   h.dev.dead = put(b.dead.size() * sizeof(int64_t));
+  h.dev.base_bytes = d;
+  h.dev.bwd_rank = put(b.bwd_rank.size() * sizeof(int32_t));
+  h.dev.bwd_det_order = put(b.bwd_det_order.size() * sizeof(int32_t));
   h.dev.bytes = d;
   h.total_bytes = h.dev_off + d;
   return h;
@@ -473,11 +594,13 @@ Built& scratch() {
   return b;
 }
 
-extern "C" int skv_plan_size(const skv_problem* prob, int policy, size_t* n_items, size_t* plan_bytes,
-                             size_t* ws_fwd_bytes, size_t* ws_bwd_bytes) {
+namespace {
+
+int plan_size(const skv_problem* prob, int policy, int shard, size_t* n_items, size_t* plan_bytes,
+              size_t* ws_fwd_bytes, size_t* ws_bwd_bytes) {
   Built& b = scratch();
   Prob q;
-  int rc = build(prob, policy, b, q);
+  int rc = build(prob, policy, b, q, shard);
   if (rc != SKV_OK) return rc;
   PlanHeader h = layout_of(q, policy, b);
   WsLayout w = ws_layout(h);
@@ -488,12 +611,12 @@ extern "C" int skv_plan_size(const skv_problem* prob, int policy, size_t* n_item
   return SKV_OK;
 }
 
-extern "C" int skv_plan(const skv_problem* prob, int policy, void* plan, size_t plan_bytes,
-                        int64_t* partition_load) {
+int write_plan(const skv_problem* prob, int policy, int shard, void* plan, size_t plan_bytes,
+               int64_t* partition_load) {
   if (!plan) return SKV_EINVAL;
   Built& b = scratch();
   Prob q;
-  int rc = build(prob, policy, b, q);
+  int rc = build(prob, policy, b, q, shard);
   if (rc != SKV_OK) return rc;
   PlanHeader h = layout_of(q, policy, b);
   if (plan_bytes < h.total_bytes) return SKV_EWORKSPACE;
@@ -504,6 +627,7 @@ extern "C" int skv_plan(const skv_problem* prob, int policy, void* plan, size_t 
   copy_to(base, h.items_off, b.items);
   copy_to(base, h.load_off, b.load);
   copy_to(base, h.dead_off, b.dead);
+  copy_to(base, h.bwd_part_host_off, b.bwd_part);
   uint8_t* dev = base + h.dev_off;
   copy_to(dev, h.dev.mtiles, b.mtiles);
   copy_to(dev, h.dev.tok_kend, b.tok_kend);
@@ -516,7 +640,43 @@ extern "C" int skv_plan(const skv_problem* prob, int policy, void* plan, size_t 
   copy_to(dev, h.dev.bwd_units, b.bwd);
   copy_to(dev, h.dev.bwd_part_off, b.bwd_part_off);
   copy_to(dev, h.dev.dead, b.dead);
+  copy_to(dev, h.dev.bwd_rank, b.bwd_rank);
+  copy_to(dev, h.dev.bwd_det_order, b.bwd_det_order);
   if (partition_load) std::memcpy(partition_load, b.load.data(), b.load.size() * sizeof(int64_t));
+  return SKV_OK;
+}
+
+}  // namespace
+
+extern "C" int skv_plan_size(const skv_problem* prob, int policy, size_t* n_items, size_t* plan_bytes,
+                             size_t* ws_fwd_bytes, size_t* ws_bwd_bytes) {
+  return plan_size(prob, policy, -1, n_items, plan_bytes, ws_fwd_bytes, ws_bwd_bytes);
+}
+
+extern "C" int skv_plan(const skv_problem* prob, int policy, void* plan, size_t plan_bytes,
+                        int64_t* partition_load) {
+  return write_plan(prob, policy, -1, plan, plan_bytes, partition_load);
+}
+
+extern "C" int skv_plan_shard_size(const skv_problem* prob, int policy, int partition, size_t* n_items,
+                                   size_t* plan_bytes, size_t* ws_fwd_bytes, size_t* ws_bwd_bytes) {
+  if (partition < 0) return SKV_EINVAL;
+  return plan_size(prob, policy, partition, n_items, plan_bytes, ws_fwd_bytes, ws_bwd_bytes);
+}
+
+extern "C" int skv_plan_shard(const skv_problem* prob, int policy, int partition, void* plan, size_t plan_bytes,
+                              int64_t* partition_load) {
+  if (partition < 0) return SKV_EINVAL;
+  return write_plan(prob, policy, partition, plan, plan_bytes, partition_load);
+}
+
+extern "C" int skv_plan_kv_layout(const void* plan, int64_t* kv_rows, int32_t* kv_heads, int32_t* shard) {
+  if (!plan) return SKV_EINVAL;
+  const PlanHeader* h = static_cast<const PlanHeader*>(plan);
+  if (h->magic != kPlanMagic || h->version != kPlanVersion) return SKV_EPLAN;
+  if (kv_rows) *kv_rows = h->kv_rows;
+  if (kv_heads) *kv_heads = h->kv_heads;
+  if (shard) *shard = h->shard;
   return SKV_OK;
 }
 
@@ -538,10 +698,8 @@ extern "C" int skv_plan_unit_partitions(const void* plan, int32_t* fwd_part, int
     const FwdUnit* u = reinterpret_cast<const FwdUnit*>(dev + h->dev.fwd_units);
     for (int64_t i = 0; i < h->n_fwd; ++i) fwd_part[i] = u[i].part;
   }
-  if (bwd_part) {
-    const BwdUnit* u = reinterpret_cast<const BwdUnit*>(dev + h->dev.bwd_units);
-    for (int64_t i = 0; i < h->n_bwd; ++i) bwd_part[i] = u[i].part;
-  }
+  if (bwd_part && h->n_bwd > 0)
+    std::memcpy(bwd_part, static_cast<const uint8_t*>(plan) + h->bwd_part_host_off, h->n_bwd * sizeof(int32_t));
   return SKV_OK;
 }
 

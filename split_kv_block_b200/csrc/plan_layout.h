@@ -24,14 +24,18 @@ struct MTile {
 };
 
 // Forward unit: one item's key range restricted to one query tile.
+// K/V buffer coordinates: key k of the unit is row k - kshift, head kvh of
+// the K/V tensors the kernels read (kshift = 0 and kvh = g for a full plan;
+// the row in the rank's shard buffer and head 0 for a shard plan).
 struct FwdUnit {
   int32_t mt;    // query tile
-  int32_t g;     // kv head
+  int32_t g;     // kv head (selects the query rows' heads)
   int32_t kbeg;  // absolute keys [kbeg, kend)
   int32_t kend;
   int32_t item;  // index into the plan's items
   int32_t part;  // partition
-  int32_t pad0, pad1;
+  int32_t kshift;
+  int32_t kvh;
 };
 
 // Forward pair: two forward units (slots) of one item, processed together by
@@ -46,7 +50,8 @@ struct FwdPair {
 };
 
 // Backward unit: one tile of <= 128 keys of one item, against every query
-// tile of the sample whose kmax exceeds kbeg.
+// tile of the sample whose kmax exceeds kbeg. K/V, dK and dV coordinates as
+// for FwdUnit.
 struct BwdUnit {
   int32_t b;
   int32_t g;
@@ -54,8 +59,8 @@ struct BwdUnit {
   int32_t kend;
   int32_t mt_begin;  // query tiles of sample b: [mt_begin, mt_end)
   int32_t mt_end;
-  int32_t item;
-  int32_t part;
+  int32_t kshift;
+  int32_t kvh;
 };
 
 // Offsets (bytes) of the arrays of the device section, relative to its start.
@@ -69,8 +74,11 @@ struct DevSection {
   uint64_t merge_off;     // int32[n_mtiles * Hkv + 1]
   uint64_t merge_list;    // int32[n_fwd]: fwd unit ids per (tile, kv head), ascending kbeg
   uint64_t bwd_units;     // BwdUnit[n_bwd]
-  uint64_t bwd_part_off;  // int32[P+1]
-  uint64_t dead;          // int64[2B]: [begin, end) keys of sample b whose dK/dV are zero
+  uint64_t bwd_part_off;  // int32[n_queues + 1]
+  uint64_t dead;          // int64[2 n_dead]: [begin, end) K/V rows whose dK/dV are zero
+  uint64_t base_bytes;    // end of the arrays every call uploads; the ones below only the deterministic backward
+  uint64_t bwd_rank;      // int32[n_bwd]: position of the unit's key tile among its (sample, kv head)'s, ascending
+  uint64_t bwd_det_order; // int32[n_bwd]: units by (sample, rank, kv head), the deterministic dispatch order
   uint64_t bytes;         // total
 };
 
@@ -81,6 +89,12 @@ struct PlanHeader {
   // problem scalars
   int32_t B, Hq, Hkv, d, block_q, chunk_kv, sub_chunks, P;
   int32_t G, tile_tokens;  // G = Hq / Hkv, tile_tokens = 128 / G
+  int32_t shard;           // -1: full plan; p: the items of partition p only (skv_plan_shard)
+  int32_t n_queues;        // work queues of the kernels: P for a full plan, 1 for a shard
+  int32_t kv_heads;        // heads per row of the K/V (dK/dV) buffers: Hkv, or 1 for a shard
+  int32_t n_dead;          // [begin, end) row ranges whose dK/dV are zero
+  int32_t empty_slots;     // (query tile, kv head) slots without a forward unit (possible in a shard)
+  int64_t kv_rows;         // rows of the K/V (dK/dV) buffers: Ltot, or the shard's key count
   int64_t Nq, Ltot;
   int64_t total_cost;
   int64_t n_items, n_mtiles, n_fwd, n_bwd;
@@ -90,7 +104,8 @@ struct PlanHeader {
   // host-side arrays, offsets from the start of the plan buffer
   uint64_t items_off;      // skv_item[n_items]
   uint64_t load_off;       // int64[P]
-  uint64_t dead_off;       // int64[2 * B]: [begin, end) keys of sample b whose dK/dV are zero
+  uint64_t dead_off;       // int64[2 * n_dead]: [begin, end) K/V rows whose dK/dV are zero
+  uint64_t bwd_part_host_off;  // int32[n_bwd]: partition of every backward unit
   uint64_t dev_off;        // start of the device section (256-aligned)
   DevSection dev;
   uint64_t total_bytes;
@@ -101,6 +116,9 @@ struct PlanHeader {
 struct WsLayout {
   uint64_t status;    // int32 status word at offset 0
   uint64_t counters;  // int32[2 * P] queue heads (forward, backward), right after it
+  uint64_t merge_ctr; // int32[2]: slots completed, merge tickets taken (forward with the merge in its tail)
+  uint64_t arrive;    // int32[n_mtiles * Hkv]: warps that have written their unit's partial, per slot
+  uint64_t ready;     // int32[n_mtiles * Hkv]: slot + 1 of the i-th completed slot
   uint64_t control;   // bytes of the control block
   uint64_t dev;       // device section copy
   uint64_t fwd_o;     // fp32 [n_fwd][128][d] partial outputs
@@ -108,6 +126,7 @@ struct WsLayout {
   uint64_t fwd_end;
   uint64_t bwd_delta; // fp32 [Nq][Hq]: D = rowsum(dO * O)
   uint64_t bwd_dq;    // fp32 [Nq][Hq][d]: dQ accumulator
+  uint64_t bwd_turn;  // int32 [n_mtiles * Hkv][8]: deterministic dQ, next rank to add per (slot, warp)
   uint64_t bwd_end;
 };
 
@@ -127,15 +146,21 @@ inline WsLayout ws_layout(const PlanHeader& h) {
   WsLayout w{};
   w.status = 0;
   w.counters = 16;
-  w.control = w.counters + 2 * sizeof(int32_t) * static_cast<uint64_t>(h.P);
+  const uint64_t n_slots = static_cast<uint64_t>(h.n_mtiles) * h.Hkv;
+  w.merge_ctr = w.counters + 2 * sizeof(int32_t) * static_cast<uint64_t>(h.P);
+  w.arrive = w.merge_ctr + 2 * sizeof(int32_t);
+  w.ready = w.arrive + sizeof(int32_t) * n_slots;
+  w.control = w.ready + sizeof(int32_t) * n_slots;
   w.dev = align_up(w.control, 256);
   uint64_t scratch = align_up(w.dev + h.dev.bytes, 256);
   w.fwd_o = scratch;
-  w.fwd_lse = align_up(w.fwd_o + static_cast<uint64_t>(h.n_fwd) * kTileM * h.d * 4, 256);
+  const uint64_t part_elem = (h.policy & SKV_PLAN_PARTIALS_BF16) ? 2 : 4;
+  w.fwd_lse = align_up(w.fwd_o + static_cast<uint64_t>(h.n_fwd) * kTileM * h.d * part_elem, 256);
   w.fwd_end = align_up(w.fwd_lse + static_cast<uint64_t>(h.n_fwd) * kTileM * 4, 256);
   w.bwd_delta = scratch;
   w.bwd_dq = align_up(w.bwd_delta + static_cast<uint64_t>(h.Nq) * h.Hq * 4, 256);
-  w.bwd_end = align_up(w.bwd_dq + static_cast<uint64_t>(h.Nq) * h.Hq * h.d * 4, 256);
+  w.bwd_turn = align_up(w.bwd_dq + static_cast<uint64_t>(h.Nq) * h.Hq * h.d * 4, 256);
+  w.bwd_end = align_up(w.bwd_turn + n_slots * 8 * sizeof(int32_t), 256);
   return w;
 }
 

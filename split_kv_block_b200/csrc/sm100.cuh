@@ -92,6 +92,54 @@ __device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, i
   return __all_sync(0xffffffffu, ok);
 }
 
+// ------------------------------------------------- cross-CTA flags (global)
+__device__ __forceinline__ int ld_acquire_gpu(const int32_t* p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_release_gpu(int32_t* p, int v) {
+  asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// Deterministic accumulation: the whole warp waits until the global turn
+// counter `turn` holds `want` (lane 0 polls with acquire loads), bounded by
+// `limit_ns` of %globaltimer time. On give-up it records kStatusTimeout; it
+// also gives up at once when another thread has recorded an error. The
+// verdict is the same on every lane.
+__device__ __forceinline__ bool turn_wait(const int32_t* turn, int want, int* status, uint64_t limit_ns, int lane) {
+  int ok = 1;
+  if (lane == 0) {
+    const uint64_t t0 = globaltimer_ns();
+    while (ld_acquire_gpu(turn) != want) {
+      if (*reinterpret_cast<volatile int*>(status) != 0) {
+        ok = 0;
+        break;
+      }
+      if (globaltimer_ns() - t0 > limit_ns) {
+        atomicCAS(status, 0, kStatusTimeout);
+        ok = 0;
+        break;
+      }
+      __nanosleep(64);
+    }
+  }
+  ok = __shfl_sync(0xffffffffu, ok, 0);
+  __syncwarp();
+  return ok != 0;
+}
+
+// Hands the turn on: every lane's earlier writes are made visible at GPU
+// scope before lane 0 stores `next` with release semantics.
+__device__ __forceinline__ void turn_pass(int32_t* turn, int next, int lane) {
+  __threadfence();
+  __syncwarp();
+  if (lane == 0) {
+    __threadfence();
+    st_release_gpu(turn, next);
+  }
+}
+
 // ---------------------------------------------------------------------- TMA
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
@@ -103,6 +151,57 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, u
       " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(smem_u32(dst)),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2)
       : "memory");
+}
+
+// ------------------------------------------------------------ L2 residency
+// Cache policies for L2-hinted accesses (createpolicy, sm_80+): evict_last
+// keeps lines ahead of normally-cached data, evict_first makes them the first
+// to go.
+__device__ __forceinline__ uint64_t l2_policy_evict_last() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+__device__ __forceinline__ uint64_t l2_policy_evict_first() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+__device__ __forceinline__ void st_global_v4_hint(float* dst, float4 v, uint64_t pol) {
+  asm volatile("st.global.L2::cache_hint.v4.f32 [%0], {%1, %2, %3, %4}, %5;" ::"l"(dst), "f"(v.x), "f"(v.y),
+               "f"(v.z), "f"(v.w), "l"(pol)
+               : "memory");
+}
+__device__ __forceinline__ void st_global_v4u_hint(void* dst, uint4 v, uint64_t pol) {
+  asm volatile("st.global.L2::cache_hint.v4.b32 [%0], {%1, %2, %3, %4}, %5;" ::"l"(dst), "r"(v.x), "r"(v.y),
+               "r"(v.z), "r"(v.w), "l"(pol)
+               : "memory");
+}
+__device__ __forceinline__ uint2 ld_cg_u2_hint(const void* src, uint64_t pol) {
+  uint2 v;
+  asm volatile("ld.global.cg.L2::cache_hint.v2.b32 {%0, %1}, [%2], %3;" : "=r"(v.x), "=r"(v.y) : "l"(src), "l"(pol)
+               : "memory");
+  return v;
+}
+__device__ __forceinline__ uint32_t ld_cg_u1_hint(const void* src, uint64_t pol) {
+  uint32_t v;
+  asm volatile("ld.global.cg.L2::cache_hint.b32 %0, [%1], %2;" : "=r"(v) : "l"(src), "l"(pol) : "memory");
+  return v;
+}
+// Loads through L2 only (.cg), with an L2 cache policy.
+__device__ __forceinline__ float4 ld_cg_v4_hint(const float* src, uint64_t pol) {
+  float4 v;
+  asm volatile("ld.global.cg.L2::cache_hint.v4.f32 {%0, %1, %2, %3}, [%4], %5;"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "l"(src), "l"(pol)
+               : "memory");
+  return v;
+}
+__device__ __forceinline__ float2 ld_cg_v2_hint(const float* src, uint64_t pol) {
+  float2 v;
+  asm volatile("ld.global.cg.L2::cache_hint.v2.f32 {%0, %1}, [%2], %3;" : "=f"(v.x), "=f"(v.y) : "l"(src), "l"(pol)
+               : "memory");
+  return v;
 }
 
 // -------------------------------------------------------------- async proxy

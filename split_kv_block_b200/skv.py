@@ -19,12 +19,15 @@ LIB_PATH = os.path.join(HERE, "libskv.so")
 
 SKV_PLAN_LPT = 0
 SKV_PLAN_STATIC = 1
+SKV_PLAN_PARTIALS_BF16 = 0x100  # flag: bf16 partial outputs (see include/skv.h)
 
 # Every function include/skv.h declares.
 EXPORTS = ("skv_plan_size", "skv_plan", "skv_plan_items", "skv_plan_unit_partitions", "skv_plan_stats", "skv_attn_fwd",
-           "skv_lse_merge",
-           "skv_attn_bwd", "skv_status", "skv_strerror", "skv_last_cuda_error", "skv_set_unit_timer",
-           "skv_set_timing_events", "skv_attn_fwd_noalloc", "skv_noalloc_status", "skv_wait_selftest")
+           "skv_attn_fwd_merged", "skv_lse_merge",
+           "skv_attn_bwd", "skv_attn_bwd_deterministic", "skv_status", "skv_strerror", "skv_last_cuda_error", "skv_set_unit_timer",
+           "skv_set_timing_events", "skv_attn_fwd_noalloc", "skv_noalloc_status", "skv_wait_selftest",
+           "skv_plan_shard_size", "skv_plan_shard", "skv_plan_kv_layout", "skv_attn_bwd_partial", "skv_lse_combine",
+           "skv_dq_combine")
 SKV_NOALLOC_SCRATCH_BYTES = 32 << 20
 SKV_KERNEL_FWD, SKV_KERNEL_MERGE, SKV_KERNEL_BWD = 0, 1, 2
 
@@ -44,7 +47,7 @@ class _Problem(ctypes.Structure):
 
 ITEM_DTYPE = np.dtype([("b", np.int32), ("c", np.int32), ("g", np.int32), ("sub", np.int32),
                        ("key_begin", np.int64), ("key_end", np.int64), ("cost", np.int64),
-                       ("partition", np.int32), ("order", np.int32)])
+                       ("partition", np.int32), ("order", np.int32), ("kv_row", np.int64)])
 
 _lib = None
 
@@ -63,8 +66,10 @@ def lib() -> ctypes.CDLL:
         L.skv_plan_stats.argtypes = [vp, vp, vp, vp, vp]
         L.skv_plan_unit_partitions.argtypes = [vp, vp, vp]
         L.skv_attn_fwd.argtypes = [vp, vp, vp, vp, vp, vp, sz, vp]
+        L.skv_attn_fwd_merged.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
         L.skv_lse_merge.argtypes = [vp, vp, vp, vp, vp, vp]
         L.skv_attn_bwd.argtypes = [vp] * 12 + [sz, vp]
+        L.skv_attn_bwd_deterministic.argtypes = [vp] * 12 + [sz, vp]
         L.skv_status.argtypes = [vp, vp]
         L.skv_strerror.argtypes = [ctypes.c_int]
         L.skv_strerror.restype = ctypes.c_char_p
@@ -73,6 +78,13 @@ def lib() -> ctypes.CDLL:
         L.skv_attn_fwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp]
         L.skv_noalloc_status.argtypes = [vp]
         L.skv_wait_selftest.argtypes = [vp, ctypes.c_uint64, ctypes.c_int, vp]
+        L.skv_plan_shard_size.argtypes = [vp, ctypes.c_int, ctypes.c_int, ctypes.POINTER(sz), ctypes.POINTER(sz),
+                                          ctypes.POINTER(sz), ctypes.POINTER(sz)]
+        L.skv_plan_shard.argtypes = [vp, ctypes.c_int, ctypes.c_int, vp, sz, vp]
+        L.skv_plan_kv_layout.argtypes = [vp, vp, vp, vp]
+        L.skv_attn_bwd_partial.argtypes = [vp] * 12 + [sz, vp]
+        L.skv_lse_combine.argtypes = [vp, vp, ctypes.c_int, ctypes.c_int64, ctypes.c_int, vp, vp, vp]
+        L.skv_dq_combine.argtypes = [vp, ctypes.c_int, ctypes.c_int64, vp, vp]
         for name in EXPORTS:
             if name not in ("skv_strerror",):
                 getattr(L, name).restype = ctypes.c_int
@@ -176,12 +188,39 @@ class Plan:
                                                                           ctypes.c_void_p(bp.ctypes.data)))
         return fp, bp
 
+    def kv_layout(self):
+        """(kv_rows, kv_heads, shard) of the K/V buffers the plan's kernels read."""
+        r, hh, sh = ctypes.c_int64(), ctypes.c_int32(), ctypes.c_int32()
+        _check("skv_plan_kv_layout", lib().skv_plan_kv_layout(self.ptr, ctypes.byref(r), ctypes.byref(hh),
+                                                              ctypes.byref(sh)))
+        return r.value, hh.value, sh.value
+
     def stats(self) -> dict:
         tc, nf, nb = ctypes.c_int64(), ctypes.c_int64(), ctypes.c_int64()
         im = ctypes.c_double()
         _check("skv_plan_stats", lib().skv_plan_stats(self.ptr, ctypes.byref(tc), ctypes.byref(nf), ctypes.byref(nb),
                                                       ctypes.byref(im)))
         return {"total_cost": tc.value, "n_fwd_units": nf.value, "n_bwd_units": nb.value, "imbalance": im.value}
+
+
+def skv_plan_shard_size(prob, partition: int, policy: int = SKV_PLAN_LPT) -> PlanSizes:
+    args = _ProblemArgs(prob)
+    out = [ctypes.c_size_t() for _ in range(4)]
+    _check("skv_plan_shard_size", lib().skv_plan_shard_size(args.ref(), policy, int(partition),
+                                                            *[ctypes.byref(o) for o in out]))
+    return PlanSizes(*[o.value for o in out])
+
+
+def skv_plan_shard(prob, partition: int, policy: int = SKV_PLAN_LPT) -> Plan:
+    """Plan of one context-parallel rank: the items of partition `partition`
+    of the global plan, K/V rows of its own items only (see include/skv.h)."""
+    args = _ProblemArgs(prob)
+    sizes = skv_plan_shard_size(prob, partition, policy)
+    buf = np.empty(sizes.plan_bytes, dtype=np.uint8)
+    loads = np.zeros(prob.num_partitions, dtype=np.int64)
+    _check("skv_plan_shard", lib().skv_plan_shard(args.ref(), policy, int(partition), ctypes.c_void_p(buf.ctypes.data),
+                                                  buf.nbytes, ctypes.c_void_p(loads.ctypes.data)))
+    return Plan(buf, loads, sizes, policy, prob)
 
 
 def skv_plan(prob, policy: int = SKV_PLAN_LPT, sizes: Optional[PlanSizes] = None, buf: Optional[np.ndarray] = None) -> Plan:
@@ -206,12 +245,24 @@ def skv_attn_fwd(plan: Plan, q, k, v, ws, stream=None):
                                               ws.numel(), _stream_ptr(stream)))
 
 
+def skv_attn_fwd_merged(plan: Plan, q, k, v, o, lse, ws, stream=None):
+    """Forward and LSE merge in one launch (the merge runs in the forward's tail)."""
+    _check("skv_attn_fwd_merged", lib().skv_attn_fwd_merged(plan.ptr, plan.prob_ref, _ptr(q), _ptr(k), _ptr(v),
+                                                            _ptr(o), _ptr(lse), _ptr(ws), ws.numel(),
+                                                            _stream_ptr(stream)))
+
+
 def skv_lse_merge(plan: Plan, ws, o, lse, stream=None):
     _check("skv_lse_merge", lib().skv_lse_merge(plan.ptr, plan.prob_ref, _ptr(ws), _ptr(o), _ptr(lse),
                                                 _stream_ptr(stream)))
 
 
-def skv_attn_bwd(plan: Plan, q, k, v, o, lse, do, dq, dk, dv, ws, stream=None):
+def skv_attn_bwd(plan: Plan, q, k, v, o, lse, do, dq, dk, dv, ws, stream=None, deterministic=False):
+    if deterministic:
+        _check("skv_attn_bwd_deterministic", lib().skv_attn_bwd_deterministic(
+            plan.ptr, plan.prob_ref, _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(do), _ptr(dq), _ptr(dk),
+            _ptr(dv), _ptr(ws), ws.numel(), _stream_ptr(stream)))
+        return
     _check("skv_attn_bwd", lib().skv_attn_bwd(plan.ptr, plan.prob_ref, _ptr(q), _ptr(k), _ptr(v), _ptr(o),
                                               _ptr(lse), _ptr(do), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(ws),
                                               ws.numel(), _stream_ptr(stream)))
@@ -237,6 +288,29 @@ def skv_noalloc_status(stream=None) -> int:
     return lib().skv_noalloc_status(_stream_ptr(stream))
 
 
+def skv_attn_bwd_partial(plan: Plan, q, k, v, o, lse, do, dq_f32, dk, dv, ws, stream=None):
+    """Backward with dQ written in fp32 (the plan's share of dQ)."""
+    _check("skv_attn_bwd_partial", lib().skv_attn_bwd_partial(plan.ptr, plan.prob_ref, _ptr(q), _ptr(k), _ptr(v),
+                                                              _ptr(o), _ptr(lse), _ptr(do), _ptr(dq_f32), _ptr(dk),
+                                                              _ptr(dv), _ptr(ws), ws.numel(), _stream_ptr(stream)))
+
+
+def skv_lse_combine(o_parts, lse_parts, o, lse, stream=None):
+    """o_parts bf16 [R, ..., d], lse_parts fp32 [R, ...] -> o, lse (rank partials combined in rank order)."""
+    n_parts = int(o_parts.shape[0])
+    d = int(o_parts.shape[-1])
+    n_rows = int(lse_parts.numel() // n_parts)
+    _check("skv_lse_combine", lib().skv_lse_combine(_ptr(o_parts), _ptr(lse_parts), n_parts, n_rows, d, _ptr(o),
+                                                    _ptr(lse), _stream_ptr(stream)))
+
+
+def skv_dq_combine(dq_parts, dq, stream=None):
+    """dq_parts fp32 [R, ...] -> dq bf16 (sum over ranks in rank order)."""
+    n_parts = int(dq_parts.shape[0])
+    _check("skv_dq_combine", lib().skv_dq_combine(_ptr(dq_parts), n_parts, int(dq_parts.numel() // n_parts), _ptr(dq),
+                                                  _stream_ptr(stream)))
+
+
 def skv_status(ws, stream=None) -> int:
     return lib().skv_status(_ptr(ws), _stream_ptr(stream))
 
@@ -254,18 +328,22 @@ def skv_set_timing_events(kernel: int, start=None, end=None):
 
 # ------------------------------------------------------------- conveniences
 def check_inputs(plan: Plan, q, k, v, do=None):
+    """Shapes, dtype and device of the call's tensors: queries in the problem's
+    layout, K/V in the plan's (the packed context, or a rank's shard rows)."""
     import torch
     p = plan.problem
-    Nq, L = p.num_tokens_q, p.num_tokens_kv
-    for name, t, shape in (("q", q, (Nq, p.num_q_heads, p.head_dim)), ("k", k, (L, p.num_kv_heads, p.head_dim)),
-                           ("v", v, (L, p.num_kv_heads, p.head_dim))) + ((("do", do, (Nq, p.num_q_heads, p.head_dim)),)
-                                                                          if do is not None else ()):
+    Nq = p.num_tokens_q
+    rows, heads, _ = plan.kv_layout()
+    for name, t, shape in (("q", q, (Nq, p.num_q_heads, p.head_dim)), ("k", k, (rows, heads, p.head_dim)),
+                           ("v", v, (rows, heads, p.head_dim))) + ((("do", do, (Nq, p.num_q_heads, p.head_dim)),)
+                                                                    if do is not None else ()):
         if tuple(t.shape) != shape or t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous():
             raise ValueError(f"{name}: expected contiguous cuda bf16 {shape}, got {tuple(t.shape)} {t.dtype} {t.device}")
 
 
-def forward(plan: Plan, q, k, v, ws=None, stream=None):
-    """Split-KV forward + LSE merge. Returns (o bf16 [Nq,Hq,d], lse fp32 [Nq,Hq])."""
+def forward(plan: Plan, q, k, v, ws=None, stream=None, fused=True):
+    """Split-KV forward + LSE merge: one launch (fused, the default) or the
+    forward and merge calls in turn. Returns (o bf16 [Nq,Hq,d], lse fp32 [Nq,Hq])."""
     import torch
     check_inputs(plan, q, k, v)
     if ws is None:
@@ -273,13 +351,17 @@ def forward(plan: Plan, q, k, v, ws=None, stream=None):
     p = plan.problem
     o = torch.empty(p.num_tokens_q, p.num_q_heads, p.head_dim, dtype=torch.bfloat16, device=q.device)
     lse = torch.empty(p.num_tokens_q, p.num_q_heads, dtype=torch.float32, device=q.device)
-    skv_attn_fwd(plan, q, k, v, ws, stream)
-    skv_lse_merge(plan, ws, o, lse, stream)
+    if fused:
+        skv_attn_fwd_merged(plan, q, k, v, o, lse, ws, stream)
+    else:
+        skv_attn_fwd(plan, q, k, v, ws, stream)
+        skv_lse_merge(plan, ws, o, lse, stream)
     return o, lse
 
 
-def backward(plan: Plan, q, k, v, o, lse, do, ws=None, stream=None):
-    """Split-KV backward. Returns (dq, dk, dv) bf16."""
+def backward(plan: Plan, q, k, v, o, lse, do, ws=None, stream=None, deterministic=False):
+    """Split-KV backward. Returns (dq, dk, dv) bf16. deterministic: dQ summed
+    over key tiles in a fixed order (bitwise reproducible, slower)."""
     import torch
     check_inputs(plan, q, k, v, do)
     if ws is None:
@@ -287,5 +369,5 @@ def backward(plan: Plan, q, k, v, o, lse, do, ws=None, stream=None):
     dq = torch.empty_like(q)
     dk = torch.empty_like(k)
     dv = torch.empty_like(v)
-    skv_attn_bwd(plan, q, k, v, o, lse, do, dq, dk, dv, ws, stream)
+    skv_attn_bwd(plan, q, k, v, o, lse, do, dq, dk, dv, ws, stream, deterministic)
     return dq, dk, dv

@@ -116,3 +116,19 @@ def test_clock_summary_names_every_throttle_reason_seen():
 def test_clock_summary_without_samples():
     out = bench.ClockSampler(0).summary()
     assert out["sm_mhz"] is None and out["reasons"] == ["unsampled"]
+
+
+def test_merge_bytes_by_hand():
+    """Partials read (fp32 row of d plus its LSE, 128 rows per forward unit),
+    merged O (bf16) and LSE (fp32) written once."""
+    prob = synth.small_problem([10, 4], [[5, 9], [3]], block_q=2, hq=4, hkv=2, d=8)
+    rows = 3 * 2 * 4
+    assert bench.merge_bytes(prob, 5) == 5 * 128 * 9 * 4 + rows * 8 * 2 + rows * 4
+
+
+def test_gpus_flag_must_match_the_ranks():
+    bench.check_world(1, 1)
+    bench.check_world(4, 4)
+    for gpus, world in ((2, 1), (1, 2), (0, 1)):
+        with pytest.raises(SystemExit):
+            bench.check_world(gpus, world)

@@ -34,11 +34,11 @@ def _rel_fro(a, b):
     return float((a - b).norm() / b.norm().clamp_min(1e-30))
 
 
-def run_gpu(prob, q, k, v, do=None, policy=skv.SKV_PLAN_LPT):
+def run_gpu(prob, q, k, v, do=None, policy=skv.SKV_PLAN_LPT, fused=True):
     plan = skv.skv_plan(prob, policy)
     qd, kd, vd, dod = _dev(q, k, v, do)
     ws = skv.alloc_workspace(plan)
-    o, lse = skv.forward(plan, qd, kd, vd, ws)
+    o, lse = skv.forward(plan, qd, kd, vd, ws, fused=fused)
     assert skv.skv_status(ws) == 0
     grads = None
     if do is not None:
@@ -80,9 +80,9 @@ def check_backward(prob, q, k, v, do, grads, groups=None):
     return errs
 
 
-def _case(prob, seed=0, backward=True, policy=skv.SKV_PLAN_LPT, groups=None):
+def _case(prob, seed=0, backward=True, policy=skv.SKV_PLAN_LPT, groups=None, fused=True):
     q, k, v, do = synth.make_tensors(prob, seed=seed, backward=backward)
-    o, lse, grads, plan = run_gpu(prob, q, k, v, do, policy)
+    o, lse, grads, plan = run_gpu(prob, q, k, v, do, policy, fused)
     check_forward(prob, q, k, v, o, lse, groups)
     if backward:
         check_backward(prob, q, k, v, do, grads, groups)
@@ -105,7 +105,7 @@ def test_random_ragged_problems(d):
     for i in range(6):
         prob = synth.random_small_problem(rng, max_len=900, max_anchors=7, d=d,
                                           heads=((4, 1), (8, 2), (4, 4), (8, 1), (16, 2), (2, 2)))
-        _case(prob, seed=i, policy=skv.SKV_PLAN_LPT if i % 3 else skv.SKV_PLAN_STATIC)
+        _case(prob, seed=i, policy=skv.SKV_PLAN_LPT if i % 3 else skv.SKV_PLAN_STATIC, fused=i % 2 == 0)
 
 
 def test_edge_anchors():
@@ -163,18 +163,29 @@ def test_ctx128k_full_size_one_group():
     _case(prob, groups=(3,))
 
 
+def test_ctx128k_full_size_chunk_items_one_group():
+    """The 128K Beta(5,1) workload at full size with whole-chunk items
+    (sub_chunks = 1, 4096-key items: the plan the benchmark times); oracle on
+    one kv-head group."""
+    prob = synth.make_problem(synth.WORKLOADS["ctx128k"], seed=0, sub_chunks=1)
+    assert prob.sub_chunks == 1
+    _case(prob, groups=(6,))
+
+
 def test_batch8_full_size_one_sample_one_group():
     """The batched workload (8 samples, contexts 8K-256K) at full size with
-    fresh anchors; oracle on one sample and one kv-head group."""
+    fresh anchors; oracle on the longest sample and on a mid-sized one, one
+    kv-head group each."""
     w = synth.WORKLOADS["batch8_logu"]
     prob = synth.redraw_anchors(synth.make_problem(w, seed=0), w, seed=11)
     q, k, v, do = synth.make_tensors(prob, seed=0, backward=True)
     o, lse, grads, plan = run_gpu(prob, q, k, v, do)
     lens = np.diff(prob.ctx_offsets)
-    b = int(np.argsort(lens)[len(lens) // 2])  # a mid-sized sample
-    sub, qs, ks, vs, dos, os_, ls, gs = _one_sample(prob, b, q, k, v, do, o, lse, grads)
-    check_forward(sub, qs, ks, vs, os_, ls, groups=(6,))
-    check_backward(sub, qs, ks, vs, dos, gs, groups=(6,))
+    order = np.argsort(lens)
+    for b, g in ((int(order[-1]), 2), (int(order[len(lens) // 2]), 6)):  # the longest, a mid-sized sample
+        sub, qs, ks, vs, dos, os_, ls, gs = _one_sample(prob, b, q, k, v, do, o, lse, grads)
+        check_forward(sub, qs, ks, vs, os_, ls, groups=(g,))
+        check_backward(sub, qs, ks, vs, dos, gs, groups=(g,))
 
 
 def test_dead_key_gradients_are_written_zero():
@@ -195,3 +206,42 @@ def test_dead_key_gradients_are_written_zero():
     torch.cuda.synchronize()
     check_backward(prob, q, k, v, do, (dq.cpu(), dk.cpu(), dv.cpu()))
     assert not torch.isnan(dk).any() and not torch.isnan(dv).any() and not torch.isnan(dq).any()
+
+
+@pytest.mark.parametrize("name", ["tiny_4k", "ctx32k_fwd"])
+def test_merge_in_the_forward_tail_equals_the_merge_kernel(name):
+    """skv_attn_fwd_merged (the merge in the forward kernel's tail) against
+    skv_attn_fwd + skv_lse_merge: the same partials merged by the same
+    arithmetic in the same order, so o and lse are bitwise equal; both
+    within tolerance of the oracle on the tiny workload."""
+    prob = synth.make_problem(synth.WORKLOADS[name], seed=4)
+    q, k, v, _ = synth.make_tensors(prob, seed=4, backward=False)
+    plan = skv.skv_plan(prob)
+    qd, kd, vd = _dev(q, k, v)
+    ws = skv.alloc_workspace(plan)
+    o1, l1 = skv.forward(plan, qd, kd, vd, ws, fused=True)
+    assert skv.skv_status(ws) == 0
+    o2, l2 = skv.forward(plan, qd, kd, vd, ws, fused=False)
+    assert skv.skv_status(ws) == 0
+    torch.cuda.synchronize()
+    assert torch.equal(o1.view(torch.int16), o2.view(torch.int16))
+    assert torch.equal(l1.view(torch.int32), l2.view(torch.int32))
+    if name == "tiny_4k":
+        check_forward(prob, q, k, v, o1.cpu(), l1.cpu())
+
+
+@pytest.mark.parametrize("fused", [False, True])
+def test_bf16_partials(fused):
+    """Plans with SKV_PLAN_PARTIALS_BF16: the same forward tolerances against
+    the oracle (the partial outputs are convex combinations of bf16 values,
+    rounded once more), through the merge kernel and through the merge in
+    the forward's tail; head_dim 64 and 128, ragged tiles, the 32K workload."""
+    flag = skv.SKV_PLAN_PARTIALS_BF16
+    cases = [(synth.make_problem(synth.WORKLOADS["tiny_4k"], seed=3), None),
+             (synth.small_problem([1001, 777, 1500], [[1000, 3, 555], [777], [1, 1499, 700, 64, 1200]],
+                                  block_q=16, chunk_kv=320, num_partitions=4, hq=8, hkv=2, d=128), None),
+             (synth.make_problem(synth.WORKLOADS["ctx32k_fwd"], seed=1), (2, 7))]
+    for prob, groups in cases:
+        q, k, v, _ = synth.make_tensors(prob, seed=3, backward=False)
+        o, lse, _, _ = run_gpu(prob, q, k, v, None, skv.SKV_PLAN_LPT | flag, fused)
+        check_forward(prob, q, k, v, o, lse, groups)

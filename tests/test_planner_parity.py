@@ -214,11 +214,33 @@ def test_plan_for_another_problem_is_refused_before_any_launch():
     for other in others:
         pr = skv._ProblemArgs(other).ref()
         assert L.skv_attn_fwd(plan.ptr, pr, f[0], f[1], f[2], f[3], 1 << 30, None) == 5
+        assert L.skv_attn_fwd_merged(plan.ptr, pr, f[0], f[1], f[2], f[4], f[5], f[3], 1 << 30, None) == 5
         assert L.skv_lse_merge(plan.ptr, pr, f[3], f[4], f[5], None) == 5
         assert L.skv_attn_bwd(plan.ptr, pr, *f[:7], f[7], f[0], f[1], 1 << 30, None) == 5
+        assert L.skv_attn_bwd_deterministic(plan.ptr, pr, *f[:7], f[7], f[0], f[1], 1 << 30, None) == 5
         assert L.skv_attn_fwd_noalloc(plan.ptr, pr, f[0], f[1], f[2], f[3], f[4], None) == 5
     # NULL problem: invalid argument; a buffer that is not a plan: SKV_EPLAN
     assert L.skv_attn_fwd(plan.ptr, None, f[0], f[1], f[2], f[3], 1 << 30, None) == 1
     junk = np.zeros(plan.buf.nbytes, dtype=np.uint8)
     assert L.skv_attn_fwd(ctypes.c_void_p(junk.ctypes.data), plan.prob_ref, f[0], f[1], f[2], f[3], 1 << 30,
                           None) == 5
+
+
+def test_bf16_partials_flag_changes_only_the_partial_workspace():
+    """SKV_PLAN_PARTIALS_BF16 keeps items, placement and work lists; the
+    forward workspace shrinks by half the partial outputs' bytes; unknown
+    policy bits are refused."""
+    prob = synth.make_problem(synth.WORKLOADS["ctx32k"], seed=0)
+    a = skv.skv_plan(prob, skv.SKV_PLAN_LPT)
+    b = skv.skv_plan(prob, skv.SKV_PLAN_LPT | skv.SKV_PLAN_PARTIALS_BF16)
+    assert np.array_equal(a.items(), b.items())
+    assert a.stats() == b.stats()
+    n_fwd = a.stats()["n_fwd_units"]
+    saved = a.sizes.ws_fwd_bytes - b.sizes.ws_fwd_bytes
+    assert n_fwd * 128 * 128 * 2 - 256 <= saved <= n_fwd * 128 * 128 * 2 + 256
+    assert a.sizes.ws_bwd_bytes == b.sizes.ws_bwd_bytes
+    st = skv.skv_plan(prob, skv.SKV_PLAN_STATIC | skv.SKV_PLAN_PARTIALS_BF16)
+    assert np.array_equal(st.items(), skv.skv_plan(prob, skv.SKV_PLAN_STATIC).items())
+    for bad in (2, 0x200, 0x101 | 0x400):
+        with pytest.raises(skv.SkvError):
+            skv.skv_plan_size(prob, bad)

@@ -10,6 +10,7 @@ import numpy as np
 import pytest
 import torch
 
+from oracle import attention as A
 from split_kv_block_b200 import skv, synth
 
 pytestmark = pytest.mark.gpu
@@ -62,6 +63,19 @@ def test_noalloc_matches_workspace_path_two_calls():
     ref = _reference(plan, q, k, v)
     _close(_noalloc(plan, q, k, v), ref)
     _close(_noalloc(plan, q, k, v), ref)
+
+
+def test_noalloc_matches_the_oracle_and_reports_ok():
+    """The tiny workload straight against the fp64 oracle, and the status
+    word of the call read back through skv_noalloc_status (no allocation)."""
+    prob = synth.make_problem(synth.WORKLOADS["tiny_4k"], seed=2)
+    plan = skv.skv_plan(prob)
+    qc, kc, vc, _ = synth.make_tensors(prob, seed=2, backward=False)
+    o, lse = _noalloc(plan, qc.cuda(), kc.cuda(), vc.cuda())
+    assert skv.skv_noalloc_status() == 0
+    O_ref, L_ref = A.attention_forward(prob, qc, kc, vc)
+    assert float((o.cpu().double() - O_ref).abs().max()) <= O_TOL
+    assert float((lse.cpu().double() - L_ref).abs().max()) <= LSE_TOL
 
 
 def test_noalloc_rejects_problems_beyond_the_scratch():
