@@ -8,6 +8,10 @@ anchor, and cross-attend to the sample's context under a block-sparse mask.
 Readings taken where the pages give no formula:
   * the block of anchor a attends to context keys [0, a) of its own sample
     (exclusive end, 1 <= a <= L); no attention among draft tokens;
+  * a problem may add a block-sparse mask over the context: a byte per
+    (anchor, block of 128 keys of the sample); the block of anchor j then
+    attends only the keys of [0, a_j) whose block is set. A block left with
+    no key gets O = 0, LSE = -inf and contributes no gradient;
   * softmax scale 1/sqrt(d); LSE is the natural log-sum-exp of the scaled
     scores;
   * grouped heads: q-head h reads kv-head h // (Hq / Hkv).
@@ -46,6 +50,23 @@ def _blocks(prob):
             yield b, j, slice(j * S, (j + 1) * S), k0, int(prob.anchors[j])
 
 
+MASK_BLOCK = 128
+
+
+def allowed_keys(prob, j: int, a: int, lo: int = 0, hi=None) -> torch.Tensor:
+    """Sample-relative keys the block of anchor j attends, within [lo, hi):
+    the prefix [0, a) and, when the problem carries a block-sparse mask, only
+    the keys kk whose block kk // 128 is set in row j of the mask (reading of
+    the pages' "block-sparse mask over the context")."""
+    hi = a if hi is None else min(hi, a)
+    kk = torch.arange(max(lo, 0), max(hi, lo), dtype=torch.long)
+    m = getattr(prob, "key_block_mask", None)
+    if m is not None and kk.numel():
+        keep = torch.from_numpy(np.asarray(m[j])[kk.numpy() // MASK_BLOCK] != 0)
+        kk = kk[keep]
+    return kk
+
+
 def attention_forward(prob, q, k, v) -> Tuple[torch.Tensor, torch.Tensor]:
     """Unsplit masked attention (the definition).
 
@@ -62,10 +83,14 @@ def attention_forward(prob, q, k, v) -> Tuple[torch.Tensor, torch.Tensor]:
     O = torch.zeros(Nq, Hq, d, dtype=F64)
     LSE = torch.zeros(Nq, Hq, dtype=F64)
     for b, j, rows, k0, a in _blocks(prob):
+        keys = k0 + allowed_keys(prob, j, a)
+        if keys.numel() == 0:          # a block that may see no key: O = 0, LSE = -inf
+            LSE[rows] = -math.inf
+            continue
         for h in range(Hq):
             g = h // G
-            Kb, Vb = k[k0:k0 + a, g], v[k0:k0 + a, g]
-            s = (q[rows, h] @ Kb.T) * scale                  # [S, a]
+            Kb, Vb = k[keys, g], v[keys, g]
+            s = (q[rows, h] @ Kb.T) * scale                  # [S, n_keys]
             m = s.max(dim=1, keepdim=True).values
             e = torch.exp(s - m)
             l = e.sum(dim=1, keepdim=True)
@@ -95,16 +120,19 @@ def attention_backward(prob, q, k, v, o, lse, do):
     dk = torch.zeros_like(k)
     dv = torch.zeros_like(v)
     for b, j, rows, k0, a in _blocks(prob):
+        keys = k0 + allowed_keys(prob, j, a)
+        if keys.numel() == 0:
+            continue
         for h in range(Hq):
             g = h // G
-            Kb, Vb = k[k0:k0 + a, g], v[k0:k0 + a, g]
+            Kb, Vb = k[keys, g], v[keys, g]
             s = (q[rows, h] @ Kb.T) * scale
             P = torch.exp(s - lse[rows, h][:, None])
             dP = do[rows, h] @ Vb.T
             dS = P * (dP - D[rows, h][:, None])
             dq[rows, h] += (dS @ Kb) * scale
-            dk[k0:k0 + a, g] += (dS.T @ q[rows, h]) * scale
-            dv[k0:k0 + a, g] += P.T @ do[rows, h]
+            dk[keys, g] += (dS.T @ q[rows, h]) * scale
+            dv[keys, g] += P.T @ do[rows, h]
     return dq, dk, dv
 
 
@@ -125,17 +153,17 @@ def chunk_partial(prob, q, k, v, b: int, key_begin: int, key_end: int):
     for bb, j, rows, k0, a in _blocks(prob):
         if bb != b:
             continue
-        lo, hi = key_begin, min(key_end, k0 + a)
-        if hi <= lo:
+        keys = k0 + allowed_keys(prob, j, a, key_begin - k0, key_end - k0)
+        if keys.numel() == 0:
             continue
         for h in range(Hq):
             g = h // G
-            s = (q[rows, h] @ k[lo:hi, g].T) * scale
+            s = (q[rows, h] @ k[keys, g].T) * scale
             m = s.max(dim=1, keepdim=True).values
             e = torch.exp(s - m)
             l = e.sum(dim=1, keepdim=True)
             LSE[rows, h] = (m + torch.log(l)).squeeze(1)
-            O[rows, h] = (e / l) @ v[lo:hi, g]
+            O[rows, h] = (e / l) @ v[keys, g]
     return O, LSE
 
 
@@ -206,17 +234,17 @@ def chunked_backward(prob, q, k, v, o, lse, do, ranges=None):
         for bb, j, rows, k0, a in _blocks(prob):
             if bb != b:
                 continue
-            lo, hi = lo_r, min(hi_r, k0 + a)
-            if hi <= lo:
+            keys = k0 + allowed_keys(prob, j, a, lo_r - k0, hi_r - k0)
+            if keys.numel() == 0:
                 continue
             for h in range(Hq):
                 g = h // G
-                Kc, Vc = k[lo:hi, g], v[lo:hi, g]
+                Kc, Vc = k[keys, g], v[keys, g]
                 P = torch.exp((q[rows, h] @ Kc.T) * scale - lse[rows, h][:, None])
                 dS = P * (do[rows, h] @ Vc.T - D[rows, h][:, None])
                 dq_c[rows, h] += (dS @ Kc) * scale
-                dk[lo:hi, g] += (dS.T @ q[rows, h]) * scale
-                dv[lo:hi, g] += P.T @ do[rows, h]
+                dk[keys, g] += (dS.T @ q[rows, h]) * scale
+                dv[keys, g] += P.T @ do[rows, h]
         dq_parts.append(dq_c)
     dq = torch.zeros_like(q)
     for p in dq_parts:
@@ -227,5 +255,10 @@ def chunked_backward(prob, q, k, v, o, lse, do, ranges=None):
 # ------------------------------------------------------------ small helpers
 def flops_fwd(prob) -> int:
     """Unmasked forward FLOPs: 2 contractions of d per (query, key) pair and
-    q-head: 4 * d * block_q * Hq * sum(a)."""
-    return 4 * prob.head_dim * prob.block_q * prob.num_q_heads * int(np.sum(prob.anchors))
+    q-head: 4 * d * block_q * Hq * (sum over anchors of their attended keys;
+    sum(a) without a block mask)."""
+    if getattr(prob, "key_block_mask", None) is None:
+        n = int(np.sum(prob.anchors))
+    else:
+        n = sum(int(allowed_keys(prob, j, a).numel()) for _b, j, _r, _k0, a in _blocks(prob))
+    return 4 * prob.head_dim * prob.block_q * prob.num_q_heads * n

@@ -47,14 +47,21 @@ class Item:
 
 def item_cost(prob, b: int, key_begin: int, key_end: int) -> int:
     """G * sum over the sample's anchors of block_q * |[lo, hi) ∩ [0, a)|,
-    written as a plain loop (relative key coordinates)."""
+    written as a plain loop (relative key coordinates). With a block-sparse
+    mask only the keys whose 128-key block is set for the anchor count."""
     G = prob.num_q_heads // prob.num_kv_heads
     k0 = int(prob.ctx_offsets[b])
     lo, hi = key_begin - k0, key_end - k0
+    mask = getattr(prob, "key_block_mask", None)
     pairs = 0
     for j in range(int(prob.anchor_offsets[b]), int(prob.anchor_offsets[b + 1])):
         a = int(prob.anchors[j])
-        pairs += prob.block_q * max(0, min(hi, a) - lo)
+        if mask is None:
+            pairs += prob.block_q * max(0, min(hi, a) - lo)
+        else:
+            for kk in range(lo, min(hi, a)):
+                if mask[j][kk // 128]:
+                    pairs += prob.block_q
     return G * pairs
 
 

@@ -82,6 +82,9 @@ class Problem:
     num_q_heads: int
     num_kv_heads: int
     head_dim: int
+    # optional block-sparse mask: uint8 [A_total, mask_stride]; entry (j, kb) != 0 lets the block of anchor
+    # j see keys [128 kb, 128 kb + 128) of its sample (on top of the prefix [0, a_j)); None = prefix only
+    key_block_mask: Optional[np.ndarray] = None
 
     @property
     def num_samples(self) -> int:
@@ -179,3 +182,26 @@ def random_small_problem(rng: np.random.Generator, *, max_samples=3, max_len=700
     sub = int(rng.choice([1, 2, 4])) if chunk % 4 == 0 else 1
     return small_problem(lens, anchors, block_q=int(rng.choice([1, 4, 16])), chunk_kv=chunk, sub_chunks=sub,
                          num_partitions=int(rng.integers(1, 9)), hq=hq, hkv=hkv, d=d)
+
+
+MASK_BLOCK = 128  # keys per block of the block-sparse mask
+
+
+def block_mask_sink_window_random(p: Problem, seed: int, sink: int = 2, window: int = 4, density: float = 0.25,
+                                  ) -> np.ndarray:
+    """A block-sparse mask over the context: for every anchor, the first `sink`
+    key blocks of its sample, the `window` blocks ending at the one that holds
+    its anchor, and each other block with probability `density` (numpy
+    default_rng(seed)). Returns uint8 [A_total, stride], stride = the largest
+    sample's block count."""
+    rng = np.random.default_rng(seed)
+    lens = np.diff(p.ctx_offsets)
+    stride = int((lens.max() + MASK_BLOCK - 1) // MASK_BLOCK)
+    A = int(p.anchor_offsets[-1])
+    m = (rng.random((A, stride)) < density).astype(np.uint8)
+    for b in range(p.num_samples):
+        for j in range(int(p.anchor_offsets[b]), int(p.anchor_offsets[b + 1])):
+            last = (int(p.anchors[j]) - 1) // MASK_BLOCK
+            m[j, :sink] = 1
+            m[j, max(0, last - window + 1):last + 1] = 1
+    return m

@@ -41,6 +41,9 @@ def _sdpa_reference(prob, q, k, v, requires_grad=False):
         vb = v[k0:k1].repeat_interleave(G, dim=1).permute(1, 0, 2)
         a_tok = torch.tensor(np.repeat(prob.anchors[j0:j1], S))
         mask = torch.arange(k1 - k0)[None, :] < a_tok[:, None]    # [n, L]
+        if prob.key_block_mask is not None:                        # and the key's block set for the anchor
+            rows = torch.from_numpy(np.repeat(prob.key_block_mask[j0:j1], S, axis=0).astype(bool))
+            mask = mask & rows[:, torch.arange(k1 - k0) // 128]
         ob = F.scaled_dot_product_attention(qb, kb, vb, attn_mask=mask)
         outs.append(ob.permute(1, 0, 2))
     return torch.cat(outs, 0), (q, k, v)
@@ -196,3 +199,97 @@ def test_flops_fwd_hand_instance_and_mask_count():
                         if kk < int(prob.anchors[j]):
                             triples += prob.num_q_heads
         assert A.flops_fwd(prob) == 4 * prob.head_dim * triples
+
+
+
+def _masked(prob, seed, density=0.4):
+    """The problem with a random block mask that leaves every anchor at least
+    its first block (so no row of the library reference is empty)."""
+    rng = np.random.default_rng(seed)
+    lens = np.diff(prob.ctx_offsets)
+    stride = int((lens.max() + 127) // 128)
+    m = (rng.random((int(prob.anchor_offsets[-1]), stride)) < density).astype(np.uint8)
+    m[:, 0] = 1
+    return prob.replace(key_block_mask=m)
+
+
+def _mask_probs():
+    yield synth.small_problem([700, 390], [[650, 129, 300], [390, 200]], block_q=2, hq=4, hkv=2, d=16)
+    yield synth.small_problem([1000], [[999, 513, 256, 40]], block_q=3, hq=8, hkv=2, d=16)
+
+
+@pytest.mark.parametrize("pi", range(2))
+def test_block_mask_forward_backward_match_library_sdpa_and_autograd(pi):
+    """Block-sparse mask: forward against torch SDPA with the explicit boolean
+    mask (prefix AND block bit), gradients against autograd through it."""
+    prob = _masked(list(_mask_probs())[pi], seed=pi)
+    q, k, v, do = _tensors(prob, seed=pi)
+    O, L = A.attention_forward(prob, q, k, v)
+    ref, (qq, kk, vv) = _sdpa_reference(prob, q, k, v, requires_grad=True)
+    assert torch.allclose(O, ref.detach(), atol=1e-12, rtol=0)
+    (ref * do.to(F64)).sum().backward()
+    gq, gk, gv = A.attention_backward(prob, q, k, v, O, L, do)
+    assert torch.allclose(gq, qq.grad, atol=1e-11, rtol=0)
+    assert torch.allclose(gk, kk.grad, atol=1e-11, rtol=0)
+    assert torch.allclose(gv, vv.grad, atol=1e-11, rtol=0)
+
+
+def test_block_mask_of_ones_is_the_prefix_mask_and_block_zero_caps_the_anchor():
+    """All blocks set: the prefix mask exactly. Only block 0 set: the prefix
+    mask with every anchor capped at 128 (a closed form of the reading)."""
+    prob = list(_mask_probs())[0]
+    q, k, v, do = _tensors(prob, seed=3)
+    stride = 6
+    ones = prob.replace(key_block_mask=np.ones((int(prob.anchor_offsets[-1]), stride), dtype=np.uint8))
+    for a_, b_ in zip(A.attention_forward(prob, q, k, v), A.attention_forward(ones, q, k, v)):
+        assert torch.equal(a_, b_)
+    first = np.zeros((int(prob.anchor_offsets[-1]), stride), dtype=np.uint8)
+    first[:, 0] = 1
+    capped = prob.replace(anchors=np.minimum(prob.anchors, 128))
+    O1, L1 = A.attention_forward(prob.replace(key_block_mask=first), q, k, v)
+    O2, L2 = A.attention_forward(capped, q, k, v)
+    assert torch.allclose(O1, O2, atol=1e-14) and torch.allclose(L1, L2, atol=1e-14)
+
+
+@pytest.mark.parametrize("chunk,sub", [(128, 1), (256, 2), (384, 3), (1024, 1)])
+def test_block_mask_split_equals_unsplit(chunk, sub):
+    prob = _masked(synth.small_problem([700, 390], [[650, 129, 300], [390, 200]], block_q=2, hq=4, hkv=2, d=16,
+                                       chunk_kv=chunk, sub_chunks=sub), seed=11)
+    q, k, v, do = _tensors(prob, seed=6)
+    O, L = A.attention_forward(prob, q, k, v)
+    Oc, Lc = A.chunked_forward(prob, q, k, v)
+    assert torch.allclose(O, Oc, atol=1e-12, rtol=0) and torch.allclose(L, Lc, atol=1e-12, rtol=0)
+    for a_, b_ in zip(A.attention_backward(prob, q, k, v, O, L, do), A.chunked_backward(prob, q, k, v, Oc, Lc, do)):
+        assert torch.allclose(a_, b_, atol=1e-12, rtol=0)
+
+
+def test_block_mask_empty_row():
+    """An anchor whose blocks are all cleared sees no key: O = 0, LSE = -inf,
+    no gradient to any key; the other blocks are as without it."""
+    prob = synth.small_problem([400], [[390, 200]], block_q=2, hq=4, hkv=2, d=16)
+    m = np.ones((2, 4), dtype=np.uint8)
+    m[0, :] = 0
+    mp = prob.replace(key_block_mask=m)
+    q, k, v, do = _tensors(prob, seed=8)
+    O, L = A.attention_forward(mp, q, k, v)
+    assert torch.all(O[0:2] == 0) and torch.all(torch.isneginf(L[0:2]))
+    alone = prob.replace(anchors=np.array([200]), anchor_offsets=np.array([0, 1], dtype=np.int32))
+    O1, L1 = A.attention_forward(alone, q[2:4], k, v)
+    assert torch.allclose(O[2:4], O1, atol=1e-14) and torch.allclose(L[2:4], L1, atol=1e-14)
+    gq, gk, gv = A.attention_backward(mp, q, k, v, O, L, do)
+    assert torch.all(gq[0:2] == 0)
+    g1 = A.attention_backward(alone, q[2:4], k, v, O1, L1, do[2:4])
+    assert torch.allclose(gk, g1[1], atol=1e-13) and torch.allclose(gv, g1[2], atol=1e-13)
+
+
+def test_flops_fwd_with_a_block_mask_brute_force():
+    prob = _masked(synth.small_problem([700, 390], [[650, 129, 300], [390, 200]], block_q=2, hq=4, hkv=2, d=16),
+                   seed=5)
+    m = prob.key_block_mask
+    triples = 0
+    for b in range(prob.num_samples):
+        for j in range(int(prob.anchor_offsets[b]), int(prob.anchor_offsets[b + 1])):
+            for kk in range(int(prob.anchors[j])):
+                if m[j, kk // 128]:
+                    triples += prob.block_q * prob.num_q_heads
+    assert A.flops_fwd(prob) == 4 * prob.head_dim * triples

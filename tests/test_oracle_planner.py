@@ -23,6 +23,9 @@ def _mask_count(prob, b, lo, hi):
     j0, j1 = int(prob.anchor_offsets[b]), int(prob.anchor_offsets[b + 1])
     a_tok = np.repeat(prob.anchors[j0:j1], S)
     mask = np.arange(k1 - k0)[None, :] < a_tok[:, None]
+    if prob.key_block_mask is not None:
+        rows = np.repeat(prob.key_block_mask[j0:j1], S, axis=0).astype(bool)
+        mask = mask & rows[:, np.arange(k1 - k0) // 128]
     G = prob.num_q_heads // prob.num_kv_heads
     return G * int(mask[:, lo - k0:hi - k0].sum())
 
@@ -162,3 +165,16 @@ def test_golden_tiny_plan_is_current():
     assert [[it.b, it.c, it.g, it.sub, it.key_begin, it.key_end, it.cost, it.partition] for it in items] == g["lpt_items"]
     assert loads == g["lpt_loads"]
     assert PL.static_plan(prob)[1] == g["static_loads"]
+
+
+
+def test_item_costs_with_a_block_mask_match_mask_count():
+    rng = np.random.default_rng(9)
+    for _ in range(15):
+        prob = synth.random_small_problem(rng)
+        lens = np.diff(prob.ctx_offsets)
+        stride = int((lens.max() + 127) // 128)
+        mask = (rng.random((int(prob.anchor_offsets[-1]), stride)) < 0.5).astype(np.uint8)
+        prob = prob.replace(key_block_mask=mask)
+        for it in PL.lpt_items(prob):
+            assert it.cost == _mask_count(prob, it.b, it.key_begin, it.key_end)
