@@ -53,18 +53,26 @@ def _blocks(prob):
 MASK_BLOCK = 128
 
 
-def allowed_keys(prob, j: int, a: int, lo: int = 0, hi=None) -> torch.Tensor:
-    """Sample-relative keys the block of anchor j attends, within [lo, hi):
-    the prefix [0, a) and, when the problem carries a block-sparse mask, only
-    the keys kk whose block kk // 128 is set in row j of the mask (reading of
-    the pages' "block-sparse mask over the context")."""
+def allowed_keys(prob, j: int, a: int, lo: int = 0, hi=None, k0: int = 0):
+    """Keys (absolute: sample start k0 added) the block of anchor j attends,
+    within the sample-relative range [lo, hi): the prefix [0, a) and, when the
+    problem carries a block-sparse mask, only the keys kk whose block kk // 128
+    is set in row j of the mask (reading of the pages' "block-sparse mask over
+    the context"). A slice without a mask, an index tensor with one."""
     hi = a if hi is None else min(hi, a)
-    kk = torch.arange(max(lo, 0), max(hi, lo), dtype=torch.long)
+    lo = max(lo, 0)
     m = getattr(prob, "key_block_mask", None)
-    if m is not None and kk.numel():
+    if m is None:
+        return slice(k0 + lo, k0 + max(hi, lo))
+    kk = torch.arange(lo, max(hi, lo), dtype=torch.long)
+    if kk.numel():
         keep = torch.from_numpy(np.asarray(m[j])[kk.numpy() // MASK_BLOCK] != 0)
         kk = kk[keep]
-    return kk
+    return k0 + kk
+
+
+def _n_keys(keys) -> int:
+    return keys.stop - keys.start if isinstance(keys, slice) else int(keys.numel())
 
 
 def attention_forward(prob, q, k, v) -> Tuple[torch.Tensor, torch.Tensor]:
@@ -83,8 +91,8 @@ def attention_forward(prob, q, k, v) -> Tuple[torch.Tensor, torch.Tensor]:
     O = torch.zeros(Nq, Hq, d, dtype=F64)
     LSE = torch.zeros(Nq, Hq, dtype=F64)
     for b, j, rows, k0, a in _blocks(prob):
-        keys = k0 + allowed_keys(prob, j, a)
-        if keys.numel() == 0:          # a block that may see no key: O = 0, LSE = -inf
+        keys = allowed_keys(prob, j, a, k0=k0)
+        if _n_keys(keys) == 0:         # a block that may see no key: O = 0, LSE = -inf
             LSE[rows] = -math.inf
             continue
         for h in range(Hq):
@@ -120,8 +128,8 @@ def attention_backward(prob, q, k, v, o, lse, do):
     dk = torch.zeros_like(k)
     dv = torch.zeros_like(v)
     for b, j, rows, k0, a in _blocks(prob):
-        keys = k0 + allowed_keys(prob, j, a)
-        if keys.numel() == 0:
+        keys = allowed_keys(prob, j, a, k0=k0)
+        if _n_keys(keys) == 0:
             continue
         for h in range(Hq):
             g = h // G
@@ -153,8 +161,8 @@ def chunk_partial(prob, q, k, v, b: int, key_begin: int, key_end: int):
     for bb, j, rows, k0, a in _blocks(prob):
         if bb != b:
             continue
-        keys = k0 + allowed_keys(prob, j, a, key_begin - k0, key_end - k0)
-        if keys.numel() == 0:
+        keys = allowed_keys(prob, j, a, key_begin - k0, key_end - k0, k0=k0)
+        if _n_keys(keys) == 0:
             continue
         for h in range(Hq):
             g = h // G
@@ -234,8 +242,8 @@ def chunked_backward(prob, q, k, v, o, lse, do, ranges=None):
         for bb, j, rows, k0, a in _blocks(prob):
             if bb != b:
                 continue
-            keys = k0 + allowed_keys(prob, j, a, lo_r - k0, hi_r - k0)
-            if keys.numel() == 0:
+            keys = allowed_keys(prob, j, a, lo_r - k0, hi_r - k0, k0=k0)
+            if _n_keys(keys) == 0:
                 continue
             for h in range(Hq):
                 g = h // G
@@ -260,5 +268,5 @@ def flops_fwd(prob) -> int:
     if getattr(prob, "key_block_mask", None) is None:
         n = int(np.sum(prob.anchors))
     else:
-        n = sum(int(allowed_keys(prob, j, a).numel()) for _b, j, _r, _k0, a in _blocks(prob))
+        n = sum(_n_keys(allowed_keys(prob, j, a)) for _b, j, _r, _k0, a in _blocks(prob))
     return 4 * prob.head_dim * prob.block_q * prob.num_q_heads * n
