@@ -42,6 +42,8 @@ WORKLOAD_TEXT = {
                "KV chunk 4096, 64 partitions, fwd+bwd",
     "batch8_logu": "8 samples, contexts log-uniform in [8192, 262144], 128 anchors x 16 draft tokens each, 32/8 heads, "
                    "d=128, KV chunk 4096, 128 partitions, fwd+bwd, anchors redrawn and replanned every step",
+    "ctx32k_sparse": "the ctx32k shapes under a block-sparse mask (per anchor: the first 2 blocks of 128 keys, the 4 "
+                     "blocks up to its own, each other block with probability 1/4), fwd+bwd",
 }
 METRIC = "split-KV attn fwd+bwd effective TFLOP/s"
 L2_BYTES = 126 * 1000 * 1000
@@ -98,9 +100,23 @@ def job_value(flops_all_ranks, seconds):
     return flops_all_ranks / seconds / 1e12
 
 
+def attended_keys(prob):
+    """Keys every anchor's block attends, summed over anchors: sum(a) under the
+    prefix mask; with a block-sparse mask, per anchor the keys of its set
+    128-key blocks that lie before a."""
+    m = getattr(prob, "key_block_mask", None)
+    if m is None:
+        return float(np.sum(prob.anchors))
+    a = np.asarray(prob.anchors, dtype=np.int64)[:, None]
+    starts = 128 * np.arange(m.shape[1], dtype=np.int64)[None, :]
+    per_block = np.clip(a - starts, 0, 128)
+    return float(((m != 0) * per_block).sum())
+
+
 def flops_of(prob, backward=True):
-    """Unmasked work: 4 d block_q Hq sum(a) forward, 2.5x that backward."""
-    f_fwd = 4.0 * prob.head_dim * prob.block_q * prob.num_q_heads * float(np.sum(prob.anchors))
+    """Unmasked work: 4 d block_q Hq per attended key of every anchor forward
+    (4 d block_q Hq sum(a) under the prefix mask), 2.5x that backward."""
+    f_fwd = 4.0 * prob.head_dim * prob.block_q * prob.num_q_heads * attended_keys(prob)
     return f_fwd, (2.5 * f_fwd if backward else 0.0)
 
 
@@ -197,7 +213,7 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------- GPU arm
-EXTRA_WORKLOADS = ("ctx128k", "batch8_logu")  # measured beside the headline workload on one GPU
+EXTRA_WORKLOADS = ("ctx128k", "batch8_logu", "ctx32k_sparse")  # measured beside the headline workload on one GPU
 
 
 def merge_bytes(prob, n_fwd_units):

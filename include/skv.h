@@ -88,6 +88,18 @@ typedef struct {
   int32_t num_q_heads;           /* Hq */
   int32_t num_kv_heads;          /* Hkv; Hq % Hkv == 0 and 128 % (Hq / Hkv) == 0 */
   int32_t head_dim;              /* d in {64, 128} */
+  /* Optional block-sparse mask over the context (NULL: the prefix mask alone).
+   * Row j (one per anchor, mask_stride bytes) holds one byte per block of 128
+   * keys of the anchor's sample: the block of anchor j attends key k (sample-
+   * relative) iff k < a_j and key_block_mask[j * mask_stride + k / 128] != 0.
+   * A block left with no key gets O = 0, LSE = -inf and no gradient. Needs
+   * mask_stride >= ceil(L_b / 128) for every sample (SKV_EINVAL otherwise).
+   * Plans of any policy carry the masked costs and loads; the kernel calls
+   * need every item to start on a 128-key block of its sample (LPT with
+   * chunk_kv / sub_chunks a multiple of 128) and return SKV_EUNSUPPORTED for
+   * other plans (the static split's pieces, for instance). */
+  const uint8_t* key_block_mask;
+  int32_t mask_stride;
 } skv_problem;
 
 /* One planned work item (a view into the plan buffer). */

@@ -19,7 +19,7 @@ STAMP = os.path.join(HERE, ".libskv.stamp")
 SOURCES = ["api.cu", "fwd.cu", "fwd2.cu", "bwd.cu", "bwd2.cu", "merge.cu", "noalloc.cu", "selftest.cu", "plan.cpp"]
 HEADERS = ["sm100.cuh", "kernels.h", "plan_layout.h", "merge_row.cuh", "tail_merge.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
-FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC,-O3", "-shared", "--expt-relaxed-constexpr"]
+FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC,-O3", "--expt-relaxed-constexpr"]
 
 
 def _nvcc() -> str:
@@ -46,11 +46,21 @@ def build(force: bool = False, verbose: bool = False) -> str:
         with open(STAMP) as f:
             if f.read().strip() == digest:
                 return LIB
-    cmd = [_nvcc(), *ARCH, *FLAGS, "-I", INCLUDE, "-o", LIB + ".tmp"] + [os.path.join(CSRC, s) for s in SOURCES]
-    if verbose:
-        cmd.insert(1, "-Xptxas=-v")
-        print(" ".join(cmd))
-    subprocess.check_call(cmd)
+    # one nvcc per source file, in parallel, then one link
+    import tempfile
+    from concurrent.futures import ThreadPoolExecutor
+    with tempfile.TemporaryDirectory(prefix="skv_build_") as tmp:
+        def compile_one(src):
+            obj = os.path.join(tmp, src + ".o")
+            cmd = [_nvcc(), *ARCH, *FLAGS, "-I", INCLUDE, "-c", os.path.join(CSRC, src), "-o", obj]
+            if verbose:
+                cmd.insert(1, "-Xptxas=-v")
+                print(" ".join(cmd))
+            subprocess.check_call(cmd)
+            return obj
+        with ThreadPoolExecutor(max_workers=max(1, min(len(SOURCES), os.cpu_count() or 1))) as pool:
+            objs = list(pool.map(compile_one, SOURCES))
+        subprocess.check_call([_nvcc(), *ARCH, "-shared", "-o", LIB + ".tmp", *objs])
     os.replace(LIB + ".tmp", LIB)
     with open(STAMP, "w") as f:
         f.write(digest)

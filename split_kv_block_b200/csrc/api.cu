@@ -195,6 +195,7 @@ namespace {
 // skv_attn_fwd_merged (partials merged into o / lse in the same launch).
 int run_fwd(const PlanHeader* h, const void* plan, const void* q, const void* k, const void* v, void* ws,
             size_t ws_bytes, void* o, float* lse, cudaStream_t stream) {
+  if (h->masked == 2) return SKV_EUNSUPPORTED;  // key tiles do not line up with the mask's blocks
   // a shard plan may own no key rows at all (more ranks than items): its K/V buffers may then be empty
   if (!q || !ws || (h->kv_rows > 0 && (!k || !v))) return SKV_EINVAL;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || reinterpret_cast<uintptr_t>(ws) % 256 != 0)
@@ -227,6 +228,13 @@ int run_fwd(const PlanHeader* h, const void* plan, const void* q, const void* k,
   p.P = h->n_queues;
   p.G = h->G;
   p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(h->d)));
+  if (h->masked) {
+    p.tile_mask = at<uint32_t>(dev, h->dev.tile_mask);
+    p.pair_tile_off = at<int32_t>(dev, h->dev.pair_tile_off);
+    p.unit_tile_off = at<int32_t>(dev, h->dev.unit_tile_off);
+    p.live_tiles = at<int32_t>(dev, h->dev.live_tiles);
+    p.mask_words = h->mask_words;
+  }
   // partials that fit in half of L2 are kept there (evict_last) until the merge reads them
   p.partials_l2_last = (w.fwd_end - w.fwd_o) <= kPartialsL2Bytes ? 1 : 0;
   if (o) {
@@ -283,6 +291,7 @@ extern "C" int skv_lse_merge(const void* plan, const skv_problem* prob, const vo
   int rc = SKV_OK;
   const PlanHeader* h = checked_plan(plan, prob, &rc);
   if (!h) return rc;
+  if (h->masked == 2) return SKV_EUNSUPPORTED;
   if (!ws || !o || !lse || !aligned16(o) || !aligned16(lse)) return SKV_EINVAL;
   const WsLayout w = ws_layout(*h);
   const uint8_t* dev = at<uint8_t>(ws, w.dev);
@@ -314,6 +323,7 @@ int run_bwd(const PlanHeader* h, const void* plan, const void* q, const void* k,
             const float* lse, const void* dout, void* dq, void* dk, void* dv, void* ws, size_t ws_bytes,
             cudaStream_t stream, bool det, bool dq_f32 = false) {
   int rc = SKV_OK;
+  if (h->masked == 2) return SKV_EUNSUPPORTED;  // key tiles do not line up with the mask's blocks
   if (!q || !o || !lse || !dout || !dq || !ws) return SKV_EINVAL;
   if (h->kv_rows > 0 && (!k || !v || !dk || !dv)) return SKV_EINVAL;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse) || !aligned16(dout) ||
@@ -360,6 +370,10 @@ int run_bwd(const PlanHeader* h, const void* plan, const void* q, const void* k,
     p.dk = static_cast<__nv_bfloat16*>(dk);
     p.dv = static_cast<__nv_bfloat16*>(dv);
     p.kv_heads = h->kv_heads;
+    if (h->masked) {
+      p.tile_mask = at<uint32_t>(dev, h->dev.tile_mask);
+      p.mask_words = h->mask_words;
+    }
     p.stamps = g_bwd_stamps;
     p.timeout_ns = kTimeoutNs;
     if (det) {

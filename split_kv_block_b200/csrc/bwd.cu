@@ -53,7 +53,11 @@ struct BwdShared {
   int32_t kend[2][128]; // absolute key end of the tile rows
 };
 
-template <int D, bool kDet>  // kDet: dQ added in ascending key order under turn counters
+// kDet: dQ added in ascending key order under turn counters. kMask: a
+// block-sparse mask (rows whose block is off attend no key of the unit); the
+// deterministic backward still walks the query tiles the mask turns off, so
+// that every unit below a tile's largest anchor takes its turn on that tile.
+template <int D, bool kDet, bool kMask>
 __global__ void __launch_bounds__(256, 1)
     bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
@@ -140,7 +144,7 @@ __global__ void __launch_bounds__(256, 1)
         ++n_units;
         for (int mt = U.mt_begin; mt < U.mt_end; ++mt) {
           const MTile M = p.mtiles[mt];
-          if (M.kmax <= U.kbeg) continue;
+          if (!tile_live<kMask && !kDet>(p, M, U.kbeg)) continue;
           if (qc >= 1 && !mbar_wait(&sh.q_empty, (qc - 1) & 1, status, lim)) { ok = false; break; }
           mbar_arrive_expect_tx(&sh.q_full, 2 * L::kTile);
           for (int db = 0; db < kDBlocks; ++db) {
@@ -187,7 +191,7 @@ __global__ void __launch_bounds__(256, 1)
         tc_fence_after();
         bool first = true;
         for (int mt = U.mt_begin; mt < U.mt_end && ok; ++mt) {
-          if (p.mtiles[mt].kmax <= U.kbeg) continue;
+          if (!tile_live<kMask && !kDet>(p, p.mtiles[mt], U.kbeg)) continue;
           if (!mbar_wait_warp(&sh.q_full, qc & 1, status, lim)) { ok = false; break; }
           tc_fence_after();
           if (leader) {
@@ -259,9 +263,11 @@ __global__ void __launch_bounds__(256, 1)
       const int nkeys = U.kend - U.kbeg;
       const int my_key = U.kbeg + t;
       const bool key_ok = t < nkeys;
+      bool had_tiles = false;
       for (int mt = U.mt_begin; mt < U.mt_end; ++mt) {
         const MTile M = p.mtiles[mt];
-        if (M.kmax <= U.kbeg) continue;
+        if (!tile_live<kMask && !kDet>(p, M, U.kbeg)) continue;
+        had_tiles = true;
         const int b2 = qc & 1;
         const int tl = t / p.G;
         const bool row_ok = tl < M.ntok;
@@ -269,7 +275,9 @@ __global__ void __launch_bounds__(256, 1)
         const int h = U.g * p.G + t % p.G;
         sh.lse2[b2][t] = row_ok ? p.lse[static_cast<size_t>(token) * p.Hq + h] * kLog2e : INFINITY;
         sh.delta[b2][t] = row_ok ? p.delta[static_cast<size_t>(token) * p.Hq + h] : 0.f;
-        sh.kend[b2][t] = row_ok ? p.tok_kend[token] : -1;
+        const bool row_on =
+            row_ok && (!kMask || ((mask_word(p.tile_mask, p.mask_words, M, U.kbeg, tl) >> (tl & 31)) & 1u));
+        sh.kend[b2][t] = row_on ? p.tok_kend[token] : -1;
         mbar_arrive(&sh.meta_full[b2]);
         if (!mbar_wait_warp(&sh.meta_full[b2], (qc >> 1) & 1, status, lim)) { ok = false; break; }
         if (!mbar_wait_warp(&sh.sdp_full, qc & 1, status, lim)) { ok = false; break; }
@@ -346,6 +354,10 @@ __global__ void __launch_bounds__(256, 1)
         tmem_ld32(lane_base + kColDV + c, vv);
         tmem_ld32(lane_base + kColDK + c, vk);
         tmem_wait_ld();
+        if (!had_tiles) {  // no query tile attends the unit's keys (a block mask): their gradients are zero
+#pragma unroll
+          for (int i = 0; i < 32; ++i) vv[i] = vk[i] = 0u;
+        }
         if (key_ok) {
 #pragma unroll
           for (int i = 0; i < 32; i += 8) {
@@ -382,7 +394,9 @@ int bwd_smem_bytes(int d) { return d == 64 ? BwdSmem<64>::kDyn : bwd2_smem_bytes
 cudaError_t launch_bwd(int d, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                        const CUtensorMap& tdo, const BwdParams& p, int grid, cudaStream_t stream) {
   if (d == 128) return launch_bwd2(tq, tk, tv, tdo, p, grid, stream);
-  auto k = p.det ? bwd_kernel<64, true> : bwd_kernel<64, false>;
+  const bool m = p.tile_mask != nullptr;
+  auto k = p.det ? (m ? bwd_kernel<64, true, true> : bwd_kernel<64, true, false>)
+                 : (m ? bwd_kernel<64, false, true> : bwd_kernel<64, false, false>);
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, BwdSmem<64>::kDyn);
   if (e != cudaSuccess) return e;
   k<<<grid, 256, BwdSmem<64>::kDyn, stream>>>(tq, tk, tv, tdo, p);

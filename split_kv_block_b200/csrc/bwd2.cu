@@ -66,8 +66,9 @@ constexpr uint32_t kColDV = 256, kColDK = 384;
 
 // kG: compile-time q-heads per kv-head (0 = runtime value p.G). kDet: dQ added
 // in ascending key order under turn counters (deterministic backward) instead
-// of fp32 atomics in any order.
-template <int kG, bool kDet>
+// of fp32 atomics in any order. kMask: a block-sparse mask (rows whose block is
+// off attend no key of the unit).
+template <int kG, bool kDet, bool kMask>
 __global__ void __launch_bounds__(384, 1)
     bwd2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                 const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
@@ -77,6 +78,10 @@ __global__ void __launch_bounds__(384, 1)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   int* status = p.status;
   const uint64_t lim = p.timeout_ns;
+  // The query tiles a unit walks skip the tiles the block mask turns off, except in the deterministic
+  // backward: there every unit below a tile's largest anchor takes its turn on that tile's dQ (adding
+  // zeros when the mask leaves it nothing), so the turn sequence is the same as without a mask.
+  constexpr bool kWalkMask = kMask && !kDet;
 
   // The 128-byte swizzle needs 1024-byte aligned tiles.
   if ((smem_u32(smem) & 1023u) != 0) {
@@ -167,7 +172,7 @@ __global__ void __launch_bounds__(384, 1)
         bool kv_loaded = false;
         for (int mt = U.mt_begin; mt < U.mt_end && ok; ++mt) {
           const MTile M = p.mtiles[mt];
-          if (M.kmax <= U.kbeg) continue;
+          if (!tile_live<kWalkMask>(p, M, U.kbeg)) continue;
           if (!load_tile(M, U.g)) { ok = false; break; }
           if (!kv_loaded) {  // after the first Q/dO tile: K/V wait for the previous unit's last MMA
             if (kv_issued >= 1 && !mbar_wait(&c.kv_empty, (kv_issued - 1) & 1, status, lim)) { ok = false; break; }
@@ -252,13 +257,13 @@ __global__ void __launch_bounds__(384, 1)
       // live query tiles in order (mt, then nxt); the liveness of the tile after nxt is loaded at the top of
       // a tile and read at its end, so no load stalls the issue of a tile's MMAs
       auto live_from = [&](int i) -> int {
-        while (i < U.mt_end && p.mtiles[i].kmax <= U.kbeg) ++i;
+        while (i < U.mt_end && !tile_live<kWalkMask>(p, p.mtiles[i], U.kbeg)) ++i;
         return i;
       };
       int mt = live_from(U.mt_begin);
       int nxt = mt < U.mt_end ? live_from(mt + 1) : U.mt_end;
       while (mt < U.mt_end) {
-        const int kmax_c = (nxt < U.mt_end && nxt + 1 < U.mt_end) ? p.mtiles[nxt + 1].kmax : 0;
+        const bool live_c = nxt < U.mt_end && nxt + 1 < U.mt_end && tile_live<kWalkMask>(p, p.mtiles[nxt + 1], U.kbeg);
         const int s = qc & 1;
         if (first) {  // a unit's first tile waits for the unit's K/V
           if (!mbar_wait_warp(&c.kv_full, (kv_waits++) & 1, status, lim)) { ok = false; break; }
@@ -306,12 +311,16 @@ __global__ void __launch_bounds__(384, 1)
         int nn = U.mt_end;
         if (nxt < U.mt_end) {
           nn = nxt + 1;
-          if (nn < U.mt_end && kmax_c <= U.kbeg) nn = live_from(nn + 1);
+          if (nn < U.mt_end && !live_c) nn = live_from(nn + 1);
         }
         mt = nxt;
         nxt = nn;
       }
       if (!ok) break;
+      // A unit without live query tiles (possible under a block mask) issues no MMA; it still waits for the
+      // previous unit's dK/dV read-out before signalling its own, so that acc_full never runs two phases ahead
+      // of the gradient warps (its parity would then name the wrong phase).
+      if (first && n_units >= 1 && !mbar_wait_warp(&c.acc_free, (n_units - 1) & 1, status, lim)) break;
       if (leader) {
         if (!first) umma_commit(&c.kv_empty);  // K/V were loaded for this unit
         umma_commit(&c.acc_full);
@@ -339,7 +348,7 @@ __global__ void __launch_bounds__(384, 1)
     float rw_lse = 0.f, rw_del = 0.f;
     int rw_ke = 0;
     bool rw_valid = false;
-    auto fetch = [&](const MTile& Mx, int g) {
+    auto fetch = [&](const MTile& Mx, int g, int kb) {
       if (t < 64) {
         const int r = 64 * wg + t;
         const int tl = r >> lgG;
@@ -348,12 +357,14 @@ __global__ void __launch_bounds__(384, 1)
         rw_lse = p.lse[static_cast<size_t>(token) * p.Hq + head];
         rw_del = p.delta[static_cast<size_t>(token) * p.Hq + head];
         rw_ke = p.tok_kend[token];
+        // a row whose block is off attends none of the unit's keys
+        if (kMask && rw_valid && !((mask_word(p.tile_mask, p.mask_words, Mx, kb, tl) >> (tl & 31)) & 1u)) rw_ke = 0;
       }
     };
     // the next live query tile of unit U at or after index i (the scan loads only at unit starts and when
     // a prefetched candidate is dead)
     auto live_from = [&](const BwdUnit& U, int i) -> int {
-      while (i < U.mt_end && p.mtiles[i].kmax <= U.kbeg) ++i;
+      while (i < U.mt_end && !tile_live<kWalkMask>(p, p.mtiles[i], U.kbeg)) ++i;
       return i;
     };
     while (ok) {
@@ -372,7 +383,7 @@ __global__ void __launch_bounds__(384, 1)
       int nxt = U.mt_end, cand = U.mt_end;
       if (mt < U.mt_end) {
         M = p.mtiles[mt];
-        fetch(M, U.g);
+        fetch(M, U.g, U.kbeg);
         nxt = live_from(U, mt + 1);
         if (nxt < U.mt_end) {
           Mn = p.mtiles[nxt];
@@ -400,10 +411,10 @@ __global__ void __launch_bounds__(384, 1)
         int nn = U.mt_end;
         MTile Mnn = Mn;
         if (nxt < U.mt_end) {
-          fetch(Mn, U.g);
+          fetch(Mn, U.g, U.kbeg);
           nn = cand;
           if (nn < U.mt_end) {
-            if (Mc.kmax > U.kbeg) {
+            if (tile_live<kWalkMask>(p, Mc, U.kbeg)) {
               Mnn = Mc;
             } else {
               nn = live_from(U, nn + 1);
@@ -575,8 +586,11 @@ int bwd2_smem_bytes() { return kSmemBytes; }
 
 cudaError_t launch_bwd2(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tdo,
                         const BwdParams& p, int grid, cudaStream_t stream) {
-  auto kern = p.det ? (p.G == 4 ? bwd2_kernel<4, true> : bwd2_kernel<0, true>)
-                    : (p.G == 4 ? bwd2_kernel<4, false> : bwd2_kernel<0, false>);
+  const bool m = p.tile_mask != nullptr;
+  auto kern = p.det ? (p.G == 4 ? (m ? bwd2_kernel<4, true, true> : bwd2_kernel<4, true, false>)
+                                : (m ? bwd2_kernel<0, true, true> : bwd2_kernel<0, true, false>))
+                    : (p.G == 4 ? (m ? bwd2_kernel<4, false, true> : bwd2_kernel<4, false, false>)
+                                : (m ? bwd2_kernel<0, false, true> : bwd2_kernel<0, false, false>));
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
   if (e != cudaSuccess) return e;
   kern<<<grid, 384, kSmemBytes, stream>>>(tq, tk, tv, tdo, p);

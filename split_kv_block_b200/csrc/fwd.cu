@@ -55,7 +55,9 @@ struct FwdBarriers {
 };
 
 // kMerge: the LSE merge runs in the kernel's tail (skv_attn_fwd_merged).
-template <int D, bool kMerge>
+// kMask: a block-sparse mask; every role walks the unit's list of live key
+// tiles and the softmax masks the rows whose block is off.
+template <int D, bool kMerge, bool kMask>
 __global__ void __launch_bounds__(256, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
@@ -131,7 +133,9 @@ __global__ void __launch_bounds__(256, 1)
         for (int db = 0; db < kDBlocks; ++db)
           tma_load_3d(smem + L::kQ + db * (kTileM * 128), &tmQ, &bars.q_full, db * 64, U.g * p.G, M.tok0);
         ++q_issued;
-        for (int kb = U.kbeg; kb < U.kend; kb += kTileN, ++kv) {
+        const int nt_p = kMask ? p.unit_tile_off[u + 1] - p.unit_tile_off[u] : (U.kend - U.kbeg + kTileN - 1) / kTileN;
+        for (int jt = 0; jt < nt_p; ++jt, ++kv) {
+          const int kb = kMask ? p.live_tiles[p.unit_tile_off[u] + jt] : U.kbeg + jt * kTileN;
           const int st = kv & 1;
           const uint32_t use = kv >> 1;
           if (use >= 1 && !mbar_wait(&bars.k_empty[st], (use - 1) & 1, status, lim)) { ok = false; break; }
@@ -180,7 +184,7 @@ __global__ void __launch_bounds__(256, 1)
         if (leader) mbar_arrive(&bars.sched_empty[slot]);
         if (u < 0) break;
         const FwdUnit U = p.units[u];
-        const int nt = (U.kend - U.kbeg + kTileN - 1) / kTileN;
+        const int nt = kMask ? p.unit_tile_off[u + 1] - p.unit_tile_off[u] : (U.kend - U.kbeg + kTileN - 1) / kTileN;
         if (!mbar_wait_warp(&bars.q_full, n_units & 1, status, lim)) break;
         tc_fence_after();
         auto issue_s = [&](uint32_t t_index, uint32_t kv_index) -> bool {
@@ -255,14 +259,17 @@ __global__ void __launch_bounds__(256, 1)
       const int tl = r / p.G;
       const bool valid = tl < M.ntok;
       const int row_end = valid ? min(p.tok_kend[M.tok0 + tl], U.kend) : U.kbeg;
-      const int nt = (U.kend - U.kbeg + kTileN - 1) / kTileN;
+      const int nt = kMask ? p.unit_tile_off[u + 1] - p.unit_tile_off[u] : (U.kend - U.kbeg + kTileN - 1) / kTileN;
       float m = -INFINITY, l = 0.f;
       bool ok = true;
       for (int j = 0; j < nt; ++j) {
         const uint32_t tj = tcount + j;
         if (!mbar_wait_warp(&bars.s_full[tj & 1], (tj >> 1) & 1, status, lim)) { ok = false; break; }
         tc_fence_after();
-        const int lim_c = row_end - (U.kbeg + j * kTileN);  // valid columns in this tile
+        const int kb = kMask ? p.live_tiles[p.unit_tile_off[u] + j] : U.kbeg + j * kTileN;
+        int lim_c = row_end - kb;  // valid columns in this tile
+        if (kMask && valid && !((mask_word(p.tile_mask, p.mask_words, M, kb, tl) >> (tl & 31)) & 1u))
+          lim_c = 0;  // the row's block is off
         float s[kTileN];
         const uint32_t scol = (tj & 1) ? kColS1 : kColS0;
 #pragma unroll
@@ -383,7 +390,8 @@ int fwd_smem_bytes(int d) { return d == 64 ? FwdSmem<64>::kDyn : FwdSmem<128>::k
 cudaError_t launch_fwd(int d, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                        const FwdParams& p, int grid, cudaStream_t stream) {
   if (d == 128) return launch_fwd2(tq, tk, tv, p, grid, stream);
-  auto k = p.o ? fwd_kernel<64, true> : fwd_kernel<64, false>;
+  auto k = p.tile_mask ? (p.o ? fwd_kernel<64, true, true> : fwd_kernel<64, false, true>)
+                       : (p.o ? fwd_kernel<64, true, false> : fwd_kernel<64, false, false>);
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, FwdSmem<64>::kDyn);
   if (e != cudaSuccess) return e;
   k<<<grid, 256, FwdSmem<64>::kDyn, stream>>>(tq, tk, tv, p);

@@ -109,8 +109,10 @@ __device__ __forceinline__ float exp_row(const uint32_t (&sv)[128], float sl2, f
 }
 
 // kMerge: the LSE merge runs in the kernel's tail (skv_attn_fwd_merged); the
-// plain forward is compiled without that code.
-template <bool kMerge>
+// plain forward is compiled without that code. kMask: a block-sparse mask;
+// every role walks the pair's list of live key tiles (the same list, so they
+// agree on the sequence) and the softmax masks the rows whose block is off.
+template <bool kMerge, bool kMask>
 __global__ void __launch_bounds__(384, 1)
     fwd2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                 const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
@@ -190,7 +192,9 @@ __global__ void __launch_bounds__(384, 1)
         }
         // K/V buffer coordinates of the pair's item: head kvh, key kb at row kb - kshift
         const int kvh = p.units[pr.slot[0]].kvh, kshift = p.units[pr.slot[0]].kshift;
-        for (int kb = pr.kbeg; kb < pr.kend && ok; kb += kTileN, ++kv) {
+        const int nt_p = kMask ? p.pair_tile_off[u + 1] - p.pair_tile_off[u] : (pr.kend - pr.kbeg + kTileN - 1) / kTileN;
+        for (int jt = 0; jt < nt_p && ok; ++jt, ++kv) {
+          const int kb = kMask ? p.live_tiles[p.pair_tile_off[u] + jt] : pr.kbeg + jt * kTileN;
           const int st = kv & 1;
           const uint32_t use = kv >> 1;
           if (use >= 1 && !mbar_wait(&c.k_empty[st], (use - 1) & 1, status, lim)) { ok = false; break; }
@@ -267,7 +271,7 @@ __global__ void __launch_bounds__(384, 1)
         if (u < 0) break;
         const FwdPair pr = p.pairs[u];
         const bool has[2] = {pr.slot[0] >= 0, pr.slot[1] >= 0};
-        const int nt = (pr.kend - pr.kbeg + kTileN - 1) / kTileN;
+        const int nt = kMask ? p.pair_tile_off[u + 1] - p.pair_tile_off[u] : (pr.kend - pr.kbeg + kTileN - 1) / kTileN;
         for (int t = 0; t < 2 && ok; ++t) {
           if (!has[t]) continue;
           if (!mbar_wait_warp(&c.q_full[t], q_use[t] & 1, status, lim)) { ok = false; break; }
@@ -354,7 +358,7 @@ __global__ void __launch_bounds__(384, 1)
       if (u < 0) break;
       ++n_units;
       const FwdPair pr = p.pairs[u];
-      const int nt = (pr.kend - pr.kbeg + kTileN - 1) / kTileN;
+      const int nt = kMask ? p.pair_tile_off[u + 1] - p.pair_tile_off[u] : (pr.kend - pr.kbeg + kTileN - 1) / kTileN;
       if (pr.slot[t] < 0) continue;  // odd tile count: this warpgroup sits the pair out
       const int sl = pr.slot[t];
       const FwdUnit U = p.units[sl];
@@ -369,7 +373,10 @@ __global__ void __launch_bounds__(384, 1)
         if (!mbar_wait_warp(&c.s_full[t], s_cnt & 1, status, lim)) { ok = false; break; }
         ++s_cnt;
         tc_fence_after();
-        const int lim_c = row_end - (pr.kbeg + j * kTileN);  // valid columns of this row in the tile
+        const int kb = kMask ? p.live_tiles[p.pair_tile_off[u] + j] : pr.kbeg + j * kTileN;
+        int lim_c = row_end - kb;  // valid columns of this row in the tile
+        if (kMask && valid && !((mask_word(p.tile_mask, p.mask_words, M, kb, tl) >> (tl & 31)) & 1u))
+          lim_c = 0;  // the row's block is off
         // the whole row of S in registers: four loads in flight, one wait
         uint32_t sv[128];
 #pragma unroll
@@ -480,7 +487,8 @@ int fwd2_smem_bytes() { return kSmemBytes; }
 
 cudaError_t launch_fwd2(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const FwdParams& p,
                         int grid, cudaStream_t stream) {
-  auto kern = p.o ? fwd2_kernel<true> : fwd2_kernel<false>;
+  auto kern = p.tile_mask ? (p.o ? fwd2_kernel<true, true> : fwd2_kernel<false, true>)
+                          : (p.o ? fwd2_kernel<true, false> : fwd2_kernel<false, false>);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
   if (e != cudaSuccess) return e;
   kern<<<grid, 384, kSmemBytes, stream>>>(tq, tk, tv, p);

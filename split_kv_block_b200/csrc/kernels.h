@@ -27,6 +27,13 @@ struct FwdParams {
   int G;
   float scale_log2;         // log2(e) / sqrt(d)
   int partials_l2_last;     // store the partials with the L2 evict_last policy (they fit in L2 beside K/V)
+  // block-sparse mask (kernels compiled with kMask): per (tile, block) token words, and the live key tiles
+  // of every forward pair (head_dim 128) or unit (head_dim 64) as first keys
+  const uint32_t* tile_mask;
+  const int32_t* pair_tile_off;  // [n_pairs + 1]
+  const int32_t* unit_tile_off;  // [n_fwd + 1]
+  const int32_t* live_tiles;
+  int mask_words;
   // LSE merge in the same launch (tail_merge.cuh) when o != nullptr; partials only otherwise.
   const int32_t* merge_off;   // [n_slots + 1]: units of slot (query tile, kv head) = mt * Hkv + g
   const int32_t* merge_list;  // forward unit ids per slot, ascending key order
@@ -65,6 +72,8 @@ struct BwdParams {
   __nv_bfloat16* dk;        // [kv_rows][kv_heads][d] (the K/V buffers' layout)
   __nv_bfloat16* dv;
   int kv_heads;             // heads per K/V row: Hkv for a full plan, 1 for a shard plan
+  const uint32_t* tile_mask;  // block-sparse mask (kernels compiled with kMask): per (tile, block) token words
+  int mask_words;
   long long* stamps;
   unsigned long long timeout_ns;
   // Deterministic dQ (det != 0): units are taken from det_order through counters[0] instead of the

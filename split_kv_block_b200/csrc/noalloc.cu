@@ -74,6 +74,7 @@ extern "C" int skv_attn_fwd_noalloc(const void* plan, const skv_problem* prob, c
   int rc = SKV_OK;
   const PlanHeader* h = checked_plan(plan, prob, &rc);
   if (!h) return rc;
+  if (h->masked == 2) return SKV_EUNSUPPORTED;  // key tiles do not line up with the mask's blocks
   if (!q || !k || !v || !o || !lse) return SKV_EINVAL;
   for (const void* ptr : {q, k, v, static_cast<const void*>(o), static_cast<const void*>(lse)})
     if (reinterpret_cast<uintptr_t>(ptr) % 16 != 0) return SKV_EINVAL;
@@ -110,6 +111,13 @@ extern "C" int skv_attn_fwd_noalloc(const void* plan, const skv_problem* prob, c
   p.part_o = reinterpret_cast<float*>(base + w.fwd_o);
   p.part_lse = reinterpret_cast<float*>(base + w.fwd_lse);
   p.partial_bf16 = (h->policy & SKV_PLAN_PARTIALS_BF16) ? 1 : 0;
+  if (h->masked) {
+    p.tile_mask = reinterpret_cast<const uint32_t*>(dev + h->dev.tile_mask);
+    p.pair_tile_off = reinterpret_cast<const int32_t*>(dev + h->dev.pair_tile_off);
+    p.unit_tile_off = reinterpret_cast<const int32_t*>(dev + h->dev.unit_tile_off);
+    p.live_tiles = reinterpret_cast<const int32_t*>(dev + h->dev.live_tiles);
+    p.mask_words = h->mask_words;
+  }
   p.stamps = nullptr;
   p.timeout_ns = 2000000000ull;
   p.P = h->n_queues;

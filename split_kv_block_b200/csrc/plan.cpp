@@ -15,6 +15,7 @@
 // O(log A) per item.
 #include <algorithm>
 #include <cstring>
+#include <iterator>
 #include <functional>
 #include <numeric>
 #include <queue>
@@ -31,6 +32,9 @@ struct Prob {
   const int64_t* ctx;
   const int32_t* aoff;
   const int64_t* anchors;
+  const uint8_t* mask;  // block-sparse mask [A][mask_stride], or nullptr
+  int mask_stride;
+  int mask_words;       // words per (tile, block): ceil(TT / 32)
 };
 
 int validate(const skv_problem* p, Prob& q) {
@@ -60,10 +64,18 @@ int validate(const skv_problem* p, Prob& q) {
     for (int32_t j = q.aoff[b]; j < q.aoff[b + 1]; ++j)
       if (q.anchors[j] < 1 || q.anchors[j] > L) return SKV_EINVAL;
   }
+  q.mask = p->key_block_mask;
+  q.mask_stride = p->mask_stride;
+  if (q.mask) {
+    if (q.mask_stride < 1) return SKV_EINVAL;
+    for (int b = 0; b < q.B; ++b)
+      if ((q.ctx[b + 1] - q.ctx[b] + kTileN - 1) / kTileN > q.mask_stride) return SKV_EINVAL;
+  }
   q.G = q.Hq / q.Hkv;
   if (q.d != 64 && q.d != 128) return SKV_EUNSUPPORTED;
   if (q.G > kTileM || kTileM % q.G != 0) return SKV_EUNSUPPORTED;
   q.TT = kTileM / q.G;
+  q.mask_words = (q.TT + 31) / 32;
   q.Nq = A * q.S;
   q.Ltot = q.ctx[q.B];
   // 32-bit indices on the device: keys and query tokens (with tile slack).
@@ -77,6 +89,10 @@ struct SampleAnchors {
   std::vector<int64_t> a;       // sorted
   std::vector<int64_t> prefix;  // prefix[i] = a[0] + ... + a[i-1]
   int64_t max_a = 0;
+  // block-sparse mask: allowed (token-of-anchor, key) pairs per anchor summed over the sample's 128-key
+  // blocks before block kb (block_prefix[kb]); a key of block kb counts for anchor j when the mask allows
+  // the block and the key lies before a_j
+  std::vector<int64_t> block_prefix;
 };
 
 // sum_j max(0, min(hi, a_j) - lo), relative coordinates, lo < hi.
@@ -105,6 +121,11 @@ struct Built {
   std::vector<BwdUnit> bwd;
   std::vector<int32_t> bwd_part_off;
   std::vector<int32_t> bwd_item, bwd_part;  // host-side: item and partition of every backward unit
+  std::vector<uint32_t> tile_mask;           // block-sparse mask: per (tile, block) words of token bits
+  std::vector<int32_t> pair_tile_off, unit_tile_off, live_tiles;
+  std::vector<std::vector<int32_t>> unit_live;  // live key tiles of every forward unit (mask only)
+  std::vector<int32_t> unit_tiles;              // scratch
+  bool mask_aligned = true;                     // items line up with the mask's blocks (kernels can run)
   std::vector<int32_t> bwd_rank, bwd_det_order;
   std::vector<int64_t> dead;  // [2 n_dead]
   int shard = -1, n_queues = 1, kv_heads = 1;
@@ -114,7 +135,27 @@ struct Built {
 };
 
 void make_items(const Prob& q, int policy, const std::vector<SampleAnchors>& sa, Built& out) {
+  // allowed (anchor, key) pairs of the keys [x, y) inside one 128-key block, counted anchor by anchor
+  auto block_part = [&](int b, int64_t x, int64_t y) -> int64_t {
+    if (y <= x) return 0;
+    const int64_t kb = x / kTileN;
+    int64_t n = 0;
+    for (int32_t j = q.aoff[b]; j < q.aoff[b + 1]; ++j)
+      if (q.mask[static_cast<size_t>(j) * q.mask_stride + kb]) n += std::max<int64_t>(0, std::min(y, q.anchors[j]) - x);
+    return n;
+  };
   auto cost = [&](int b, int64_t lo_abs, int64_t hi_abs) {
+    if (q.mask) {
+      // whole blocks from the per-block prefix sums, the partial blocks at either end anchor by anchor
+      const int64_t lo = lo_abs - q.ctx[b], hi = hi_abs - q.ctx[b];
+      const int64_t f0 = (lo + kTileN - 1) / kTileN, f1 = hi / kTileN;
+      int64_t n;
+      if (f0 <= f1)
+        n = sa[b].block_prefix[f1] - sa[b].block_prefix[f0] + block_part(b, lo, f0 * kTileN) + block_part(b, f1 * kTileN, hi);
+      else
+        n = block_part(b, lo, hi);  // inside one block
+      return static_cast<int64_t>(q.G) * q.S * n;
+    }
     return static_cast<int64_t>(q.G) * q.S * pair_sum(sa[b], lo_abs - q.ctx[b], hi_abs - q.ctx[b]);
   };
   out.items.clear();
@@ -243,10 +284,44 @@ void make_lists(const Prob& q, const std::vector<SampleAnchors>& sa, int shard, 
       const int64_t nt = std::min<int64_t>(q.TT, t_end - t0);
       int64_t amax = 0;
       for (int64_t j = t0 / q.S; j <= (t0 + nt - 1) / q.S; ++j) amax = std::max(amax, q.anchors[j]);
-      out.mtiles.push_back({b, static_cast<int32_t>(t0), static_cast<int32_t>(nt), static_cast<int32_t>(q.ctx[b] + amax)});
+      MTile M{};
+      M.b = b;
+      M.tok0 = static_cast<int32_t>(t0);
+      M.ntok = static_cast<int32_t>(nt);
+      M.kmax = static_cast<int32_t>(q.ctx[b] + amax);
+      M.kbase = static_cast<int32_t>(q.ctx[b]);
+      out.mtiles.push_back(M);
     }
   }
   out.sample_mt[q.B] = static_cast<int32_t>(out.mtiles.size());
+
+  // block-sparse mask: per (tile, block) the tile's tokens that attend keys of the block
+  out.tile_mask.clear();
+  if (q.mask) {
+    int64_t entries = 0;
+    for (auto& M : out.mtiles) {
+      M.mbase = static_cast<int32_t>(entries);
+      entries += (q.ctx[M.b + 1] - q.ctx[M.b] + kTileN - 1) / kTileN;
+    }
+    out.tile_mask.assign(static_cast<size_t>(entries) * q.mask_words, 0u);
+    for (const auto& M : out.mtiles) {
+      const int64_t nkb = (q.ctx[M.b + 1] - q.ctx[M.b] + kTileN - 1) / kTileN;
+      for (int t = 0; t < M.ntok; ++t) {
+        const int64_t j = (M.tok0 + t) / q.S;
+        const uint8_t* row = q.mask + static_cast<size_t>(j) * q.mask_stride;
+        const int64_t a = q.anchors[j];
+        for (int64_t kb = 0; kb < nkb && kb * kTileN < a; ++kb)
+          if (row[kb]) out.tile_mask[static_cast<size_t>(M.mbase + kb) * q.mask_words + t / 32] |= 1u << (t % 32);
+      }
+    }
+  }
+  // live blocks of tile mt among the sample-relative blocks [kb0, kb1)
+  auto block_live = [&](int32_t mt, int64_t kb) -> bool {
+    const uint32_t* w = out.tile_mask.data() + static_cast<size_t>(out.mtiles[mt].mbase + kb) * q.mask_words;
+    for (int i = 0; i < q.mask_words; ++i)
+      if (w[i]) return true;
+    return false;
+  };
 
   // K/V rows of every item, and the items each work queue runs in placement order
   out.shard = shard;
@@ -275,6 +350,7 @@ void make_lists(const Prob& q, const std::vector<SampleAnchors>& sa, int shard, 
     if (in_plan[id]) by_queue[shard < 0 ? out.items[id].partition : 0].push_back(id);
 
   out.fwd.clear();
+  out.unit_live.clear();
   out.fwd_part_off.assign(out.n_queues + 1, 0);
   out.pairs.clear();
   out.pair_off.assign(out.n_queues + 1, 0);
@@ -295,12 +371,19 @@ void make_lists(const Prob& q, const std::vector<SampleAnchors>& sa, int shard, 
       const int32_t kvh = shard < 0 ? it.g : 0;
       // forward: live query tiles, longest key range first (ties by tile index). Tiles reaching past
       // the item's end all have its full range and come first in index order; only the others,
-      // few per item, need sorting.
+      // few per item, need sorting. With a block mask a tile is live when one of its tokens attends
+      // a key of one of the item's blocks, and its extent is its count of live blocks.
       tiles.clear();
       size_t n_full = 0;
+      const int64_t kb_lo = (it.key_begin - q.ctx[it.b]) / kTileN;
+      const int64_t kb_hi = (it.key_end - q.ctx[it.b] + kTileN - 1) / kTileN;
       for (int32_t mt = out.sample_mt[it.b]; mt < out.sample_mt[it.b + 1]; ++mt) {
         const int64_t kmax = out.mtiles[mt].kmax;
-        if (kmax >= it.key_end) {
+        if (q.mask) {
+          int64_t n_live = 0;
+          for (int64_t kb = kb_lo; kb < kb_hi; ++kb) n_live += block_live(mt, kb);
+          if (n_live > 0) tiles.push_back({-n_live, mt});
+        } else if (kmax >= it.key_end) {
           tiles.insert(tiles.begin() + static_cast<std::ptrdiff_t>(n_full++), {-(it.key_end - it.key_begin), mt});
         } else if (kmax > it.key_begin) {
           tiles.push_back({-(kmax - it.key_begin), mt});
@@ -319,6 +402,15 @@ void make_lists(const Prob& q, const std::vector<SampleAnchors>& sa, int shard, 
         u.part = it.partition;
         u.kshift = kshift;
         u.kvh = kvh;
+        if (q.mask) {
+          // the unit's live key tiles: from its first to its last live block
+          out.unit_tiles.clear();
+          for (int64_t kb = kb_lo; kb < kb_hi; ++kb)
+            if (block_live(u.mt, kb)) out.unit_tiles.push_back(static_cast<int32_t>(q.ctx[it.b] + kb * kTileN));
+          u.kbeg = out.unit_tiles.front();
+          u.kend = static_cast<int32_t>(std::min<int64_t>(out.unit_tiles.back() + kTileN, it.key_end));
+          out.unit_live.push_back(out.unit_tiles);
+        }
         // consecutive tiles (similar key extents) share a pair; the first is the longer
         if (ti % 2 == 0) {
           FwdPair pr{};
@@ -329,7 +421,10 @@ void make_lists(const Prob& q, const std::vector<SampleAnchors>& sa, int shard, 
           pr.part = it.partition;
           out.pairs.push_back(pr);
         } else {
-          out.pairs.back().slot[1] = static_cast<int32_t>(out.fwd.size());
+          FwdPair& pr = out.pairs.back();
+          pr.slot[1] = static_cast<int32_t>(out.fwd.size());
+          pr.kbeg = std::min(pr.kbeg, u.kbeg);  // with a block mask the second tile may reach further
+          pr.kend = std::max(pr.kend, u.kend);
         }
         out.fwd.push_back(u);
       }
@@ -361,6 +456,31 @@ void make_lists(const Prob& q, const std::vector<SampleAnchors>& sa, int shard, 
   out.fwd_part_off[out.n_queues] = static_cast<int32_t>(out.fwd.size());
   out.pair_off[out.n_queues] = static_cast<int32_t>(out.pairs.size());
   out.bwd_part_off[out.n_queues] = static_cast<int32_t>(out.bwd.size());
+
+  // block-sparse mask: the live key tiles of every forward pair (union of its two units', ascending)
+  // and of every forward unit, as first keys; pairs' lists first, then units'
+  out.pair_tile_off.clear();
+  out.unit_tile_off.clear();
+  out.live_tiles.clear();
+  if (q.mask) {
+    out.pair_tile_off.push_back(0);
+    for (const auto& pr : out.pairs) {
+      const auto& a = out.unit_live[pr.slot[0]];
+      if (pr.slot[1] < 0) {
+        out.live_tiles.insert(out.live_tiles.end(), a.begin(), a.end());
+      } else {
+        const auto& c = out.unit_live[pr.slot[1]];
+        std::set_union(a.begin(), a.end(), c.begin(), c.end(), std::back_inserter(out.live_tiles));
+      }
+      out.pair_tile_off.push_back(static_cast<int32_t>(out.live_tiles.size()));
+    }
+    const int32_t base = static_cast<int32_t>(out.live_tiles.size());
+    out.unit_tile_off.push_back(base);
+    for (size_t u = 0; u < out.fwd.size(); ++u) {
+      out.live_tiles.insert(out.live_tiles.end(), out.unit_live[u].begin(), out.unit_live[u].end());
+      out.unit_tile_off.push_back(static_cast<int32_t>(out.live_tiles.size()));
+    }
+  }
 
   // Deterministic backward: the rank of every unit's key tile among the plan's key tiles of its (sample,
   // kv head) in ascending key order, and the dispatch order (sample, rank, kv head). Items of one (sample,
@@ -467,8 +587,56 @@ int build(const skv_problem* prob, int policy, Built& out, Prob& q, int shard = 
     sa[b].max_a = sa[b].a.empty() ? 0 : sa[b].a.back();
   }
   if (shard >= q.P) return SKV_EINVAL;
+  if (q.mask) {
+    for (int b = 0; b < q.B; ++b) {
+      const int64_t nkb = (q.ctx[b + 1] - q.ctx[b] + kTileN - 1) / kTileN;
+      std::vector<int64_t>& bp = sa[b].block_prefix;
+      bp.assign(nkb + 1, 0);
+      for (int32_t j = q.aoff[b]; j < q.aoff[b + 1]; ++j) {
+        const uint8_t* row = q.mask + static_cast<size_t>(j) * q.mask_stride;
+        const int64_t a = q.anchors[j];
+        for (int64_t kb = 0; kb < nkb && kb * kTileN < a; ++kb)
+          if (row[kb]) bp[kb + 1] += std::min<int64_t>(a, (kb + 1) * kTileN) - kb * kTileN;
+      }
+      for (int64_t kb = 0; kb < nkb; ++kb) bp[kb + 1] += bp[kb];
+    }
+  }
   make_items(q, policy, sa, out);
   place(q, policy, out);
+  // the kernels need every item's key tiles to line up with the mask's 128-key blocks
+  out.mask_aligned = true;
+  if (q.mask)
+    for (const auto& it : out.items)
+      if ((it.key_begin - q.ctx[it.b]) % kTileN != 0) out.mask_aligned = false;
+  if (q.mask && !out.mask_aligned) {
+    // plan (costs, loads, imbalance) only: no work lists, the kernel calls refuse such a plan
+    for (auto& it : out.items) it.kv_row = shard < 0 ? it.key_begin : -1;
+    out.shard = shard;
+    out.n_queues = shard < 0 ? q.P : 1;
+    out.kv_heads = shard < 0 ? q.Hkv : 1;
+    out.kv_rows = 0;
+    out.mtiles.clear();
+    out.sample_mt.assign(q.B + 1, 0);
+    out.tok_kend.clear();
+    out.tile_mask.clear();
+    out.fwd.clear();
+    out.pairs.clear();
+    out.bwd.clear();
+    out.bwd_item.clear();
+    out.bwd_part.clear();
+    out.bwd_rank.clear();
+    out.bwd_det_order.clear();
+    out.fwd_part_off.assign(out.n_queues + 1, 0);
+    out.pair_off.assign(out.n_queues + 1, 0);
+    out.bwd_part_off.assign(out.n_queues + 1, 0);
+    out.merge_off.assign(1, 0);
+    out.merge_list.clear();
+    out.pair_tile_off.clear();
+    out.unit_tile_off.clear();
+    out.live_tiles.clear();
+    out.dead.clear();
+    return SKV_OK;
+  }
   make_lists(q, sa, shard, out);
   return SKV_OK;
 }
@@ -505,6 +673,8 @@ PlanHeader layout_of(const Prob& q, int policy, const Built& b) {
   h.kv_rows = b.kv_rows;
   h.n_dead = static_cast<int32_t>(b.dead.size() / 2);
   h.empty_slots = 0;
+  h.masked = q.mask ? (b.mask_aligned ? 1 : 2) : 0;
+  h.mask_words = q.mask_words;
   for (size_t i = 0; i + 1 < b.merge_off.size(); ++i) h.empty_slots += b.merge_off[i + 1] == b.merge_off[i];
   uint64_t off = align_up(sizeof(PlanHeader), 256);
   h.items_off = off;
@@ -529,6 +699,10 @@ PlanHeader layout_of(const Prob& q, int policy, const Built& b) {
   h.dev.bwd_units = put(b.bwd.size() * sizeof(BwdUnit));
   h.dev.bwd_part_off = put(b.bwd_part_off.size() * sizeof(int32_t));
   h.dev.dead = put(b.dead.size() * sizeof(int64_t));
+  h.dev.tile_mask = put(b.tile_mask.size() * sizeof(uint32_t));
+  h.dev.pair_tile_off = put(b.pair_tile_off.size() * sizeof(int32_t));
+  h.dev.unit_tile_off = put(b.unit_tile_off.size() * sizeof(int32_t));
+  h.dev.live_tiles = put(b.live_tiles.size() * sizeof(int32_t));
   h.dev.base_bytes = d;
   h.dev.bwd_rank = put(b.bwd_rank.size() * sizeof(int32_t));
   h.dev.bwd_det_order = put(b.bwd_det_order.size() * sizeof(int32_t));
@@ -560,6 +734,12 @@ uint64_t problem_fingerprint(const skv_problem* p) {
   }
   const int32_t A = p->anchor_offsets[p->num_samples];
   for (int32_t j = 0; j < A; ++j) f.add(p->anchors[j]);
+  const int32_t has_mask = p->key_block_mask ? 1 : 0;
+  f.add(has_mask);
+  if (p->key_block_mask) {
+    f.add(p->mask_stride);
+    for (size_t i = 0; i < static_cast<size_t>(A) * p->mask_stride; ++i) f.add(p->key_block_mask[i]);
+  }
   return f.h;
 }
 
@@ -640,6 +820,10 @@ int write_plan(const skv_problem* prob, int policy, int shard, void* plan, size_
   copy_to(dev, h.dev.bwd_units, b.bwd);
   copy_to(dev, h.dev.bwd_part_off, b.bwd_part_off);
   copy_to(dev, h.dev.dead, b.dead);
+  copy_to(dev, h.dev.tile_mask, b.tile_mask);
+  copy_to(dev, h.dev.pair_tile_off, b.pair_tile_off);
+  copy_to(dev, h.dev.unit_tile_off, b.unit_tile_off);
+  copy_to(dev, h.dev.live_tiles, b.live_tiles);
   copy_to(dev, h.dev.bwd_rank, b.bwd_rank);
   copy_to(dev, h.dev.bwd_det_order, b.bwd_det_order);
   if (partition_load) std::memcpy(partition_load, b.load.data(), b.load.size() * sizeof(int64_t));

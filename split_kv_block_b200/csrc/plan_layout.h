@@ -18,9 +18,12 @@ constexpr int kTileN = 128;  // keys per tile
 // the kv group): row r is token tok0 + r / G, q-head g * G + r % G.
 struct MTile {
   int32_t b;
-  int32_t tok0;  // first query token (packed index)
-  int32_t ntok;  // tokens in the tile, <= 128 / G
-  int32_t kmax;  // absolute key end: ctx_offsets[b] + max anchor over its tokens
+  int32_t tok0;   // first query token (packed index)
+  int32_t ntok;   // tokens in the tile, <= 128 / G
+  int32_t kmax;   // absolute key end: ctx_offsets[b] + max anchor over its tokens
+  int32_t kbase;  // first key of the sample (ctx_offsets[b])
+  int32_t mbase;  // block-sparse mask: entry of (this tile, block 0) in the tile-block words
+  int32_t pad0, pad1;
 };
 
 // Forward unit: one item's key range restricted to one query tile.
@@ -49,6 +52,12 @@ struct FwdPair {
   int32_t pad;
 };
 
+// Block-sparse mask, per (query tile, key block of 128 keys of the sample):
+// mask_words words whose bit t says that token t of the tile attends keys of
+// the block (its anchor's mask bit is set and its anchor lies past the
+// block's first key). Word group of (tile mt, block kb) starts at
+// (mtiles[mt].mbase + kb) * mask_words.
+
 // Backward unit: one tile of <= 128 keys of one item, against every query
 // tile of the sample whose kmax exceeds kbeg. K/V, dK and dV coordinates as
 // for FwdUnit.
@@ -76,6 +85,10 @@ struct DevSection {
   uint64_t bwd_units;     // BwdUnit[n_bwd]
   uint64_t bwd_part_off;  // int32[n_queues + 1]
   uint64_t dead;          // int64[2 n_dead]: [begin, end) K/V rows whose dK/dV are zero
+  uint64_t tile_mask;     // uint32[n_tile_blocks * mask_words] (block-sparse mask only)
+  uint64_t pair_tile_off; // int32[n_fwd_pairs + 1]: live key tiles of every forward pair (mask only)
+  uint64_t unit_tile_off; // int32[n_fwd + 1]: live key tiles of every forward unit (mask only)
+  uint64_t live_tiles;    // int32[...]: first keys of those live key tiles, pairs' then units'
   uint64_t base_bytes;    // end of the arrays every call uploads; the ones below only the deterministic backward
   uint64_t bwd_rank;      // int32[n_bwd]: position of the unit's key tile among its (sample, kv head)'s, ascending
   uint64_t bwd_det_order; // int32[n_bwd]: units by (sample, rank, kv head), the deterministic dispatch order
@@ -94,6 +107,9 @@ struct PlanHeader {
   int32_t kv_heads;        // heads per row of the K/V (dK/dV) buffers: Hkv, or 1 for a shard
   int32_t n_dead;          // [begin, end) row ranges whose dK/dV are zero
   int32_t empty_slots;     // (query tile, kv head) slots without a forward unit (possible in a shard)
+  int32_t masked;          // block-sparse mask: 0 none; 1 the kernels can run; 2 items do not line up with
+                           // the mask's 128-key blocks (plan for costs and loads only, kernel calls refused)
+  int32_t mask_words;      // words per (tile, block): ceil(tile_tokens / 32)
   int64_t kv_rows;         // rows of the K/V (dK/dV) buffers: Ltot, or the shard's key count
   int64_t Nq, Ltot;
   int64_t total_cost;

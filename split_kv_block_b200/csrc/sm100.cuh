@@ -140,6 +140,34 @@ __device__ __forceinline__ void turn_pass(int32_t* turn, int next, int lane) {
   }
 }
 
+// ------------------------------------------------------- block-sparse mask
+// The mask word of (query tile M, key block starting at absolute key kb) that
+// holds token tl of the tile; bit tl % 32 says whether the token attends keys
+// of the block.
+template <class Tile>
+__device__ __forceinline__ uint32_t mask_word(const uint32_t* tile_mask, int mask_words, const Tile& M, int kb,
+                                              int tl) {
+  return tile_mask[static_cast<size_t>(M.mbase + ((kb - M.kbase) >> 7)) * mask_words + (tl >> 5)];
+}
+// Whether any token of tile M attends a key of the block starting at kb.
+template <class Tile>
+__device__ __forceinline__ bool mask_block_live(const uint32_t* tile_mask, int mask_words, const Tile& M, int kb) {
+  const uint32_t* w = tile_mask + static_cast<size_t>(M.mbase + ((kb - M.kbase) >> 7)) * mask_words;
+  uint32_t any = 0;
+  for (int i = 0; i < mask_words; ++i) any |= w[i];
+  return any != 0;
+}
+
+// Whether query tile M has a row that attends a key of the key tile starting
+// at kb (a backward unit's keys): some anchor of the tile lies past kb and,
+// with a block-sparse mask, some token's block is on. Every role of a
+// backward kernel walks the query tiles with this one test, so all of them
+// agree on the sequence.
+template <bool kMask, class Params, class Tile>
+__device__ __forceinline__ bool tile_live(const Params& p, const Tile& M, int kb) {
+  return M.kmax > kb && (!kMask || mask_block_live(p.tile_mask, p.mask_words, M, kb));
+}
+
 // ---------------------------------------------------------------------- TMA
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");

@@ -42,7 +42,8 @@ class _Problem(ctypes.Structure):
     _fields_ = [("num_samples", ctypes.c_int32), ("ctx_offsets", ctypes.c_void_p), ("anchor_offsets", ctypes.c_void_p),
                 ("anchors", ctypes.c_void_p), ("block_q", ctypes.c_int32), ("chunk_kv", ctypes.c_int32),
                 ("sub_chunks", ctypes.c_int32), ("num_partitions", ctypes.c_int32), ("num_q_heads", ctypes.c_int32),
-                ("num_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32)]
+                ("num_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32), ("key_block_mask", ctypes.c_void_p),
+                ("mask_stride", ctypes.c_int32)]
 
 
 ITEM_DTYPE = np.dtype([("b", np.int32), ("c", np.int32), ("g", np.int32), ("sub", np.int32),
@@ -122,9 +123,13 @@ class _ProblemArgs:
         self.ctx = np.ascontiguousarray(prob.ctx_offsets, dtype=np.int64)
         self.aoff = np.ascontiguousarray(prob.anchor_offsets, dtype=np.int32)
         self.anchors = np.ascontiguousarray(prob.anchors, dtype=np.int64)
+        m = getattr(prob, "key_block_mask", None)
+        self.mask = None if m is None else np.ascontiguousarray(m, dtype=np.uint8)
         self.s = _Problem(len(self.ctx) - 1, self.ctx.ctypes.data, self.aoff.ctypes.data,
                           self.anchors.ctypes.data if self.anchors.size else 0, prob.block_q, prob.chunk_kv,
-                          prob.sub_chunks, prob.num_partitions, prob.num_q_heads, prob.num_kv_heads, prob.head_dim)
+                          prob.sub_chunks, prob.num_partitions, prob.num_q_heads, prob.num_kv_heads, prob.head_dim,
+                          self.mask.ctypes.data if self.mask is not None and self.mask.size else 0,
+                          int(self.mask.shape[1]) if self.mask is not None else 0)
 
     def ref(self):
         return ctypes.byref(self.s)

@@ -51,6 +51,7 @@ class Workload:
     sub_chunks: int = 1
     backward: bool = True
     anchor_low: Optional[int] = None  # lower bound of the uniform range (default L // 8)
+    mask: Optional[str] = None        # "sink_window_random": block_mask_sink_window_random(seed) on top
 
 
 WORKLOADS = {
@@ -66,6 +67,10 @@ WORKLOADS = {
     "ctx128k": Workload("ctx128k", (131072,), 1, 64, "beta51", 32, 8, 128, 16, 4096, 64),
     # 8 samples, context lengths log-uniform in [8192, 262144], 128 anchors each.
     "batch8_logu": Workload("batch8_logu", None, 8, 128, "uniform", 32, 8, 128, 16, 4096, 128),
+    # the 32K shapes under a block-sparse mask: per anchor the first 2 key blocks of 128, the 4 blocks up
+    # to its own, and each other block with probability 1/4.
+    "ctx32k_sparse": Workload("ctx32k_sparse", (32768,), 1, 32, "uniform", 32, 8, 128, 16, 2048, 16,
+                              mask="sink_window_random"),
 }
 
 
@@ -128,10 +133,13 @@ def make_problem(w: Workload, seed: int = 0, *, sub_chunks: Optional[int] = None
     ctx_off[1:] = np.cumsum(lens)
     anc_off = np.zeros(len(lens) + 1, dtype=np.int32)
     anc_off[1:] = np.cumsum([len(a) for a in anchors])
-    return Problem(ctx_off, anc_off, np.concatenate(anchors).astype(np.int64), w.block_q, w.chunk_kv,
-                   w.sub_chunks if sub_chunks is None else sub_chunks,
-                   w.num_partitions if num_partitions is None else num_partitions,
-                   w.num_q_heads, w.num_kv_heads, w.head_dim)
+    p = Problem(ctx_off, anc_off, np.concatenate(anchors).astype(np.int64), w.block_q, w.chunk_kv,
+                w.sub_chunks if sub_chunks is None else sub_chunks,
+                w.num_partitions if num_partitions is None else num_partitions,
+                w.num_q_heads, w.num_kv_heads, w.head_dim)
+    if w.mask == "sink_window_random":
+        p = p.replace(key_block_mask=block_mask_sink_window_random(p, seed))
+    return p
 
 
 def redraw_anchors(p: Problem, w: Workload, seed: int) -> Problem:
@@ -139,7 +147,10 @@ def redraw_anchors(p: Problem, w: Workload, seed: int) -> Problem:
     rng = np.random.default_rng(seed)
     lens = np.diff(p.ctx_offsets)
     anchors = [draw_anchors(rng, int(L), w.anchors_per_sample, w.anchor_dist, w.anchor_low) for L in lens]
-    return p.replace(anchors=np.concatenate(anchors).astype(np.int64))
+    p = p.replace(anchors=np.concatenate(anchors).astype(np.int64))
+    if w.mask == "sink_window_random":
+        p = p.replace(key_block_mask=block_mask_sink_window_random(p, seed))
+    return p
 
 
 def randn_bf16(shape, seed: int, k: int) -> torch.Tensor:

@@ -16,7 +16,7 @@ import bench  # noqa: E402
 from split_kv_block_b200 import skv, synth  # noqa: E402
 
 
-@pytest.mark.parametrize("name", ["tiny_4k", "ctx32k"])
+@pytest.mark.parametrize("name", ["tiny_4k", "ctx32k", "ctx32k_sparse"])
 def test_flops_match_the_planners_unmasked_count(name):
     """4 d per unmasked (token, key, q-head) triple forward, 2.5x that backward; the
     planner counts the triples independently (its realized item costs)."""

@@ -55,6 +55,10 @@ def check_forward(prob, q, k, v, o, lse, groups=None):
         o, lse, prob = o[:, qh], lse[:, qh], sub
     O_ref, L_ref = A.attention_forward(prob, q, k, v)
     err_o = float((o.double() - O_ref).abs().max()) if o.numel() else 0.0
+    # rows that attend no key (possible under a block-sparse mask): LSE = -inf on both sides
+    none = torch.isneginf(L_ref)
+    assert torch.equal(torch.isneginf(lse), none), "rows without keys differ"
+    lse, L_ref = lse.double()[~none], L_ref[~none]
     err_l = float((lse.double() - L_ref).abs().max()) if lse.numel() else 0.0
     assert err_o <= O_TOL, f"O max-abs {err_o}"
     assert err_l <= LSE_TOL, f"LSE max-abs {err_l}"

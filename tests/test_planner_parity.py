@@ -244,3 +244,72 @@ def test_bf16_partials_flag_changes_only_the_partial_workspace():
     for bad in (2, 0x200, 0x101 | 0x400):
         with pytest.raises(skv.SkvError):
             skv.skv_plan_size(prob, bad)
+
+
+def _masked_problem(rng, density=0.5):
+    prob = synth.random_small_problem(rng, max_len=1500, max_anchors=6)
+    chunk = int(rng.choice([128, 256, 512]))
+    sub = int(rng.choice([s for s in (1, 2, 4) if (chunk // s) % 128 == 0]))
+    lens = np.diff(prob.ctx_offsets)
+    stride = int((lens.max() + 127) // 128) + int(rng.integers(0, 3))
+    mask = (rng.random((int(prob.anchor_offsets[-1]), stride)) < density).astype(np.uint8)
+    return prob.replace(chunk_kv=chunk, sub_chunks=sub, key_block_mask=mask)
+
+
+def test_block_mask_plans_bit_exact():
+    """Items, realized costs under a block-sparse mask, LPT partitions and
+    loads: bit-exact to the oracle planner on random masked problems, for the
+    LPT plan and for the static split (whose pieces cut blocks: partial blocks
+    counted key by key)."""
+    rng = np.random.default_rng(31)
+    for i in range(200):
+        prob = _masked_problem(rng)
+        _compare(prob, skv.SKV_PLAN_LPT)
+        if i % 4 == 0:
+            _compare(prob, skv.SKV_PLAN_STATIC)
+    for i in range(20):  # chunks that are not a multiple of 128 keys
+        prob = _masked_problem(rng).replace(chunk_kv=int(rng.choice([100, 320])), sub_chunks=1)
+        _compare(prob, skv.SKV_PLAN_LPT)
+    w = synth.WORKLOADS["ctx32k"]
+    prob = synth.make_problem(w, seed=0)
+    prob = prob.replace(key_block_mask=synth.block_mask_sink_window_random(prob, seed=0))
+    _compare(prob, skv.SKV_PLAN_LPT)
+
+
+def test_block_mask_refusals():
+    """Plans whose items do not start on 128-key blocks (the static split's
+    pieces, chunks that are not a multiple of 128 keys) are made for their
+    costs and loads, but every kernel call refuses them on the host
+    (SKV_EUNSUPPORTED); a mask row shorter than a sample's block count is
+    refused by the planner."""
+    rng = np.random.default_rng(4)
+    # one 1000-key sample on 3 partitions: the static split cuts at keys 333 and 666
+    prob = synth.small_problem([1000], [[999, 400, 100]], block_q=16, chunk_kv=256, num_partitions=3, hq=8, hkv=2,
+                               d=128)
+    prob = prob.replace(key_block_mask=(rng.random((3, 8)) < 0.6).astype(np.uint8))
+    f = _fake_dev()
+    L = skv.lib()
+    for plan in (skv.skv_plan(prob, skv.SKV_PLAN_STATIC), skv.skv_plan(prob.replace(chunk_kv=320, sub_chunks=1))):
+        pr = plan.prob_ref
+        assert L.skv_attn_fwd(plan.ptr, pr, f[0], f[1], f[2], f[3], 1 << 30, None) == 3
+        assert L.skv_attn_fwd_merged(plan.ptr, pr, f[0], f[1], f[2], f[4], f[5], f[3], 1 << 30, None) == 3
+        assert L.skv_lse_merge(plan.ptr, pr, f[3], f[4], f[5], None) == 3
+        assert L.skv_attn_bwd(plan.ptr, pr, *f[:7], f[7], f[0], f[1], 1 << 30, None) == 3
+        assert L.skv_attn_fwd_noalloc(plan.ptr, pr, f[0], f[1], f[2], f[3], f[4], None) == 3
+    lens = np.diff(prob.ctx_offsets)
+    short = prob.key_block_mask[:, :int((lens.max() + 127) // 128) - 1]
+    with pytest.raises(skv.SkvError) as e:
+        skv.skv_plan(prob.replace(key_block_mask=np.ascontiguousarray(short)))
+    assert e.value.code == 1
+
+
+def test_block_mask_changes_the_fingerprint():
+    """A plan made for one mask is refused with another mask of the same shape."""
+    rng = np.random.default_rng(6)
+    prob = _masked_problem(rng)
+    plan = skv.skv_plan(prob)
+    other = prob.key_block_mask.copy()
+    other[0, 0] ^= 1
+    f = _fake_dev()
+    pr = skv._ProblemArgs(prob.replace(key_block_mask=other)).ref()
+    assert skv.lib().skv_attn_fwd(plan.ptr, pr, f[0], f[1], f[2], f[3], 1 << 30, None) == 5
