@@ -65,9 +65,47 @@ def item_cost(prob, b: int, key_begin: int, key_end: int) -> int:
     return G * pairs
 
 
-def lpt_items(prob) -> List[Item]:
-    """All (b, c, g, s) items in (b, c, g, s) order, with their cost."""
+TILE_M = 128   # query rows per tile: 128 / G consecutive tokens x the G q-heads of a kv group
+TILE_N = 128   # keys per key tile
+
+
+def item_tile_cost(prob, b: int, key_begin: int, key_end: int) -> int:
+    """Cost calibrated to the work the kernels execute (a
+    refinement of the realized cost): the query rows of sample b are cut into
+    tiles of 128 / G consecutive tokens (G q-heads each, 128 rows), the item's
+    keys into tiles of 128 keys from key_begin; every (query tile, key tile)
+    block in which some token attends some key runs as a whole 128 x 128
+    block, so the cost is 128 * 128 per such block. Plain loops."""
+    G = prob.num_q_heads // prob.num_kv_heads
+    tt = TILE_M // G
+    S = prob.block_q
+    k0 = int(prob.ctx_offsets[b])
+    t_begin, t_end = int(prob.anchor_offsets[b]) * S, int(prob.anchor_offsets[b + 1]) * S
+    mask = getattr(prob, "key_block_mask", None)
+    blocks = 0
+    for t0 in range(t_begin, t_end, tt):
+        tokens = range(t0, min(t0 + tt, t_end))
+        for kb in range(key_begin, key_end, TILE_N):
+            ke = min(kb + TILE_N, key_end)
+            live = False
+            for tok in tokens:
+                j = tok // S
+                a = int(prob.anchors[j])
+                for kk in range(kb - k0, ke - k0):
+                    if kk < a and (mask is None or mask[j][kk // 128]):
+                        live = True
+                        break
+                if live:
+                    break
+            blocks += live
+    return TILE_M * TILE_N * blocks
+
+
+def lpt_items(prob, cost: str = "exact") -> List[Item]:
+    """All (b, c, g, s) items in (b, c, g, s) order, with their cost: the
+    realized attention cost ("exact") or the executed tile work ("tiles")."""
     C, sub = prob.chunk_kv, prob.sub_chunks
+    cost_fn = item_tile_cost if cost == "tiles" else item_cost
     cs = C // sub
     items = []
     for b in range(prob.num_samples):
@@ -80,7 +118,7 @@ def lpt_items(prob) -> List[Item]:
                     lo, hi = c * C + s * cs, min(c * C + (s + 1) * cs, c_end)
                     if hi <= lo:
                         continue
-                    items.append(Item(b, c, g, s, k0 + lo, k0 + hi, item_cost(prob, b, k0 + lo, k0 + hi)))
+                    items.append(Item(b, c, g, s, k0 + lo, k0 + hi, cost_fn(prob, b, k0 + lo, k0 + hi)))
     return items
 
 
@@ -103,9 +141,9 @@ def lpt_assign(costs: List[int], num_partitions: int, keys=None) -> List[int]:
     return part
 
 
-def lpt_plan(prob):
+def lpt_plan(prob, cost: str = "exact"):
     """Returns (items with partitions, partition loads)."""
-    items = lpt_items(prob)
+    items = lpt_items(prob, cost)
     part = lpt_assign([it.cost for it in items], prob.num_partitions,
                       keys=[(it.b, it.c, it.g, it.sub) for it in items])
     out = [Item(it.b, it.c, it.g, it.sub, it.key_begin, it.key_end, it.cost, p) for it, p in zip(items, part)]

@@ -178,3 +178,35 @@ def test_item_costs_with_a_block_mask_match_mask_count():
         prob = prob.replace(key_block_mask=mask)
         for it in PL.lpt_items(prob):
             assert it.cost == _mask_count(prob, it.b, it.key_begin, it.key_end)
+
+
+def test_tile_cost_hand_instance():
+    """One sample of 300 keys, anchors 100 and 260, block_q 16, 4 q-heads on
+    one kv head (G = 4): a query tile holds 32 tokens, i.e. both anchors (one
+    tile). Key tiles of the item [0, 300): [0,128) and [128,256) hold keys the
+    anchor 260 block attends, [256,300) holds key 256..259 for it: 3 live
+    blocks, 3 * 128 * 128. The item [200, 300) alone: key tiles [200,300) is
+    one tile, live (anchor 260): 1 block."""
+    prob = synth.small_problem([300], [[100, 260]], block_q=16, hq=4, hkv=1, d=64)
+    assert PL.item_tile_cost(prob, 0, 0, 300) == 3 * 128 * 128
+    assert PL.item_tile_cost(prob, 0, 200, 300) == 128 * 128
+    # anchors 100 and 120 only: the keys [128, 300) are attended by nobody
+    prob2 = prob.replace(anchors=np.array([100, 120]))
+    assert PL.item_tile_cost(prob2, 0, 0, 300) == 128 * 128
+
+
+def test_tile_cost_bounds_the_exact_cost():
+    """Every attended (row, key) pair lies in a live block, so the tile cost
+    is at least the exact cost, and at most 128 * 128 per key tile and query
+    tile of the sample."""
+    rng = np.random.default_rng(12)
+    for _ in range(20):
+        prob = synth.random_small_problem(rng, max_len=500)
+        G = prob.num_q_heads // prob.num_kv_heads
+        for it in PL.lpt_items(prob):
+            tc = PL.item_tile_cost(prob, it.b, it.key_begin, it.key_end)
+            assert tc >= it.cost
+            n_tok = (int(prob.anchor_offsets[it.b + 1]) - int(prob.anchor_offsets[it.b])) * prob.block_q
+            n_qt = -(-n_tok // (128 // G))
+            n_kt = -(-(it.key_end - it.key_begin) // 128)
+            assert tc <= 128 * 128 * n_qt * n_kt
