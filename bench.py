@@ -238,7 +238,7 @@ def run_workload(args, name, steps, warmup, rank, world, local_rank, e2e):
     q, k, v, do = synth.make_tensors(prob, seed=seed, backward=backward)
     q, k, v = q.to(dev), k.to(dev), v.to(dev)
     do = do.to(dev) if backward else None
-    policy = skv.SKV_PLAN_STATIC if args.policy == "static" else skv.SKV_PLAN_LPT
+    policy = {"static": skv.SKV_PLAN_STATIC, "lpt": skv.SKV_PLAN_LPT, "lpt_tiles": skv.SKV_PLAN_LPT_TILES}[args.policy]
     if args.partials == "bf16":
         policy |= skv.SKV_PLAN_PARTIALS_BF16
     redraw = name == "batch8_logu"
@@ -700,7 +700,7 @@ def main():
     ap.add_argument("--impl", default="skv", choices=["skv", "reference"])
     ap.add_argument("--workload", default="ctx32k", choices=sorted(synth.WORKLOADS))
     ap.add_argument("--seed", type=int, default=0)
-    ap.add_argument("--policy", default="lpt", choices=["lpt", "static"])
+    ap.add_argument("--policy", default="lpt", choices=["lpt", "static", "lpt_tiles"])
     ap.add_argument("--sub-chunks", type=int, default=None)
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--no-e2e", action="store_true")

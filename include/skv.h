@@ -65,6 +65,13 @@ enum skv_status_code {
 enum skv_plan_policy {
   SKV_PLAN_LPT = 0,    /* cost-aware LPT over (b, c, g, s) items ("LPT Scheduling") */
   SKV_PLAN_STATIC = 1, /* equal-token contiguous split, the baseline LPT replaces */
+  /* LPT with a cost calibrated to the executed work: query rows in tiles of
+   * 128 / G tokens x G heads, an item's keys in tiles of 128 from its start,
+   * and 128 * 128 per (query tile, key tile) block in which some token
+   * attends some key. Same items and tie-break as SKV_PLAN_LPT; the items'
+   * costs and the loads are in these units. Under a block mask it needs the
+   * items to start on 128-key blocks (SKV_EUNSUPPORTED otherwise). */
+  SKV_PLAN_LPT_TILES = 2,
   /* Flag, OR-ed into either policy: the forward stores each chunk's partial
    * output in bf16 instead of fp32 (the partial LSE stays fp32), halving the
    * partials' memory traffic and workspace. A partial output is a convex

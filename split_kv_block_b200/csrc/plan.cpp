@@ -93,6 +93,10 @@ struct SampleAnchors {
   // blocks before block kb (block_prefix[kb]); a key of block kb counts for anchor j when the mask allows
   // the block and the key lies before a_j
   std::vector<int64_t> block_prefix;
+  // executed-tile cost (SKV_PLAN_LPT_TILES): the largest anchor of every query tile of the sample, sorted;
+  // under a block mask, per 128-key block the number of query tiles with a token that attends it
+  std::vector<int64_t> tile_kmax_sorted;
+  std::vector<int32_t> live_tiles_of_block;
 };
 
 // sum_j max(0, min(hi, a_j) - lo), relative coordinates, lo < hi.
@@ -145,6 +149,19 @@ void make_items(const Prob& q, int policy, const std::vector<SampleAnchors>& sa,
     return n;
   };
   auto cost = [&](int b, int64_t lo_abs, int64_t hi_abs) {
+    if (policy == SKV_PLAN_LPT_TILES) {
+      // 128 x 128 per (query tile, key tile) block in which some token attends some key
+      int64_t blocks = 0;
+      for (int64_t kb = lo_abs - q.ctx[b]; kb < hi_abs - q.ctx[b]; kb += kTileN) {
+        if (q.mask) {
+          blocks += sa[b].live_tiles_of_block[kb / kTileN];
+        } else {
+          const auto& km = sa[b].tile_kmax_sorted;
+          blocks += km.end() - std::upper_bound(km.begin(), km.end(), kb);  // tiles whose largest anchor > kb
+        }
+      }
+      return blocks * kTileM * kTileN;
+    }
     if (q.mask) {
       // whole blocks from the per-block prefix sums, the partial blocks at either end anchor by anchor
       const int64_t lo = lo_abs - q.ctx[b], hi = hi_abs - q.ctx[b];
@@ -159,7 +176,7 @@ void make_items(const Prob& q, int policy, const std::vector<SampleAnchors>& sa,
     return static_cast<int64_t>(q.G) * q.S * pair_sum(sa[b], lo_abs - q.ctx[b], hi_abs - q.ctx[b]);
   };
   out.items.clear();
-  if (policy == SKV_PLAN_LPT) {
+  if (policy == SKV_PLAN_LPT || policy == SKV_PLAN_LPT_TILES) {
     const int64_t cs = q.C / q.sub;
     for (int b = 0; b < q.B; ++b) {
       const int64_t k0 = q.ctx[b], L = q.ctx[b + 1] - k0;
@@ -235,7 +252,7 @@ void place(const Prob& q, int policy, Built& out) {
   out.placement.resize(n);
   std::iota(out.placement.begin(), out.placement.end(), 0);
   out.load.assign(q.P, 0);
-  if (policy == SKV_PLAN_LPT) {
+  if (policy == SKV_PLAN_LPT || policy == SKV_PLAN_LPT_TILES) {
     // Items are generated in (b, c, g, s) order, so the index breaks ties.
     std::sort(out.placement.begin(), out.placement.end(), [&](int32_t x, int32_t y) {
       if (out.items[x].cost != out.items[y].cost) return out.items[x].cost > out.items[y].cost;
@@ -573,9 +590,8 @@ void make_lists(const Prob& q, const std::vector<SampleAnchors>& sa, int shard, 
 }
 
 int build(const skv_problem* prob, int policy, Built& out, Prob& q, int shard = -1) {
-  if ((policy & ~SKV_PLAN_PARTIALS_BF16) != SKV_PLAN_LPT && (policy & ~SKV_PLAN_PARTIALS_BF16) != SKV_PLAN_STATIC)
-    return SKV_EINVAL;
   policy &= ~SKV_PLAN_PARTIALS_BF16;
+  if (policy != SKV_PLAN_LPT && policy != SKV_PLAN_STATIC && policy != SKV_PLAN_LPT_TILES) return SKV_EINVAL;
   int rc = validate(prob, q);
   if (rc != SKV_OK) return rc;
   std::vector<SampleAnchors> sa(q.B);
@@ -599,6 +615,31 @@ int build(const skv_problem* prob, int policy, Built& out, Prob& q, int shard = 
           if (row[kb]) bp[kb + 1] += std::min<int64_t>(a, (kb + 1) * kTileN) - kb * kTileN;
       }
       for (int64_t kb = 0; kb < nkb; ++kb) bp[kb + 1] += bp[kb];
+    }
+  }
+  if (policy == SKV_PLAN_LPT_TILES) {
+    if (q.mask && (q.C % kTileN != 0 || (q.C / q.sub) % kTileN != 0)) return SKV_EUNSUPPORTED;
+    for (int b = 0; b < q.B; ++b) {
+      const int64_t t_begin = static_cast<int64_t>(q.aoff[b]) * q.S, t_end = static_cast<int64_t>(q.aoff[b + 1]) * q.S;
+      const int64_t nkb = (q.ctx[b + 1] - q.ctx[b] + kTileN - 1) / kTileN;
+      auto& km = sa[b].tile_kmax_sorted;
+      km.clear();
+      sa[b].live_tiles_of_block.assign(q.mask ? nkb : 0, 0);
+      for (int64_t t0 = t_begin; t0 < t_end; t0 += q.TT) {
+        const int64_t t1 = std::min<int64_t>(t0 + q.TT, t_end);
+        int64_t amax = 0;
+        for (int64_t j = t0 / q.S; j <= (t1 - 1) / q.S; ++j) amax = std::max(amax, q.anchors[j]);
+        km.push_back(amax);
+        if (q.mask) {
+          for (int64_t kb = 0; kb < nkb; ++kb) {
+            bool live = false;
+            for (int64_t j = t0 / q.S; j <= (t1 - 1) / q.S && !live; ++j)
+              live = q.mask[static_cast<size_t>(j) * q.mask_stride + kb] && q.anchors[j] > kb * kTileN;
+            sa[b].live_tiles_of_block[kb] += live;
+          }
+        }
+      }
+      std::sort(km.begin(), km.end());
     }
   }
   make_items(q, policy, sa, out);

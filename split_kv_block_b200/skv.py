@@ -19,6 +19,7 @@ LIB_PATH = os.path.join(HERE, "libskv.so")
 
 SKV_PLAN_LPT = 0
 SKV_PLAN_STATIC = 1
+SKV_PLAN_LPT_TILES = 2          # LPT on the executed-tile cost (see include/skv.h)
 SKV_PLAN_PARTIALS_BF16 = 0x100  # flag: bf16 partial outputs (see include/skv.h)
 
 # Every function include/skv.h declares.

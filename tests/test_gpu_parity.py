@@ -249,3 +249,12 @@ def test_bf16_partials(fused):
         q, k, v, _ = synth.make_tensors(prob, seed=3, backward=False)
         o, lse, _, _ = run_gpu(prob, q, k, v, None, skv.SKV_PLAN_LPT | flag, fused)
         check_forward(prob, q, k, v, o, lse, groups)
+
+
+def test_tile_cost_plans():
+    """Plans placed on the executed-tile cost run the same kernels: the tiny
+    workload and a ragged problem, forward and backward."""
+    _case(synth.make_problem(synth.WORKLOADS["tiny_4k"], seed=2), seed=2, policy=skv.SKV_PLAN_LPT_TILES)
+    prob = synth.small_problem([1001, 777, 1500], [[1000, 3, 555], [777], [1, 1499, 700, 64, 1200]], block_q=16,
+                               chunk_kv=320, num_partitions=4, hq=8, hkv=2, d=128)
+    _case(prob, seed=6, policy=skv.SKV_PLAN_LPT_TILES)

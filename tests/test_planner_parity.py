@@ -16,6 +16,8 @@ def _compare(prob, policy):
     got = plan.items()
     if policy == skv.SKV_PLAN_LPT:
         ref, loads = PL.lpt_plan(prob)
+    elif policy == skv.SKV_PLAN_LPT_TILES:
+        ref, loads = PL.lpt_plan(prob, cost="tiles")
     else:
         ref, loads = PL.static_plan(prob)
     assert len(got) == len(ref)
@@ -241,7 +243,7 @@ def test_bf16_partials_flag_changes_only_the_partial_workspace():
     assert a.sizes.ws_bwd_bytes == b.sizes.ws_bwd_bytes
     st = skv.skv_plan(prob, skv.SKV_PLAN_STATIC | skv.SKV_PLAN_PARTIALS_BF16)
     assert np.array_equal(st.items(), skv.skv_plan(prob, skv.SKV_PLAN_STATIC).items())
-    for bad in (2, 0x200, 0x101 | 0x400):
+    for bad in (3, 0x200, 0x101 | 0x400):
         with pytest.raises(skv.SkvError):
             skv.skv_plan_size(prob, bad)
 
@@ -313,3 +315,28 @@ def test_block_mask_changes_the_fingerprint():
     f = _fake_dev()
     pr = skv._ProblemArgs(prob.replace(key_block_mask=other)).ref()
     assert skv.lib().skv_attn_fwd(plan.ptr, pr, f[0], f[1], f[2], f[3], 1 << 30, None) == 5
+
+
+
+def test_tile_cost_plans_bit_exact():
+    """SKV_PLAN_LPT_TILES (LPT on the executed-tile cost): items, costs,
+    partitions and loads bit-exact to the oracle, on the tiny workload and on
+    random problems with and without block masks."""
+    _compare(synth.make_problem(synth.WORKLOADS["tiny_4k"], seed=0), skv.SKV_PLAN_LPT_TILES)
+    rng = np.random.default_rng(77)
+    for i in range(60):
+        prob = synth.random_small_problem(rng, max_len=600)
+        if i % 3 == 0:
+            prob = _masked_problem(rng)
+            prob = prob.replace(ctx_offsets=prob.ctx_offsets)  # aligned chunks from _masked_problem
+        _compare(prob, skv.SKV_PLAN_LPT_TILES)
+
+
+def test_tile_cost_at_least_the_exact_cost_on_the_workloads():
+    """On the benchmark workloads the executed tile work exceeds the attended
+    work by the tile rounding (and the two anchors that share a query tile)."""
+    for name in ("ctx32k", "ctx128k", "batch8_logu"):
+        prob = synth.make_problem(synth.WORKLOADS[name], seed=0)
+        exact = skv.skv_plan(prob).stats()["total_cost"]
+        tiles = skv.skv_plan(prob, skv.SKV_PLAN_LPT_TILES).stats()["total_cost"]
+        assert exact <= tiles <= 1.2 * exact
