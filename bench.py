@@ -356,6 +356,7 @@ def run_workload(args, name, steps, warmup, rank, world, local_rank, e2e):
     static = skv.skv_plan(p0, skv.SKV_PLAN_STATIC).stats()["imbalance"]
 
     realized = realized_busy_imbalance(skv, p0, policy, q, k, v, do, ws, o, lse, dq, dk, dv, stream, dev, fused)
+    lpt_device = device_lpt_us(skv, p0, policy, dev, stream)
 
     peaks = load_peaks()
     kms = {kid: statistics.mean(t) for kid, t in t_kern.items()}
@@ -399,6 +400,7 @@ def run_workload(args, name, steps, warmup, rank, world, local_rank, e2e):
         "context_tokens_per_s": round(ctx_tokens / total, 1),
         "imbalance": {"lpt": lpt, "static": static, "realized": realized},
         "planner_us": round(statistics.median(planner_s) * 1e6, 1),
+        "lpt_device_us": lpt_device,
         "gpu_launches": kernels_per_step * K,
         "clocks": clocks.summary(),
     }
@@ -420,6 +422,7 @@ def run_gpu(args, rank, world, local_rank):
                    "parallelism": f"replicas x{world}" if world > 1 else "1 GPU, P virtual partitions"},
     }
     for key in ("roofline", "kernels", "kernel_ms", "merge", "context_tokens_per_s", "imbalance", "planner_us",
+                "lpt_device_us",
                 "gpu_launches", "clocks", "e2e"):
         if key in rec:
             out[key] = rec[key]
@@ -433,6 +436,31 @@ def run_gpu(args, rank, world, local_rank):
             r, _ = run_workload(args, name, min(args.steps, 20), args.warmup, rank, world, local_rank, False)
             out["workloads"][name] = r
     return out, prob
+
+
+def device_lpt_us(skv, prob, policy, dev, stream):
+    """The LPT placement of the step plan's items on the GPU (skv_lpt_place_device,
+    one CTA), median of 10 launches timed with CUDA events on the launch stream;
+    checked against the host plan's partitions. None beyond its size limits."""
+    plan = skv.skv_plan(prob, policy)
+    it = plan.items()
+    P = prob.num_partitions
+    if len(it) > 16384 or P > 4096 or (policy & 0xff) == skv.SKV_PLAN_STATIC:
+        return None
+    costs = torch.from_numpy(it["cost"].astype(np.int64)).to(dev)
+    part = torch.empty(len(it), dtype=torch.int32, device=dev)
+    loads = torch.empty(P, dtype=torch.int64, device=dev)
+    times = []
+    for _ in range(12):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        skv.skv_lpt_place_device(costs, P, part, loads, stream)
+        b.record(stream)
+        b.synchronize()
+        times.append(a.elapsed_time(b) * 1e3)
+    if not np.array_equal(part.cpu().numpy(), it["partition"]):
+        raise RuntimeError("device LPT placement differs from the host plan")
+    return round(statistics.median(times[2:]), 1)
 
 
 def realized_busy_imbalance(skv, prob, policy, q, k, v, do, ws, o, lse, dq, dk, dv, stream, dev, fused=True):
