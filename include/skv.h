@@ -178,6 +178,28 @@ int skv_plan_shard(const skv_problem* prob, int policy, int partition, void* pla
  * for a full plan). Any pointer may be NULL. */
 int skv_plan_kv_layout(const void* plan, int64_t* kv_rows, int32_t* kv_heads, int32_t* shard);
 
+/* Limits of skv_lpt_place_device (one CTA, its shared memory). */
+#define SKV_LPT_DEVICE_MAX_ITEMS 16384
+#define SKV_LPT_DEVICE_MAX_PARTITIONS 4096
+
+/*
+ * skv_lpt_place_device — the LPT placement of skv_plan computed on the GPU
+ * ("Split-KV: Breaking the Context Parallelism Bottleneck in Diffusion
+ * Drafter Training", section "LPT Scheduling": longest first onto the
+ * least-loaded partition; planned every step), for callers whose item costs
+ * are on the device. costs: device int64 [n_items] (>= 0), items in the order
+ * whose index breaks ties (skv_plan's (b, c, g, sub) order); writes partition
+ * (device int32 [n_items]) and loads (device int64 [n_partitions]). Items go
+ * longest first, ties by lower index, each to the partition with the smallest
+ * (load, index): the same bits as skv_plan's partitions and partition loads.
+ * One CTA (a bitonic sort in shared memory, then one warp places the items).
+ * SKV_EUNSUPPORTED beyond SKV_LPT_DEVICE_MAX_ITEMS items or
+ * SKV_LPT_DEVICE_MAX_PARTITIONS partitions; SKV_EINVAL for NULL pointers or
+ * n_partitions < 1. Enqueued on `stream`.
+ */
+int skv_lpt_place_device(const int64_t* costs, int64_t n_items, int32_t n_partitions, int32_t* partition,
+                         int64_t* loads, skv_stream_t stream);
+
 /* Items of a plan in (b, c, g, sub) order; *items points into `plan`. */
 int skv_plan_items(const void* plan, const skv_item** items, size_t* n_items);
 

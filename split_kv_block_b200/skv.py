@@ -28,7 +28,7 @@ EXPORTS = ("skv_plan_size", "skv_plan", "skv_plan_items", "skv_plan_unit_partiti
            "skv_attn_bwd", "skv_attn_bwd_deterministic", "skv_status", "skv_strerror", "skv_last_cuda_error", "skv_set_unit_timer",
            "skv_set_timing_events", "skv_attn_fwd_noalloc", "skv_noalloc_status", "skv_wait_selftest",
            "skv_plan_shard_size", "skv_plan_shard", "skv_plan_kv_layout", "skv_attn_bwd_partial", "skv_lse_combine",
-           "skv_dq_combine")
+           "skv_dq_combine", "skv_lpt_place_device")
 SKV_NOALLOC_SCRATCH_BYTES = 32 << 20
 SKV_KERNEL_FWD, SKV_KERNEL_MERGE, SKV_KERNEL_BWD = 0, 1, 2
 
@@ -87,6 +87,7 @@ def lib() -> ctypes.CDLL:
         L.skv_attn_bwd_partial.argtypes = [vp] * 12 + [sz, vp]
         L.skv_lse_combine.argtypes = [vp, vp, ctypes.c_int, ctypes.c_int64, ctypes.c_int, vp, vp, vp]
         L.skv_dq_combine.argtypes = [vp, ctypes.c_int, ctypes.c_int64, vp, vp]
+        L.skv_lpt_place_device.argtypes = [vp, ctypes.c_int64, ctypes.c_int32, vp, vp, vp]
         for name in EXPORTS:
             if name not in ("skv_strerror",):
                 getattr(L, name).restype = ctypes.c_int
@@ -315,6 +316,13 @@ def skv_dq_combine(dq_parts, dq, stream=None):
     n_parts = int(dq_parts.shape[0])
     _check("skv_dq_combine", lib().skv_dq_combine(_ptr(dq_parts), n_parts, int(dq_parts.numel() // n_parts), _ptr(dq),
                                                   _stream_ptr(stream)))
+
+
+def skv_lpt_place_device(costs, n_partitions: int, partition, loads, stream=None):
+    """LPT placement on the GPU: costs int64 [n] (device), partition int32 [n]
+    and loads int64 [P] (device outputs); the same bits as skv_plan's."""
+    _check("skv_lpt_place_device", lib().skv_lpt_place_device(_ptr(costs), int(costs.numel()), int(n_partitions),
+                                                              _ptr(partition), _ptr(loads), _stream_ptr(stream)))
 
 
 def skv_status(ws, stream=None) -> int:
