@@ -138,3 +138,35 @@ def test_two_gloo_ranks_exchange_and_merge_equal_the_unsplit_oracle(tmp_path):
             dv[kb:ke, g] = res[r]["dv"][kb:ke, g]
     assert torch.all(owner == 1)
     assert torch.allclose(dk, gk, atol=1e-11, rtol=0) and torch.allclose(dv, gv, atol=1e-11, rtol=0)
+
+
+def test_shard_layout_of_every_rank():
+    """The shard plans of all ranks: each rank's K/V rows are its items' keys
+    (one kv head per row) in (b, c, g, s) order, cp.shard_kv places exactly
+    those rows, and the ranks' rows together hold every (key, kv head) once."""
+    import sys
+    sys.path.insert(0, ROOT)
+    from split_kv_block_b200 import cp, skv, synth
+    prob = synth.small_problem([700, 390, 128], [[650, 129, 300], [390, 200], [128]], block_q=16, chunk_kv=128,
+                               sub_chunks=2, num_partitions=3, hq=8, hkv=2, d=64)
+    _, k, _, _ = synth.make_tensors(prob, seed=1, backward=False)
+    seen = torch.zeros(k.shape[0], k.shape[1], dtype=torch.int32)
+    for r in range(prob.num_partitions):
+        plan = skv.skv_plan_shard(prob, r)
+        rows, heads, shard = plan.kv_layout()
+        assert heads == 1 and shard == r
+        ks = cp.shard_kv(plan, k)
+        assert tuple(ks.shape) == (rows, 1, k.shape[-1])
+        it = plan.items()
+        mine = it[it["partition"] == r]
+        assert (it["kv_row"][it["partition"] != r] == -1).all()
+        order = np.lexsort((mine["sub"], mine["g"], mine["c"], mine["b"]))
+        row = 0
+        for i in order:
+            g, kb, ke = int(mine["g"][i]), int(mine["key_begin"][i]), int(mine["key_end"][i])
+            assert int(mine["kv_row"][i]) == row
+            assert torch.equal(ks[row:row + ke - kb, 0], k[kb:ke, g])
+            seen[kb:ke, g] += 1
+            row += ke - kb
+        assert row == rows
+    assert torch.all(seen == 1)
