@@ -148,9 +148,11 @@ def kernel_digest(kernel):
     return h.hexdigest()[:16]
 
 
-def profiled_traffic(kernel, workload):
+def profiled_traffic(kernel, workload, setup=None):
     """DRAM bytes (read + write) per launch from the committed ncu summary,
-    or None when the kernel's sources changed since that capture."""
+    or None when the kernel's sources changed since that capture, or when the
+    run's setup (policy, partials, queues, merge, sub-chunks) differs from the
+    captured one."""
     path = os.path.join(ROOT, "profiles", "dram_traffic.json")
     try:
         with open(path) as f:
@@ -158,6 +160,8 @@ def profiled_traffic(kernel, workload):
     except (OSError, ValueError):
         return None
     if not rec or rec.get("source_digest") != kernel_digest(kernel):
+        return None
+    if setup is not None and rec.get("setup") is not None and rec["setup"] != setup:
         return None
     return rec.get("dram_bytes_per_launch")
 
@@ -241,8 +245,13 @@ def run_workload(args, name, steps, warmup, rank, world, local_rank, e2e):
     policy = {"static": skv.SKV_PLAN_STATIC, "lpt": skv.SKV_PLAN_LPT, "lpt_tiles": skv.SKV_PLAN_LPT_TILES}[args.policy]
     if args.partials == "bf16":
         policy |= skv.SKV_PLAN_PARTIALS_BF16
+    if args.queues == "one":
+        policy |= skv.SKV_PLAN_ONE_QUEUE
     redraw = name == "batch8_logu"
     fused = args.fused_merge  # the merge in the forward kernel's tail, or its own launch (default: faster here)
+    # what a DRAM-traffic capture of this workload must have run with to stand for this run
+    setup = {"policy": args.policy, "partials": args.partials, "queues": args.queues,
+             "merge": "fused" if fused else "separate", "sub_chunks": prob.sub_chunks}
 
     # anchors of every step (the batched workload redraws them each step)
     step_probs = [synth.redraw_anchors(prob, w, seed * 1000 + i) if redraw else prob for i in range(warmup + steps)]
@@ -367,7 +376,7 @@ def run_workload(args, name, steps, warmup, rank, world, local_rank, e2e):
                 "unit": "TFLOP/s", "frac": round(a / peaks["bf16_tflops"], 4),
                 "frac_of_sustained": (round(a / peaks["bf16_tflops_sustained"], 4)
                                       if peaks.get("bf16_tflops_sustained") else None),
-                "traffic": profiled_traffic(kernel, name),
+                "traffic": profiled_traffic(kernel, name, setup),
                 "peak_source": f"{peaks['source']} bf16 dense (burst)"}
 
     kernels = {"fwd": tensor_roof("fwd_kernel", f_fwd_all / K, kms[skv.SKV_KERNEL_FWD])}
@@ -377,7 +386,7 @@ def run_workload(args, name, steps, warmup, rank, world, local_rank, e2e):
         m_gbs = mbytes_all / K / kms[skv.SKV_KERNEL_MERGE] / 1e9
         kernels["merge"] = {"bound": "hbm", "kernel": "merge_kernel", "achieved": round(m_gbs, 1),
                             "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(m_gbs / peaks["hbm_gbs"], 4),
-                            "traffic": profiled_traffic("merge_kernel", name),
+                            "traffic": profiled_traffic("merge_kernel", name, setup),
                             "peak_source": f"{peaks['source']} HBM copy"}
     if backward:
         kernels["bwd"] = tensor_roof("bwd_kernel", f_bwd_all / K, kms[skv.SKV_KERNEL_BWD])
@@ -388,7 +397,7 @@ def run_workload(args, name, steps, warmup, rank, world, local_rank, e2e):
     rec = {
         "workload": f"{name}: {WORKLOAD_TEXT[name]}", "value": round(value, 3), "unit": "TFLOP/s", "steps": K,
         "warmup": warmup, "ms_per_step": round(total / K * 1e3, 4), "seed": args.seed, "policy": args.policy,
-        "sub_chunks": prob.sub_chunks, "partials": args.partials,
+        "sub_chunks": prob.sub_chunks, "partials": args.partials, "queues": args.queues,
         "l2": (f"inputs larger than L2 (K+V {kv_bytes / 2**20:.0f} MiB > 126 MB): no flush, {K} steps back "
                "to back between two events, host planning of the next step overlapping the GPU")
               if stream_mode else "flushed before every step (256 MiB write outside the step's event window)",
@@ -418,7 +427,8 @@ def run_gpu(args, rank, world, local_rank):
         "warmup": rec["warmup"], "ms_per_step": rec["ms_per_step"], "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": rec["workload"], "seed": args.seed, "policy": args.policy,
-                   "sub_chunks": rec["sub_chunks"], "partials": rec["partials"], "l2": rec["l2"],
+                   "sub_chunks": rec["sub_chunks"], "partials": rec["partials"], "queues": rec["queues"],
+                   "l2": rec["l2"],
                    "parallelism": f"replicas x{world}" if world > 1 else "1 GPU, P virtual partitions"},
     }
     for key in ("roofline", "kernels", "kernel_ms", "merge", "context_tokens_per_s", "imbalance", "planner_us",
@@ -440,8 +450,10 @@ def run_gpu(args, rank, world, local_rank):
 
 def device_lpt_us(skv, prob, policy, dev, stream):
     """The LPT placement of the step plan's items on the GPU (skv_lpt_place_device,
-    one CTA), median of 10 launches timed with CUDA events on the launch stream;
-    checked against the host plan's partitions. None beyond its size limits."""
+    one CTA): device time per launch, 20 launches back to back between two CUDA
+    events on the launch stream, queued behind a 1 ms spin so that no host
+    latency falls between them; median of 5 such runs. Checked against the
+    host plan's partitions. None beyond its size limits."""
     plan = skv.skv_plan(prob, policy)
     it = plan.items()
     P = prob.num_partitions
@@ -450,17 +462,21 @@ def device_lpt_us(skv, prob, policy, dev, stream):
     costs = torch.from_numpy(it["cost"].astype(np.int64)).to(dev)
     part = torch.empty(len(it), dtype=torch.int32, device=dev)
     loads = torch.empty(P, dtype=torch.int64, device=dev)
+    skv.skv_lpt_place_device(costs, P, part, loads, stream)  # warm-up
     times = []
-    for _ in range(12):
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        skv.skv_lpt_place_device(costs, P, part, loads, stream)
-        b.record(stream)
-        b.synchronize()
-        times.append(a.elapsed_time(b) * 1e3)
+    with torch.cuda.stream(stream):
+        for _ in range(5):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            torch.cuda._sleep(2_000_000)
+            a.record(stream)
+            for _ in range(20):
+                skv.skv_lpt_place_device(costs, P, part, loads, stream)
+            b.record(stream)
+            b.synchronize()
+            times.append(a.elapsed_time(b) * 1e3 / 20)
     if not np.array_equal(part.cpu().numpy(), it["partition"]):
         raise RuntimeError("device LPT placement differs from the host plan")
-    return round(statistics.median(times[2:]), 1)
+    return round(statistics.median(times), 1)
 
 
 def realized_busy_imbalance(skv, prob, policy, q, k, v, do, ws, o, lse, dq, dk, dv, stream, dev, fused=True):
@@ -734,6 +750,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extra", action="store_true", help="time the headline workload only")
+    ap.add_argument("--queues", default="partition", choices=["partition", "one"],
+                    help="work queues of the kernels: one per partition, or one for all (SKV_PLAN_ONE_QUEUE)")
     ap.add_argument("--partials", default="fp32", choices=["fp32", "bf16"],
                     help="storage of the per-chunk partial outputs between the forward and the merge")
     ap.add_argument("--fused-merge", action="store_true",

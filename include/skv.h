@@ -79,7 +79,16 @@ enum skv_plan_policy {
    * the largest |V| to the merged output (about 1.1e-2 for N(0,1) values)
    * and nothing to the LSE. skv_plan_size, the forward and the merge read
    * the format from the plan. */
-  SKV_PLAN_PARTIALS_BF16 = 0x100
+  SKV_PLAN_PARTIALS_BF16 = 0x100,
+  /* Flag, OR-ed into any policy: the kernels of a full plan take their work
+   * units from one queue that holds every item in placement order (costliest
+   * first, each item's units together) instead of one queue per partition.
+   * The items, costs, partitions and loads do not change. On one GPU the
+   * CTAs that share a queue run neighbouring units at the same time, so an
+   * item's K/V tiles are read by many CTAs while they are in L2 rather than
+   * by the few CTAs of one partition, one after another. A shard plan always
+   * has one queue. */
+  SKV_PLAN_ONE_QUEUE = 0x200
 };
 
 /* One split-KV problem. Host pointers; read during the call only. */

@@ -282,12 +282,13 @@ void place(const Prob& q, int policy, Built& out) {
   out.imbalance = out.total_cost > 0 ? static_cast<double>(mx) * q.P / static_cast<double>(out.total_cost) - 1.0 : 0.0;
 }
 
-// shard < 0: the full plan: every partition's items on P work queues; the
+// shard < 0: the full plan: every partition's items on P work queues (one
+// queue holding all items in placement order with `one_queue`); the
 // K/V buffers are the packed context, all kv heads per row. shard = p: the
 // items of partition p only, on one work queue; the K/V buffers hold those
 // items' keys, one kv head per row, items in (b, c, g, s) order (the layout a
 // context-parallel rank keeps of its own chunks).
-void make_lists(const Prob& q, const std::vector<SampleAnchors>& sa, int shard, Built& out) {
+void make_lists(const Prob& q, const std::vector<SampleAnchors>& sa, int shard, bool one_queue, Built& out) {
   // query tiles
   out.mtiles.clear();
   out.sample_mt.assign(q.B + 1, 0);
@@ -341,8 +342,9 @@ void make_lists(const Prob& q, const std::vector<SampleAnchors>& sa, int shard, 
   };
 
   // K/V rows of every item, and the items each work queue runs in placement order
+  const bool per_partition = shard < 0 && !one_queue;
   out.shard = shard;
-  out.n_queues = shard < 0 ? q.P : 1;
+  out.n_queues = per_partition ? q.P : 1;
   out.kv_heads = shard < 0 ? q.Hkv : 1;
   std::vector<char> in_plan(out.items.size(), shard < 0 ? 1 : 0);
   if (shard < 0) {
@@ -364,7 +366,7 @@ void make_lists(const Prob& q, const std::vector<SampleAnchors>& sa, int shard, 
   }
   std::vector<std::vector<int32_t>> by_queue(out.n_queues);
   for (int32_t id : out.placement)
-    if (in_plan[id]) by_queue[shard < 0 ? out.items[id].partition : 0].push_back(id);
+    if (in_plan[id]) by_queue[per_partition ? out.items[id].partition : 0].push_back(id);
 
   out.fwd.clear();
   out.unit_live.clear();
@@ -590,7 +592,8 @@ void make_lists(const Prob& q, const std::vector<SampleAnchors>& sa, int shard, 
 }
 
 int build(const skv_problem* prob, int policy, Built& out, Prob& q, int shard = -1) {
-  policy &= ~SKV_PLAN_PARTIALS_BF16;
+  const bool one_queue = (policy & SKV_PLAN_ONE_QUEUE) != 0;
+  policy &= ~(SKV_PLAN_PARTIALS_BF16 | SKV_PLAN_ONE_QUEUE);
   if (policy != SKV_PLAN_LPT && policy != SKV_PLAN_STATIC && policy != SKV_PLAN_LPT_TILES) return SKV_EINVAL;
   int rc = validate(prob, q);
   if (rc != SKV_OK) return rc;
@@ -653,7 +656,7 @@ int build(const skv_problem* prob, int policy, Built& out, Prob& q, int shard = 
     // plan (costs, loads, imbalance) only: no work lists, the kernel calls refuse such a plan
     for (auto& it : out.items) it.kv_row = shard < 0 ? it.key_begin : -1;
     out.shard = shard;
-    out.n_queues = shard < 0 ? q.P : 1;
+    out.n_queues = shard < 0 && !one_queue ? q.P : 1;
     out.kv_heads = shard < 0 ? q.Hkv : 1;
     out.kv_rows = 0;
     out.mtiles.clear();
@@ -678,7 +681,7 @@ int build(const skv_problem* prob, int policy, Built& out, Prob& q, int shard = 
     out.dead.clear();
     return SKV_OK;
   }
-  make_lists(q, sa, shard, out);
+  make_lists(q, sa, shard, one_queue, out);
   return SKV_OK;
 }
 

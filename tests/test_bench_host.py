@@ -72,6 +72,17 @@ def test_traffic_is_reported_only_for_the_captured_sources(tmp_path, monkeypatch
     assert bench.profiled_traffic("fwd_kernel", "ctx32k") is None
 
 
+def test_traffic_is_reported_only_for_the_captured_setup(tmp_path, monkeypatch):
+    digest = bench.kernel_digest("fwd_kernel")
+    setup = {"policy": "lpt", "partials": "fp32", "queues": "partition", "merge": "separate", "sub_chunks": 1}
+    root = _fake_root(tmp_path, {"fwd_kernel": {"ctx32k": {"source_digest": digest, "dram_bytes_per_launch": 5,
+                                                           "setup": setup}}})
+    monkeypatch.setattr(bench, "ROOT", root)
+    assert bench.profiled_traffic("fwd_kernel", "ctx32k", dict(setup)) == 5
+    for key, other in (("partials", "bf16"), ("queues", "one"), ("merge", "fused"), ("sub_chunks", 4)):
+        assert bench.profiled_traffic("fwd_kernel", "ctx32k", {**setup, key: other}) is None
+
+
 def test_digest_follows_every_listed_source(tmp_path, monkeypatch):
     """Editing any file of a kernel's source list changes its digest."""
     src = tmp_path / "split_kv_block_b200" / "csrc"

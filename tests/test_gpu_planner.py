@@ -55,3 +55,41 @@ def test_device_lpt_edge_cases():
             ref[i] = p
             ld[p] += costs[i]
         assert part.cpu().tolist() == ref and loads.cpu().tolist() == ld
+
+
+def _host_lpt(costs, P):
+    """Sorted by (cost desc, index); each item to the smallest (load, partition)."""
+    import heapq
+    heap = [(0, p) for p in range(P)]
+    part = [0] * len(costs)
+    for i in sorted(range(len(costs)), key=lambda i: (-costs[i], i)):
+        ld, p = heapq.heappop(heap)
+        part[i] = p
+        heapq.heappush(heap, (ld + costs[i], p))
+    loads = [0] * P
+    for ld, p in heap:
+        loads[p] = ld
+    return part, loads
+
+
+@pytest.mark.parametrize("n,P,scale", [(0, 3, 10), (1000, 1, 10), (1000, 17, 10), (777, 33, 10**6), (2000, 64, 3),
+                                       (1248, 128, 10**9), (3000, 129, 10**9), (16384, 1000, 10**4),
+                                       (5000, 4096, 10**7), (300, 40, 2**50), (300, 200, 2**60)])
+def test_device_lpt_every_path(n, P, scale):
+    """Every placement path of the kernel: keys packed with the loads in
+    registers (up to 32, 64 and 128 partitions) or in shared memory (more
+    partitions), and unpacked when a cost or the costs' sum reaches 2^51;
+    the item and partition limits; random costs with many ties."""
+    rng = np.random.default_rng(n * 7 + P)
+    costs = rng.integers(0, scale, size=n, dtype=np.int64) if n else np.zeros(0, dtype=np.int64)
+    c = torch.from_numpy(costs).cuda() if n else torch.zeros(1, dtype=torch.int64, device="cuda")
+    part = torch.full((max(n, 1),), -1, dtype=torch.int32, device="cuda")
+    loads = torch.empty(P, dtype=torch.int64, device="cuda")
+    L = skv.lib()
+    import ctypes
+    assert L.skv_lpt_place_device(ctypes.c_void_p(c.data_ptr()), n, P, ctypes.c_void_p(part.data_ptr()),
+                                  ctypes.c_void_p(loads.data_ptr()), None) == 0
+    torch.cuda.synchronize()
+    ref_part, ref_loads = _host_lpt(costs.tolist(), P)
+    assert part.cpu().tolist()[:n] == ref_part
+    assert loads.cpu().tolist() == ref_loads

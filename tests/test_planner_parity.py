@@ -243,7 +243,7 @@ def test_bf16_partials_flag_changes_only_the_partial_workspace():
     assert a.sizes.ws_bwd_bytes == b.sizes.ws_bwd_bytes
     st = skv.skv_plan(prob, skv.SKV_PLAN_STATIC | skv.SKV_PLAN_PARTIALS_BF16)
     assert np.array_equal(st.items(), skv.skv_plan(prob, skv.SKV_PLAN_STATIC).items())
-    for bad in (3, 0x200, 0x101 | 0x400):
+    for bad in (3, 0x400, 0x101 | 0x800):
         with pytest.raises(skv.SkvError):
             skv.skv_plan_size(prob, bad)
 
@@ -340,3 +340,22 @@ def test_tile_cost_at_least_the_exact_cost_on_the_workloads():
         exact = skv.skv_plan(prob).stats()["total_cost"]
         tiles = skv.skv_plan(prob, skv.SKV_PLAN_LPT_TILES).stats()["total_cost"]
         assert exact <= tiles <= 1.2 * exact
+
+
+def test_one_queue_flag_changes_only_the_queues():
+    """SKV_PLAN_ONE_QUEUE keeps the items, costs, partitions, loads and the
+    K/V layout; unknown bits stay refused."""
+    for name in ("ctx32k", "batch8_logu"):
+        prob = synth.make_problem(synth.WORKLOADS[name], seed=0)
+        for policy in (skv.SKV_PLAN_LPT, skv.SKV_PLAN_STATIC):
+            a = skv.skv_plan(prob, policy)
+            b = skv.skv_plan(prob, policy | skv.SKV_PLAN_ONE_QUEUE)
+            assert np.array_equal(a.items(), b.items())
+            assert np.array_equal(a.partition_load, b.partition_load)
+            assert a.stats() == b.stats()
+            # the workspace holds the plan's device lists: only the queue offsets shrink (3 x P int32)
+            for x, y in ((a.sizes.ws_fwd_bytes, b.sizes.ws_fwd_bytes), (a.sizes.ws_bwd_bytes, b.sizes.ws_bwd_bytes)):
+                assert 0 <= x - y <= 3 * 4 * prob.num_partitions + 3 * 256
+            assert a.kv_layout()[0] == b.kv_layout()[0]
+    with pytest.raises(skv.SkvError):
+        skv.skv_plan_size(prob, 0x400 | skv.SKV_PLAN_ONE_QUEUE)
