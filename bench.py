@@ -245,8 +245,8 @@ def run_workload(args, name, steps, warmup, rank, world, local_rank, e2e):
     policy = {"static": skv.SKV_PLAN_STATIC, "lpt": skv.SKV_PLAN_LPT, "lpt_tiles": skv.SKV_PLAN_LPT_TILES}[args.policy]
     if args.partials == "bf16":
         policy |= skv.SKV_PLAN_PARTIALS_BF16
-    if args.queues == "one":
-        policy |= skv.SKV_PLAN_ONE_QUEUE
+    if args.queues == "partition":
+        policy |= skv.SKV_PLAN_PARTITION_QUEUES
     redraw = name == "batch8_logu"
     fused = args.fused_merge  # the merge in the forward kernel's tail, or its own launch (default: faster here)
     # what a DRAM-traffic capture of this workload must have run with to stand for this run
@@ -750,8 +750,9 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extra", action="store_true", help="time the headline workload only")
-    ap.add_argument("--queues", default="partition", choices=["partition", "one"],
-                    help="work queues of the kernels: one per partition, or one for all (SKV_PLAN_ONE_QUEUE)")
+    ap.add_argument("--queues", default="one", choices=["one", "partition"],
+                    help="work queues of the kernels: one for all items (default), or one per partition "
+                         "(SKV_PLAN_PARTITION_QUEUES)")
     ap.add_argument("--partials", default="fp32", choices=["fp32", "bf16"],
                     help="storage of the per-chunk partial outputs between the forward and the merge")
     ap.add_argument("--fused-merge", action="store_true",

@@ -81,14 +81,17 @@ enum skv_plan_policy {
    * the format from the plan. */
   SKV_PLAN_PARTIALS_BF16 = 0x100,
   /* Flag, OR-ed into any policy: the kernels of a full plan take their work
-   * units from one queue that holds every item in placement order (costliest
-   * first, each item's units together) instead of one queue per partition.
-   * The items, costs, partitions and loads do not change. On one GPU the
-   * CTAs that share a queue run neighbouring units at the same time, so an
-   * item's K/V tiles are read by many CTAs while they are in L2 rather than
-   * by the few CTAs of one partition, one after another. A shard plan always
-   * has one queue. */
-  SKV_PLAN_ONE_QUEUE = 0x200
+   * units from one queue per partition (a CTA starts on the queue of
+   * partition floor(i P / grid) and moves to the next when it is empty)
+   * instead of the default single queue that holds every item in placement
+   * order (costliest first, each item's units together). The items, costs,
+   * partitions and loads do not change. On one GPU the default is faster:
+   * the CTAs that share the queue run neighbouring units at the same time,
+   * so an item's K/V tiles are read by many CTAs while they are in L2, not
+   * by the few CTAs of one partition one after another (on the 128K
+   * workload the forward's DRAM reads drop from 5.4x to 1.04x the K/V
+   * bytes). A shard plan always has one queue. */
+  SKV_PLAN_PARTITION_QUEUES = 0x200
 };
 
 /* One split-KV problem. Host pointers; read during the call only. */

@@ -16,7 +16,7 @@ INCLUDE = os.path.join(os.path.dirname(HERE), "include")
 LIB = os.path.join(HERE, "libskv.so")
 STAMP = os.path.join(HERE, ".libskv.stamp")
 
-SOURCES = ["api.cu", "fwd.cu", "fwd2.cu", "fwd3.cu", "bwd.cu", "bwd2.cu", "merge.cu", "noalloc.cu", "selftest.cu", "lpt_device.cu",
+SOURCES = ["api.cu", "fwd.cu", "fwd2.cu", "bwd.cu", "bwd2.cu", "merge.cu", "noalloc.cu", "selftest.cu", "lpt_device.cu",
            "plan.cpp"]
 HEADERS = ["sm100.cuh", "kernels.h", "plan_layout.h", "merge_row.cuh", "tail_merge.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

@@ -23,8 +23,6 @@
 // O = 0.
 #include <cuda_runtime.h>
 
-#include <cstdlib>
-
 #include "kernels.h"
 #include "sm100.cuh"
 #include "tail_merge.cuh"
@@ -391,10 +389,7 @@ int fwd_smem_bytes(int d) { return d == 64 ? FwdSmem<64>::kDyn : FwdSmem<128>::k
 // head_dim 64 runs the one-tile kernel above; head_dim 128 the two-tile kernel of fwd2.cu
 cudaError_t launch_fwd(int d, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                        const FwdParams& p, int grid, cudaStream_t stream) {
-  if (d == 128) {
-    static const bool v3 = std::getenv("SKV_FWD3") != nullptr;  // A/B switch, temporary
-    return v3 ? launch_fwd3(tq, tk, tv, p, grid, stream) : launch_fwd2(tq, tk, tv, p, grid, stream);
-  }
+  if (d == 128) return launch_fwd2(tq, tk, tv, p, grid, stream);
   auto k = p.tile_mask ? (p.o ? fwd_kernel<64, true, true> : fwd_kernel<64, false, true>)
                        : (p.o ? fwd_kernel<64, true, false> : fwd_kernel<64, false, false>);
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, FwdSmem<64>::kDyn);

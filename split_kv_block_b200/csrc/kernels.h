@@ -13,17 +13,17 @@ struct FwdParams {
   const MTile* mtiles;
   const int32_t* tok_kend;
   const FwdUnit* units;
-  const int32_t* part_off;  // [P+1]
+  const int32_t* part_off;  // [P+1] units of each work queue
   const FwdPair* pairs;     // head_dim 128 kernel: pairs of units
-  const int32_t* pair_off;  // [P+1]
-  int32_t* counters;        // [P] queue heads, zero at launch
+  const int32_t* pair_off;  // [P+1] pairs of each work queue
+  int32_t* counters;        // [P] queue heads, zero at launch (P: the plan's work queues)
   int* status;
   float* part_o;            // [n_fwd][128][d], fp32 or (partial_bf16) bf16 elements
   float* part_lse;          // [n_fwd][128]
   int partial_bf16;         // partial outputs stored as bf16 (SKV_PLAN_PARTIALS_BF16)
   long long* stamps;        // optional [2 n_fwd] %globaltimer start/end per unit
   unsigned long long timeout_ns;
-  int P;
+  int P;                    // work queues of the plan
   int G;
   float scale_log2;         // log2(e) / sqrt(d)
   int partials_l2_last;     // store the partials with the L2 evict_last policy (they fit in L2 beside K/V)
@@ -98,8 +98,6 @@ cudaError_t launch_fwd(int d, const CUtensorMap& tq, const CUtensorMap& tk, cons
 cudaError_t launch_fwd2(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const FwdParams& p,
                         int grid, cudaStream_t stream);  // head_dim 128: pairs of query tiles
 int fwd2_smem_bytes();
-cudaError_t launch_fwd3(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const FwdParams& p,
-                        int grid, cudaStream_t stream);  // head_dim 128: 64-key score sub-tiles
 // CTAs of the forward launch: one per SM, at most one per work unit (pair for head_dim 128)
 int fwd_grid(int d, int sms, long long n_units, long long n_pairs);
 cudaError_t launch_merge(int d, const MergeParams& p, cudaStream_t stream);

@@ -282,8 +282,8 @@ void place(const Prob& q, int policy, Built& out) {
   out.imbalance = out.total_cost > 0 ? static_cast<double>(mx) * q.P / static_cast<double>(out.total_cost) - 1.0 : 0.0;
 }
 
-// shard < 0: the full plan: every partition's items on P work queues (one
-// queue holding all items in placement order with `one_queue`); the
+// shard < 0: the full plan: one work queue holding every item in placement
+// order (`one_queue`), or every partition's items on its own queue; the
 // K/V buffers are the packed context, all kv heads per row. shard = p: the
 // items of partition p only, on one work queue; the K/V buffers hold those
 // items' keys, one kv head per row, items in (b, c, g, s) order (the layout a
@@ -592,8 +592,8 @@ void make_lists(const Prob& q, const std::vector<SampleAnchors>& sa, int shard, 
 }
 
 int build(const skv_problem* prob, int policy, Built& out, Prob& q, int shard = -1) {
-  const bool one_queue = (policy & SKV_PLAN_ONE_QUEUE) != 0;
-  policy &= ~(SKV_PLAN_PARTIALS_BF16 | SKV_PLAN_ONE_QUEUE);
+  const bool one_queue = (policy & SKV_PLAN_PARTITION_QUEUES) == 0;
+  policy &= ~(SKV_PLAN_PARTIALS_BF16 | SKV_PLAN_PARTITION_QUEUES);
   if (policy != SKV_PLAN_LPT && policy != SKV_PLAN_STATIC && policy != SKV_PLAN_LPT_TILES) return SKV_EINVAL;
   int rc = validate(prob, q);
   if (rc != SKV_OK) return rc;

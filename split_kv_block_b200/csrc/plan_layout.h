@@ -77,9 +77,9 @@ struct DevSection {
   uint64_t mtiles;        // MTile[n_mtiles]
   uint64_t tok_kend;      // int32[Nq]: absolute key end of every query token
   uint64_t fwd_units;     // FwdUnit[n_fwd]
-  uint64_t fwd_part_off;  // int32[P+1]: units of partition p are [off[p], off[p+1])
+  uint64_t fwd_part_off;  // int32[n_queues + 1]: units of work queue q are [off[q], off[q+1])
   uint64_t fwd_pairs;     // FwdPair[n_fwd_pairs]
-  uint64_t fwd_pair_off;  // int32[P+1]: pairs of partition p are [off[p], off[p+1])
+  uint64_t fwd_pair_off;  // int32[n_queues + 1]: pairs of work queue q are [off[q], off[q+1])
   uint64_t merge_off;     // int32[n_mtiles * Hkv + 1]
   uint64_t merge_list;    // int32[n_fwd]: fwd unit ids per (tile, kv head), ascending kbeg
   uint64_t bwd_units;     // BwdUnit[n_bwd]
@@ -103,7 +103,7 @@ struct PlanHeader {
   int32_t B, Hq, Hkv, d, block_q, chunk_kv, sub_chunks, P;
   int32_t G, tile_tokens;  // G = Hq / Hkv, tile_tokens = 128 / G
   int32_t shard;           // -1: full plan; p: the items of partition p only (skv_plan_shard)
-  int32_t n_queues;        // work queues of the kernels: P for a full plan, 1 for a shard
+  int32_t n_queues;        // work queues of the kernels: 1, or P for a full plan with partition queues
   int32_t kv_heads;        // heads per row of the K/V (dK/dV) buffers: Hkv, or 1 for a shard
   int32_t n_dead;          // [begin, end) row ranges whose dK/dV are zero
   int32_t empty_slots;     // (query tile, kv head) slots without a forward unit (possible in a shard)

@@ -21,7 +21,7 @@ SKV_PLAN_LPT = 0
 SKV_PLAN_STATIC = 1
 SKV_PLAN_LPT_TILES = 2          # LPT on the executed-tile cost (see include/skv.h)
 SKV_PLAN_PARTIALS_BF16 = 0x100  # flag: bf16 partial outputs (see include/skv.h)
-SKV_PLAN_ONE_QUEUE = 0x200      # flag: one work queue for all partitions (see include/skv.h)
+SKV_PLAN_PARTITION_QUEUES = 0x200  # flag: one work queue per partition (see include/skv.h)
 
 # Every function include/skv.h declares.
 EXPORTS = ("skv_plan_size", "skv_plan", "skv_plan_items", "skv_plan_unit_partitions", "skv_plan_stats", "skv_attn_fwd",

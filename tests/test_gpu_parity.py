@@ -260,12 +260,12 @@ def test_tile_cost_plans():
     _case(prob, seed=6, policy=skv.SKV_PLAN_LPT_TILES)
 
 
-def test_one_queue_plans():
-    """SKV_PLAN_ONE_QUEUE (every item's units on one work queue, costliest
-    item first): forward and backward against the oracle, head_dim 64 and
-    128, ragged tiles, both merges, and the 128K workload on one kv-head
-    group."""
-    flag = skv.SKV_PLAN_ONE_QUEUE
+def test_partition_queue_plans():
+    """SKV_PLAN_PARTITION_QUEUES (one work queue per partition, CTAs stealing
+    from the next queue when theirs is empty): forward and backward against
+    the oracle, head_dim 64 and 128, ragged tiles, both merges, and the 128K
+    workload on one kv-head group."""
+    flag = skv.SKV_PLAN_PARTITION_QUEUES
     _case(synth.make_problem(synth.WORKLOADS["tiny_4k"], seed=4), seed=4, policy=skv.SKV_PLAN_LPT | flag)
     prob = synth.small_problem([1001, 777, 1500], [[1000, 3, 555], [777], [1, 1499, 700, 64, 1200]], block_q=16,
                                chunk_kv=320, num_partitions=4, hq=8, hkv=2, d=128)

@@ -151,17 +151,18 @@ def _expected_unit_counts(prob, items):
 def test_unit_partitions_match_item_partitions(seed):
     rng = np.random.default_rng(500 + seed)
     prob = synth.random_small_problem(rng, max_len=3000, max_anchors=9, d=128, heads=((8, 2), (16, 4), (4, 1)))
-    plan = skv.skv_plan(prob)
-    fp, bp = plan.unit_partitions()
-    st = plan.stats()
-    assert len(fp) == st["n_fwd_units"] and len(bp) == st["n_bwd_units"]
     P = prob.num_partitions
-    assert np.all((fp >= 0) & (fp < P)) and np.all((bp >= 0) & (bp < P))
-    # the work lists are grouped by partition
-    assert np.all(np.diff(fp) >= 0) and np.all(np.diff(bp) >= 0)
-    ef, eb = _expected_unit_counts(prob, plan.items())
-    assert np.bincount(fp, minlength=P).tolist() == ef.tolist()
-    assert np.bincount(bp, minlength=P).tolist() == eb.tolist()
+    for flag in (0, skv.SKV_PLAN_PARTITION_QUEUES):
+        plan = skv.skv_plan(prob, skv.SKV_PLAN_LPT | flag)
+        fp, bp = plan.unit_partitions()
+        st = plan.stats()
+        assert len(fp) == st["n_fwd_units"] and len(bp) == st["n_bwd_units"]
+        assert np.all((fp >= 0) & (fp < P)) and np.all((bp >= 0) & (bp < P))
+        if flag:  # one work queue per partition: the work lists are grouped by partition
+            assert np.all(np.diff(fp) >= 0) and np.all(np.diff(bp) >= 0)
+        ef, eb = _expected_unit_counts(prob, plan.items())
+        assert np.bincount(fp, minlength=P).tolist() == ef.tolist()
+        assert np.bincount(bp, minlength=P).tolist() == eb.tolist()
 
 
 def test_unit_partitions_of_the_32k_workload():
@@ -342,20 +343,20 @@ def test_tile_cost_at_least_the_exact_cost_on_the_workloads():
         assert exact <= tiles <= 1.2 * exact
 
 
-def test_one_queue_flag_changes_only_the_queues():
-    """SKV_PLAN_ONE_QUEUE keeps the items, costs, partitions, loads and the
-    K/V layout; unknown bits stay refused."""
+def test_partition_queues_flag_changes_only_the_queues():
+    """SKV_PLAN_PARTITION_QUEUES keeps the items, costs, partitions, loads
+    and the K/V layout; unknown bits stay refused."""
     for name in ("ctx32k", "batch8_logu"):
         prob = synth.make_problem(synth.WORKLOADS[name], seed=0)
         for policy in (skv.SKV_PLAN_LPT, skv.SKV_PLAN_STATIC):
             a = skv.skv_plan(prob, policy)
-            b = skv.skv_plan(prob, policy | skv.SKV_PLAN_ONE_QUEUE)
+            b = skv.skv_plan(prob, policy | skv.SKV_PLAN_PARTITION_QUEUES)
             assert np.array_equal(a.items(), b.items())
             assert np.array_equal(a.partition_load, b.partition_load)
             assert a.stats() == b.stats()
-            # the workspace holds the plan's device lists: only the queue offsets shrink (3 x P int32)
-            for x, y in ((a.sizes.ws_fwd_bytes, b.sizes.ws_fwd_bytes), (a.sizes.ws_bwd_bytes, b.sizes.ws_bwd_bytes)):
+            # the workspace holds the plan's device lists: only the queue offsets grow (3 x P int32)
+            for x, y in ((b.sizes.ws_fwd_bytes, a.sizes.ws_fwd_bytes), (b.sizes.ws_bwd_bytes, a.sizes.ws_bwd_bytes)):
                 assert 0 <= x - y <= 3 * 4 * prob.num_partitions + 3 * 256
             assert a.kv_layout()[0] == b.kv_layout()[0]
     with pytest.raises(skv.SkvError):
-        skv.skv_plan_size(prob, 0x400 | skv.SKV_PLAN_ONE_QUEUE)
+        skv.skv_plan_size(prob, 0x400 | skv.SKV_PLAN_PARTITION_QUEUES)
