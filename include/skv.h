@@ -83,14 +83,16 @@ enum skv_plan_policy {
   /* Flag, OR-ed into any policy: the kernels of a full plan take their work
    * units from one queue per partition (a CTA starts on the queue of
    * partition floor(i P / grid) and moves to the next when it is empty)
-   * instead of the default single queue that holds every item in placement
-   * order (costliest first, each item's units together). The items, costs,
+   * instead of the default single queue that holds every item, each item's
+   * units together: samples in the order of their costliest item, a
+   * sample's items in placement order (costliest first). The items, costs,
    * partitions and loads do not change. On one GPU the default is faster:
    * the CTAs that share the queue run neighbouring units at the same time,
    * so an item's K/V tiles are read by many CTAs while they are in L2, not
    * by the few CTAs of one partition one after another (on the 128K
    * workload the forward's DRAM reads drop from 5.4x to 1.04x the K/V
-   * bytes). A shard plan always has one queue. */
+   * bytes), and only one or two samples' queries and gradients are in use
+   * at a time. A shard plan always has one queue. */
   SKV_PLAN_PARTITION_QUEUES = 0x200
 };
 

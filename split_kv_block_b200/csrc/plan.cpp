@@ -367,6 +367,17 @@ void make_lists(const Prob& q, const std::vector<SampleAnchors>& sa, int shard, 
   std::vector<std::vector<int32_t>> by_queue(out.n_queues);
   for (int32_t id : out.placement)
     if (in_plan[id]) by_queue[per_partition ? out.items[id].partition : 0].push_back(id);
+  if (!per_partition && q.B > 1) {
+    // One queue: samples in the order of their costliest item, each sample's items in placement order.
+    // The CTAs then work on one or two samples at a time, so those samples' queries, output gradients and
+    // dQ accumulator stay in L2 instead of every sample's at once.
+    std::vector<int32_t> rank(q.B, -1);
+    int32_t next = 0;
+    for (int32_t id : by_queue[0])
+      if (rank[out.items[id].b] < 0) rank[out.items[id].b] = next++;
+    std::stable_sort(by_queue[0].begin(), by_queue[0].end(),
+                     [&](int32_t x, int32_t y) { return rank[out.items[x].b] < rank[out.items[y].b]; });
+  }
 
   out.fwd.clear();
   out.unit_live.clear();
