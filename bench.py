@@ -217,7 +217,7 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------- GPU arm
-EXTRA_WORKLOADS = ("ctx128k", "batch8_logu", "ctx32k_sparse")  # measured beside the headline workload on one GPU
+EXTRA_WORKLOADS = ("ctx128k", "batch8_logu", "ctx32k_sparse", "tiny_4k")  # beside the headline on one GPU; tiny_4k runs the head_dim-64 kernels
 
 
 def merge_bytes(prob, n_fwd_units):
