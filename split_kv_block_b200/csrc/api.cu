@@ -49,7 +49,9 @@ Staging g_stage[kSlots];
 int g_stage_next = 0;
 std::vector<void*> g_retired;  // outgrown staging buffers, released with the process
 
-int upload(const void* src, size_t n, void* dst, cudaStream_t stream) {
+// Copies `zeros` zero bytes followed by the n bytes at src to dst, in one
+// host-to-device copy.
+int upload(const void* src, size_t n, void* dst, cudaStream_t stream, size_t zeros = 0) {
   std::lock_guard<std::mutex> lock(g_stage_mu);
   Staging& s = g_stage[g_stage_next];
   g_stage_next = (g_stage_next + 1) % kSlots;
@@ -63,13 +65,14 @@ int upload(const void* src, size_t n, void* dst, cudaStream_t stream) {
     e = cudaEventCreateWithFlags(&s.done, cudaEventDisableTiming);
     if (e != cudaSuccess) return cuda_fail(e);
   }
-  if (s.cap < n) {
+  const size_t total = zeros + n;
+  if (s.cap < total) {
     // Grow geometrically and keep the old buffer until exit: cudaFreeHost
     // synchronizes the device, which would stall the caller's pipeline
     // whenever a larger plan arrives (plans change size every step when the
     // anchors are redrawn).
     size_t cap = size_t(1) << 20;
-    while (cap < n) cap <<= 1;
+    while (cap < total) cap <<= 1;
     void* fresh = nullptr;
     e = cudaHostAlloc(&fresh, cap, cudaHostAllocDefault);
     if (e != cudaSuccess) return cuda_fail(e);
@@ -77,8 +80,9 @@ int upload(const void* src, size_t n, void* dst, cudaStream_t stream) {
     s.host = fresh;
     s.cap = cap;
   }
-  std::memcpy(s.host, src, n);
-  e = cudaMemcpyAsync(dst, s.host, n, cudaMemcpyHostToDevice, stream);
+  std::memset(s.host, 0, zeros);
+  std::memcpy(static_cast<uint8_t*>(s.host) + zeros, src, n);
+  e = cudaMemcpyAsync(dst, s.host, total, cudaMemcpyHostToDevice, stream);
   if (e != cudaSuccess) return cuda_fail(e);
   e = cudaEventRecord(s.done, stream);
   if (e != cudaSuccess) return cuda_fail(e);
@@ -138,12 +142,12 @@ bool aligned16(const void* p) { return reinterpret_cast<uintptr_t>(p) % 16 == 0;
 // uploads the arrays only the deterministic backward reads.
 int prepare_ws(const PlanHeader& h, const void* plan, void* ws, const WsLayout& w, cudaStream_t stream,
                bool full = false) {
-  // status word, queue counters and merge counters: one contiguous control block
-  cudaError_t e = cudaMemsetAsync(at<uint8_t>(ws, w.status), 0, w.control, stream);
-  if (e != cudaSuccess) return cuda_fail(e);
+  // The control block (status word, queue and merge counters) is cleared and the plan's device section
+  // copied behind it by one host-to-device copy: zeros up to the device section, then the section.
   const uint64_t n = full ? h.dev.bytes : h.dev.base_bytes;
-  if (n > 0) return upload(static_cast<const uint8_t*>(plan) + h.dev_off, n, at<uint8_t>(ws, w.dev), stream);
-  return SKV_OK;
+  if (n > 0) return upload(static_cast<const uint8_t*>(plan) + h.dev_off, n, at<uint8_t>(ws, w.status), stream, w.dev);
+  const cudaError_t e = cudaMemsetAsync(at<uint8_t>(ws, w.status), 0, w.control, stream);
+  return e == cudaSuccess ? SKV_OK : cuda_fail(e);
 }
 
 }  // namespace

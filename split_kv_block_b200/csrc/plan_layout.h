@@ -128,7 +128,8 @@ struct PlanHeader {
 };
 
 // Workspace layout: control block (status word and queue counters, cleared by
-// one memset per call), device plan section, then the pass-specific scratch.
+// the same host-to-device copy that uploads the plan's device section behind
+// it, once per call), device plan section, then the pass-specific scratch.
 struct WsLayout {
   uint64_t status;    // int32 status word at offset 0
   uint64_t counters;  // int32[2 * P] queue heads (forward, backward), right after it

@@ -273,3 +273,26 @@ def test_partition_queue_plans():
     _case(prob, seed=7, policy=skv.SKV_PLAN_STATIC | flag, fused=False)
     _case(synth.make_problem(synth.WORKLOADS["ctx128k"], seed=0), seed=0, policy=skv.SKV_PLAN_LPT | flag,
           groups=(5,))
+
+
+def test_queue_modes_compute_the_same_bits():
+    """The work queues only decide which CTA runs a unit and when: every
+    forward unit's partial, hence the merged O and LSE, and the deterministic
+    backward's dQ, dK and dV are the same bits with one queue and with one
+    queue per partition (ctx32k, and a ragged three-sample problem)."""
+    for prob in (synth.make_problem(synth.WORKLOADS["ctx32k"], seed=1),
+                 synth.small_problem([1001, 777, 1500], [[1000, 3, 555], [777], [1, 1499, 700, 64, 1200]],
+                                     block_q=16, chunk_kv=320, num_partitions=4, hq=8, hkv=2, d=128)):
+        q, k, v, do = synth.make_tensors(prob, seed=2, backward=True)
+        qd, kd, vd, dod = _dev(q, k, v, do)
+        outs = []
+        for flag in (0, skv.SKV_PLAN_PARTITION_QUEUES):
+            plan = skv.skv_plan(prob, skv.SKV_PLAN_LPT | flag)
+            ws = skv.alloc_workspace(plan)
+            o, lse = skv.forward(plan, qd, kd, vd, ws, fused=False)
+            grads = skv.backward(plan, qd, kd, vd, o, lse, dod, ws, deterministic=True)
+            assert skv.skv_status(ws) == 0
+            torch.cuda.synchronize()
+            outs.append([o.cpu(), lse.cpu()] + [g.cpu() for g in grads])
+        for a, b in zip(*outs):
+            assert torch.equal(a, b)
