@@ -26,8 +26,6 @@
 // 1, 2 TMEM allocator, 4..7 softmax of tile 0, 8..11 softmax of tile 1.
 #include <cuda_runtime.h>
 
-#include <type_traits>
-
 #include "kernels.h"
 #include "sm100.cuh"
 #include "tail_merge.cuh"
@@ -76,30 +74,10 @@ __device__ __forceinline__ float row_max64(const uint32_t (&sv)[64]) {
   return fmaxf(fmax3(mx[0], mx[1], mx[2]), mx[3]);
 }
 
-// 2^x on the FMA pipe, for x >= -125 (smaller x gives about 2^-125, below 3e-38, instead of less; the
-// caller keeps masked entries, which are -inf, on the special-function unit). Cody and Waite's range reduction:
-// x = n + f with n = round(x) (adding 1.5 * 2^23 leaves n in the low mantissa bits) and |f| <= 1/2;
-// 2^f by the cubic of smallest maximum relative error on [-1/2, 1/2] (Remez exchange; the coefficients
-// and the bound, 7.5e-5, come from split_kv_block_b200/exp2_poly.py); n is added to the exponent bits.
-// The P values are rounded to bf16 (relative step 2^-9) before the MMA, so the cubic's error is
-// below their rounding; the row sums see it at 7.5e-5 relative at most.
-__device__ __forceinline__ float exp2_fma(float x) {
-  x = fmaxf(x, -125.f);
-  const float t = x + 12582912.f;
-  const float f = x - (t - 12582912.f);
-  float q = fmaf(0.0551716685f, f, 0.242611125f);
-  q = fmaf(q, f, 0.693260968f);
-  q = fmaf(q, f, 0.999928057f);
-  return __int_as_float(__float_as_int(q) + (__float_as_int(t) << 23));
-}
-
 // P = 2^(s sl2 - m_use) over one 64-column score row (masked entries are -inf -> 0), stored as bf16
 // pairs into the first 32 TMEM columns at tS; returns the row sum. With kMax it also returns, in
 // raw_max, the maximum of the raw scores (three-input maxima on the ALU pipe beside the exponentials).
-// With kFma one exponential in four runs on the FMA pipe (exp2_fma): the two query tiles' softmax
-// warps share each SM quarter's special-function unit, which bounds this loop; rows with masked
-// columns keep every exponential on that unit.
-template <bool kMax, bool kFma>
+template <bool kMax>
 __device__ __forceinline__ float exp_row64(const uint32_t (&sv)[64], float sl2, float m_use, uint32_t tS,
                                            float& raw_max) {
   float rs[4] = {0.f, 0.f, 0.f, 0.f};
@@ -118,7 +96,7 @@ __device__ __forceinline__ float exp_row64(const uint32_t (&sv)[64], float sl2, 
       const float x0 = ex2(fmaf(s0, sl2, -m_use));
       const float x1 = ex2(fmaf(s1, sl2, -m_use));
       const float x2 = ex2(fmaf(s2, sl2, -m_use));
-      const float x3 = kFma ? exp2_fma(fmaf(s3, sl2, -m_use)) : ex2(fmaf(s3, sl2, -m_use));
+      const float x3 = ex2(fmaf(s3, sl2, -m_use));
       rs[0] += x0;
       rs[1] += x1;
       rs[2] += x2;
@@ -391,19 +369,13 @@ __global__ void __launch_bounds__(384, 1)
           for (int i = 0; i < 64; ++i)
             if (i >= lim_c) sv[i] = __float_as_uint(-INFINITY);
         }
-        // the exponentials: a quarter on the FMA pipe unless a column of the warp's rows is masked
-        const bool fma_ok = __all_sync(0xffffffffu, lim_c >= 64);
-        auto exp_pass = [&](auto max_tag, float m_use, float& raw_out) -> float {
-          constexpr bool kM = decltype(max_tag)::value;
-          return fma_ok ? exp_row64<kM, true>(sv, sl2, m_use, tS, raw_out) : exp_row64<kM, false>(sv, sl2, m_use, tS, raw_out);
-        };
         float raw;
         if (s == 0) {
           // first sub-tile of the unit: the reference is its maximum (-inf for a row without keys)
           m_ref = row_max64(sv) * sl2;
-          l = exp_pass(std::false_type{}, m_ref == -INFINITY ? 0.f : m_ref, raw);
+          l = exp_row64<false>(sv, sl2, m_ref == -INFINITY ? 0.f : m_ref, tS, raw);
         } else {
-          const float add = exp_pass(std::true_type{}, m_ref == -INFINITY ? 0.f : m_ref, raw);
+          const float add = exp_row64<true>(sv, sl2, m_ref == -INFINITY ? 0.f : m_ref, tS, raw);
           const float tmax = raw * sl2;
           const bool move = tmax > m_ref + 8.f;
           if (__any_sync(0xffffffffu, move)) {
@@ -425,7 +397,7 @@ __global__ void __launch_bounds__(384, 1)
             }
             tmem_wait_st();  // also orders the first pass's P stores before the rewrite
             m_ref = m_new;
-            l = l * alpha + exp_pass(std::false_type{}, m_ref == -INFINITY ? 0.f : m_ref, raw);
+            l = l * alpha + exp_row64<false>(sv, sl2, m_ref == -INFINITY ? 0.f : m_ref, tS, raw);
           } else {
             l += add;
           }
