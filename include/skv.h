@@ -92,11 +92,7 @@ enum skv_plan_policy {
    * by the few CTAs of one partition one after another (on the 128K
    * workload the forward's DRAM reads drop from 5.4x to 1.04x the K/V
    * bytes), and only one or two samples' queries and gradients are in use
-   * at a time. On a single queue without a block mask, the queue's last 148
-   * pairs of query tiles (about one wave of CTAs) that span two key tiles or
-   * more are split in two by key range, so the last wave ends on short
-   * units; the extra forward units add partials to the merge. A shard plan
-   * always has one queue. */
+   * at a time. A shard plan always has one queue. */
   SKV_PLAN_PARTITION_QUEUES = 0x200
 };
 

@@ -14,7 +14,6 @@
 // computed from the sample's sorted anchors and their prefix sums in
 // O(log A) per item.
 #include <algorithm>
-#include <cstdint>
 #include <cstring>
 #include <iterator>
 #include <functional>
@@ -391,23 +390,6 @@ void make_lists(const Prob& q, const std::vector<SampleAnchors>& sa, int shard, 
   out.bwd_part_off.assign(out.n_queues + 1, 0);
   std::vector<std::pair<int64_t, int32_t>> tiles;
   std::vector<std::pair<int32_t, int32_t>> item_fwd(out.items.size(), {0, 0});  // [first forward unit, count]
-  // One queue without a block mask: each of the last kTailPairs pairs of the queue that spans two key
-  // tiles or more is split at a key tile boundary into two pairs of about half its key range, so the last
-  // wave of CTAs ends on short units (kTailPairs: about one wave of a 148-SM GPU). The second halves are
-  // units of their own; their partials join the merge like any other, after the first halves' partials
-  // of the same query tile (ascending key order).
-  constexpr int64_t kTailPairs = 148;
-  int64_t split_from = INT64_MAX, pair_idx = 0;
-  if (!per_partition && !q.mask) {
-    int64_t n_pairs = 0;
-    for (int32_t id : by_queue[0]) {
-      const skv_item& it = out.items[id];
-      int64_t n = 0;
-      for (int32_t mt = out.sample_mt[it.b]; mt < out.sample_mt[it.b + 1]; ++mt) n += out.mtiles[mt].kmax > it.key_begin;
-      n_pairs += (n + 1) / 2;
-    }
-    split_from = n_pairs - kTailPairs;
-  }
   std::vector<int64_t> item_cov_end(out.items.size(), 0);  // end of the keys the item's backward units cover
   for (int p = 0; p < out.n_queues; ++p) {
     out.fwd_part_off[p] = static_cast<int32_t>(out.fwd.size());
@@ -476,33 +458,6 @@ void make_lists(const Prob& q, const std::vector<SampleAnchors>& sa, int shard, 
         }
         out.fwd.push_back(u);
       }
-      // split this item's pairs that fall in the queue's last kTailPairs
-      const size_t item_pairs_end = out.pairs.size(), item_pairs_begin = item_pairs_end - (tiles.size() + 1) / 2;
-      for (size_t pi = item_pairs_begin; pi < item_pairs_end; ++pi, ++pair_idx) {
-        if (pair_idx < split_from) continue;
-        const int32_t kb = out.pairs[pi].kbeg, ke = out.pairs[pi].kend;
-        const int64_t nt = (static_cast<int64_t>(ke) - kb + kTileN - 1) / kTileN;
-        if (nt < 2) continue;
-        const int32_t mid = kb + static_cast<int32_t>((nt + 1) / 2 * kTileN);
-        FwdPair hi{};
-        hi.slot[0] = hi.slot[1] = -1;
-        hi.kbeg = mid;
-        hi.kend = ke;
-        hi.part = out.pairs[pi].part;
-        int n_hi = 0;
-        for (int k = 0; k < 2; ++k) {
-          const int32_t us = out.pairs[pi].slot[k];
-          if (us < 0 || out.fwd[us].kend <= mid) continue;
-          FwdUnit u2 = out.fwd[us];
-          u2.kbeg = mid;
-          out.fwd[us].kend = mid;
-          hi.slot[n_hi++] = static_cast<int32_t>(out.fwd.size());
-          out.fwd.push_back(u2);
-        }
-        out.pairs[pi].kend = mid;
-        out.pairs.push_back(hi);  // the longer of the second halves first
-      }
-      item_fwd[id].second = static_cast<int32_t>(out.fwd.size()) - item_fwd[id].first;
       // backward: key tiles below the sample's largest anchor
       const int64_t kmax_b = q.ctx[it.b] + sa[it.b].max_a;
       // first query tile whose largest anchor reaches past the key tile start (later dead tiles,

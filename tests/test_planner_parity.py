@@ -161,65 +161,18 @@ def test_unit_partitions_match_item_partitions(seed):
         if flag:  # one work queue per partition: the work lists are grouped by partition
             assert np.all(np.diff(fp) >= 0) and np.all(np.diff(bp) >= 0)
         ef, eb = _expected_unit_counts(prob, plan.items())
-        if not flag:
-            ef = ef + _tail_split_extra(prob, plan.items())
         assert np.bincount(fp, minlength=P).tolist() == ef.tolist()
         assert np.bincount(bp, minlength=P).tolist() == eb.tolist()
-
-
-def _tail_split_extra(prob, items, tail=148):
-    """Forward units the one-queue plan adds per partition by splitting the
-    queue's last `tail` pairs (those spanning two key tiles or more) at the
-    key tile boundary after half their tiles (rounded up): one unit for the
-    pair's longer tile, one more for the shorter tile if it reaches past the
-    split. Queue order: samples by their costliest item, then placement
-    order; an item's live tiles sorted by key extent (longest first, ties by
-    index) and paired in that order."""
-    S, G = prob.block_q, prob.num_q_heads // prob.num_kv_heads
-    tt = 128 // G
-    rank = {}
-    for i in sorted(range(len(items)), key=lambda i: int(items[i]["order"])):
-        rank.setdefault(int(items[i]["b"]), len(rank))
-    queue = sorted(range(len(items)), key=lambda i: (rank[int(items[i]["b"])], int(items[i]["order"])))
-    pairs = []
-    for i in queue:
-        r = items[i]
-        b, kb, ke = int(r["b"]), int(r["key_begin"]), int(r["key_end"])
-        c0, a0, a1 = int(prob.ctx_offsets[b]), int(prob.anchor_offsets[b]), int(prob.anchor_offsets[b + 1])
-        ntok = (a1 - a0) * S
-        ext = []
-        for t0 in range(0, ntok, tt):
-            kmax = c0 + max(int(prob.anchors[j]) for j in range(a0 + t0 // S, a0 + (min(t0 + tt, ntok) - 1) // S + 1))
-            if kmax > kb:
-                ext.append(min(kmax, ke) - kb)
-        ext.sort(reverse=True)
-        for k in range(0, len(ext), 2):
-            pairs.append((int(r["partition"]), ext[k:k + 2]))
-    extra = np.zeros(prob.num_partitions, dtype=np.int64)
-    for part, e in pairs[max(0, len(pairs) - tail):]:
-        nt = (e[0] + 127) // 128
-        if nt >= 2:
-            mid = (nt + 1) // 2 * 128
-            extra[part] += 1 + (len(e) > 1 and e[1] > mid)
-    return extra
 
 
 def test_unit_partitions_of_the_32k_workload():
-    """One work queue (the default): the forward units are the live (item,
-    query tile) pairs plus the second halves of the split tail pairs; with one
-    queue per partition nothing is split."""
     prob = synth.make_problem(synth.WORKLOADS["ctx32k"], seed=0)
+    plan = skv.skv_plan(prob)
+    fp, bp = plan.unit_partitions()
+    ef, eb = _expected_unit_counts(prob, plan.items())
     P = prob.num_partitions
-    for flag in (0, skv.SKV_PLAN_PARTITION_QUEUES):
-        plan = skv.skv_plan(prob, skv.SKV_PLAN_LPT | flag)
-        fp, bp = plan.unit_partitions()
-        ef, eb = _expected_unit_counts(prob, plan.items())
-        if not flag:
-            extra = _tail_split_extra(prob, plan.items())
-            assert 148 <= extra.sum() <= 2 * 148
-            ef = ef + extra
-        assert np.bincount(fp, minlength=P).tolist() == ef.tolist()
-        assert np.bincount(bp, minlength=P).tolist() == eb.tolist()
+    assert np.bincount(fp, minlength=P).tolist() == ef.tolist()
+    assert np.bincount(bp, minlength=P).tolist() == eb.tolist()
 
 
 def test_plans_do_not_depend_on_earlier_calls():
@@ -391,10 +344,8 @@ def test_tile_cost_at_least_the_exact_cost_on_the_workloads():
 
 
 def test_partition_queues_flag_changes_only_the_queues():
-    """SKV_PLAN_PARTITION_QUEUES keeps the items, costs, partitions, loads,
-    the backward units and the K/V layout; the single queue only adds the
-    split tail's forward units (at most two per split pair, 148 pairs) and
-    their partials; unknown bits stay refused."""
+    """SKV_PLAN_PARTITION_QUEUES keeps the items, costs, partitions, loads
+    and the K/V layout; unknown bits stay refused."""
     for name in ("ctx32k", "batch8_logu"):
         prob = synth.make_problem(synth.WORKLOADS[name], seed=0)
         for policy in (skv.SKV_PLAN_LPT, skv.SKV_PLAN_STATIC):
@@ -402,14 +353,10 @@ def test_partition_queues_flag_changes_only_the_queues():
             b = skv.skv_plan(prob, policy | skv.SKV_PLAN_PARTITION_QUEUES)
             assert np.array_equal(a.items(), b.items())
             assert np.array_equal(a.partition_load, b.partition_load)
-            sa, sb = a.stats(), b.stats()
-            extra = sa.pop("n_fwd_units") - sb.pop("n_fwd_units")
-            assert sa == sb and 0 <= extra <= 2 * 148
-            # the workspace: the extra units' partials (fp32 [128][d] and [128] LSE each) and their list
-            # entries in one, the queue offsets (3 x P int32) in the other
-            part = 128 * (prob.head_dim + 1) * 4
-            assert 0 <= a.sizes.ws_fwd_bytes - b.sizes.ws_fwd_bytes - extra * part <= extra * 64 + 4 * 256
-            assert abs(a.sizes.ws_bwd_bytes - b.sizes.ws_bwd_bytes) <= extra * 64 + 3 * 4 * prob.num_partitions + 4 * 256
+            assert a.stats() == b.stats()
+            # the workspace holds the plan's device lists: only the queue offsets grow (3 x P int32)
+            for x, y in ((b.sizes.ws_fwd_bytes, a.sizes.ws_fwd_bytes), (b.sizes.ws_bwd_bytes, a.sizes.ws_bwd_bytes)):
+                assert 0 <= x - y <= 3 * 4 * prob.num_partitions + 3 * 256
             assert a.kv_layout()[0] == b.kv_layout()[0]
     with pytest.raises(skv.SkvError):
         skv.skv_plan_size(prob, 0x400 | skv.SKV_PLAN_PARTITION_QUEUES)
