@@ -14,7 +14,9 @@
 //     so one half's softmax runs while the other half's MMAs execute.
 //   * P^T stays in TMEM and feeds dV += P^T dO as the A operand; dS^T goes to
 //     shared memory once and serves as the A operand of dK += dS^T Q and the
-//     B operand of dQ^T = K^T dS^T.
+//     B operand of dQ^T = K^T dS^T. A half's gradient MMAs run dQ^T first,
+//     then dV and dK, so its dQ^T is read out and reduced while the tensor
+//     core still works on the half's dV and dK.
 //   * dQ is produced transposed (TMEM lane = head-dim index), so the fp32
 //     reduction into the shared dQ accumulator writes 128 consecutive floats
 //     of a row per warpgroup instruction.
@@ -277,6 +279,13 @@ __global__ void __launch_bounds__(384, 1)
           }
           tc_fence_after();
           if (leader) {
+            // dQ^T of the half's rows = K^T dS^T -> B_h, first: the gradient warps read it out and reduce it
+            // while the tensor core runs the half's dV and dK
+#pragma unroll
+            for (int ks = 0; ks < 128 / 16; ++ks)
+              umma_bf16(tmem + col_b(h), sdesc_add(dK_mn, ks * 2048), sdesc_add(dS_mn, h * 16384 + ks * 2048), idQ,
+                        ks > 0);
+            umma_commit(&c.dq_full[h]);
             // dV += P^T dO over the half's 64 rows (A = P^T_h from TMEM)
 #pragma unroll
             for (int k4 = 0; k4 < 4; ++k4) {
@@ -286,7 +295,8 @@ __global__ void __launch_bounds__(384, 1)
             }
             umma_commit(&c.dv_done[h]);
             if (h == 1) umma_commit(&c.do_empty[s]);
-            // dK += dS^T Q over the half's rows
+            // dK += dS^T Q over the half's rows (the next tile's dS^T is written only after its S^T/dP^T, whose
+            // commit covers this MMA)
 #pragma unroll
             for (int k4 = 0; k4 < 4; ++k4) {
               const uint32_t acc = (first && h == 0 && k4 == 0) ? 0u : 1u;
@@ -294,12 +304,6 @@ __global__ void __launch_bounds__(384, 1)
                         sdesc_add(dQ_mn, s * kTileBytes + (64 * h + 16 * k4) * 128), idKV, acc);
             }
             if (h == 1) umma_commit(&c.q_empty[s]);
-            // dQ^T of the half's rows = K^T dS^T -> B_h
-#pragma unroll
-            for (int ks = 0; ks < 128 / 16; ++ks)
-              umma_bf16(tmem + col_b(h), sdesc_add(dK_mn, ks * 2048), sdesc_add(dS_mn, h * 16384 + ks * 2048), idQ,
-                        ks > 0);
-            umma_commit(&c.dq_full[h]);
           }
           __syncwarp();
           // this half of the unit's next tile, as soon as A_h and B_h are free
