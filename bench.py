@@ -217,7 +217,10 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------- GPU arm
-EXTRA_WORKLOADS = ("ctx128k", "batch8_logu", "ctx32k_sparse", "tiny_4k")  # beside the headline on one GPU; tiny_4k runs the head_dim-64 kernels
+# Beside the headline on one GPU: (workload, LPT sub-chunks or None for the workload's own). The 128K
+# workload is also timed with its chunks split in four, the granularity at which its plan is within 1 %;
+# tiny_4k runs the head_dim-64 kernels.
+EXTRA_WORKLOADS = (("ctx128k", None), ("ctx128k", 4), ("batch8_logu", None), ("ctx32k_sparse", None), ("tiny_4k", None))
 
 
 def merge_bytes(prob, n_fwd_units):
@@ -228,16 +231,20 @@ def merge_bytes(prob, n_fwd_units):
     return n_fwd_units * 128 * (prob.head_dim + 1) * 4 + rows * prob.head_dim * 2 + rows * 4
 
 
-def run_workload(args, name, steps, warmup, rank, world, local_rank, e2e):
+def run_workload(args, name, steps, warmup, rank, world, local_rank, e2e, sub_chunks=None):
     """Time `steps` whole steps of workload `name` (after `warmup` untimed ones)
-    on this rank's GPU and return its record."""
+    on this rank's GPU and return its record. sub_chunks: the LPT item split
+    (None: --sub-chunks for the headline workload, the workload's own
+    otherwise)."""
     from split_kv_block_b200 import skv
 
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     w = synth.WORKLOADS[name]
     seed = args.seed + rank
-    prob = synth.make_problem(w, seed=seed, sub_chunks=args.sub_chunks if name == args.workload else None)
+    if sub_chunks is None and name == args.workload:
+        sub_chunks = args.sub_chunks
+    prob = synth.make_problem(w, seed=seed, sub_chunks=sub_chunks)
     backward = w.backward
     q, k, v, do = synth.make_tensors(prob, seed=seed, backward=backward)
     q, k, v = q.to(dev), k.to(dev), v.to(dev)
@@ -440,11 +447,11 @@ def run_gpu(args, rank, world, local_rank):
         # the other target workloads, each timed on its own (same contract: warm-up, then steps timed with
         # CUDA events, clocks sampled during its timed region)
         out["workloads"] = {}
-        for name in EXTRA_WORKLOADS:
-            if name == args.workload:
+        for name, sub in EXTRA_WORKLOADS:
+            if name == args.workload and sub is None:
                 continue
-            r, _ = run_workload(args, name, min(args.steps, 20), args.warmup, rank, world, local_rank, False)
-            out["workloads"][name] = r
+            r, _ = run_workload(args, name, min(args.steps, 20), args.warmup, rank, world, local_rank, False, sub)
+            out["workloads"][name if sub is None else f"{name}_sub{sub}"] = r
     return out, prob
 
 
