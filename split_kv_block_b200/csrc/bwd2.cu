@@ -287,9 +287,9 @@ __global__ void __launch_bounds__(384, 1)
         if (!mbar_wait_warp(&c.kv_full, (kv_waits++) & 1, status, lim)) break;
         // The two halves advance independently: each issues S^T/dP^T of its next tile as soon as the tile's
         // Q/dO are loaded and its A_h/B_h are free, and that tile's gradient MMAs as soon as its warpgroup has
-        // written P^T and dS^T and the other half's gradient MMAs of the previous step are issued; whichever
-        // half is ready goes first, so a half waiting for its buffers never holds up the other. A Q/dO stage
-        // is released after both halves' gradient MMAs of its tile.
+        // written P^T and dS^T; whichever half is ready goes first. Half 0 issues the unit's first gradient
+        // MMAs (they overwrite dV/dK) before half 1's; a Q/dO stage is released after both halves' gradient
+        // MMAs of its tile.
         int ti[2] = {0, 0};          // unit-local index of the half's next tile
         bool sdp_next[2] = {true, true};
         int grads_done[2] = {-1, -1};  // last tile whose gradient MMAs the half issued
@@ -326,11 +326,9 @@ __global__ void __launch_bounds__(384, 1)
               sdp_next[h] = false;
               prog = true;
             } else {
-              // the halves' gradient MMAs alternate, half 0 first (dV and dK then accumulate in a fixed order,
-              // so they are the same bits from run to run; half 0's first ones overwrite the unit's dV/dK)
-              bool r = h == 0 ? grads_done[1] >= ti[h] - 1 : grads_done[0] >= ti[h];
-              r = r && ready(&c.pds_full[h], i & 1);
-              if (r && ti[h] == 0 && h == 0) r = n_units == 0 || ready(&c.acc_free, (n_units - 1) & 1);
+              bool r = ready(&c.pds_full[h], i & 1);
+              if (r && ti[h] == 0)
+                r = h == 0 ? (n_units == 0 || ready(&c.acc_free, (n_units - 1) & 1)) : grads_done[0] >= 0;
               if (!r) continue;
               tc_fence_after();
               issue_grads(i, h, ti[h] == 0);
