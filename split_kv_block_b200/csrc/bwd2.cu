@@ -62,19 +62,6 @@ constexpr int kCtl = kDS + 128 * 128 * 2;
 constexpr int kSmemBytes = kCtl + static_cast<int>(sizeof(Ctl));
 static_assert(kSmemBytes <= 232448, "shared memory budget");
 
-// Non-blocking test of an mbarrier phase.
-__device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-
 __device__ __forceinline__ uint32_t col_a(int h) { return 64u * h; }         // S^T, then P^T, of half h
 __device__ __forceinline__ uint32_t col_b(int h) { return 128u + 64u * h; }  // dP^T, then dQ^T, of half h
 constexpr uint32_t kColDV = 256, kColDK = 384;
@@ -232,39 +219,33 @@ __global__ void __launch_bounds__(384, 1)
     const uint64_t dS_mn = sdesc_sw128(smem_u32(smem + kDS), 16384, 1024);     // dS^T as B of dQ^T
     uint32_t n_units = 0, qc = 0, kv_waits = 0;
     bool ok = true;
-
-    // Warp-uniform, non-blocking test of a phase (lane 0's view).
-    auto ready = [&](uint64_t* bar, uint32_t parity) -> bool {
-      return __shfl_sync(0xffffffffu, mbar_test(bar, parity) ? 1 : 0, 0) != 0;
-    };
-    // The gradient MMAs of half h for global tile number i: dQ^T first (its read-out and reduction then
-    // overlap the half's dV and dK), dV, dK. `first`: the unit's first tile (half 0 overwrites dV/dK).
-    auto issue_grads = [&](uint32_t i, int h, bool first) {
+    // S^T and dP^T of half h of tile number i: rows 64h..64h+63 of its Q / dO tile, into A_h / B_h once
+    // half h of tile i - 1 has consumed A_h (its dV) and its dQ^T has been read out of B_h
+    auto issue_sdp = [&](uint32_t i, int h) -> bool {
       const int s = i & 1;
+      const uint32_t use = i >> 1;
+      if (!mbar_wait_warp(&c.q_full[s], use & 1, status, lim)) return false;
+      if (!mbar_wait_warp(&c.do_full[s], use & 1, status, lim)) return false;
+      if (i >= 1 && (!mbar_wait_warp(&c.dv_done[h], (i - 1) & 1, status, lim) ||
+                     !mbar_wait_warp(&c.dq_free[h], (i - 1) & 1, status, lim)))
+        return false;
+      tc_fence_after();
+      const uint32_t rows = s * kTileBytes + h * 8192;
       if (leader) {
 #pragma unroll
-        for (int ks = 0; ks < 128 / 16; ++ks)
-          umma_bf16(tmem + col_b(h), sdesc_add(dK_mn, ks * 2048), sdesc_add(dS_mn, h * 16384 + ks * 2048), idQ,
-                    ks > 0);
-        umma_commit(&c.dq_full[h]);
-        // dV += P^T dO over the half's 64 rows (A = P^T_h from TMEM)
-#pragma unroll
-        for (int k4 = 0; k4 < 4; ++k4) {
-          const uint32_t acc = (first && h == 0 && k4 == 0) ? 0u : 1u;
-          umma_bf16_ts(tmem + kColDV, tmem + col_a(h) + 8 * k4,
-                       sdesc_add(dDO_mn, s * kTileBytes + (64 * h + 16 * k4) * 128), idKV, acc);
+        for (int ks = 0; ks < kD / 16; ++ks) {
+          const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
+          umma_bf16(tmem + col_a(h), sdesc_add(dK_k, off), sdesc_add(dQ_k, rows + off), idS, ks > 0);
         }
-        umma_commit(&c.dv_done[h]);
-        // dK += dS^T Q over the half's rows (the next tile's dS^T is written only after its S^T/dP^T, whose
-        // commit covers this MMA)
 #pragma unroll
-        for (int k4 = 0; k4 < 4; ++k4) {
-          const uint32_t acc = (first && h == 0 && k4 == 0) ? 0u : 1u;
-          umma_bf16(tmem + kColDK, sdesc_add(dS_k, h * 16384 + k4 * 32),
-                    sdesc_add(dQ_mn, s * kTileBytes + (64 * h + 16 * k4) * 128), idKV, acc);
+        for (int ks = 0; ks < kD / 16; ++ks) {
+          const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
+          umma_bf16(tmem + col_b(h), sdesc_add(dV_k, off), sdesc_add(dDO_k, rows + off), idS, ks > 0);
         }
+        umma_commit(&c.sdp_full[h]);
       }
       __syncwarp();
+      return true;
     };
     while (ok) {
       const int slot = n_units & 1;
@@ -274,112 +255,78 @@ __global__ void __launch_bounds__(384, 1)
       if (leader) mbar_arrive(&c.sched_empty[slot]);
       if (u < 0) break;
       const BwdUnit U = p.units[u];
-      // The unit's live query tiles, counted by the whole warp (lane l tests tiles mt_begin + l, + 32, ...).
-      // The producer and the gradient warps walk the same tiles in the same order; the issuer needs only
-      // their number.
-      int n_live = 0;
-      for (int i0 = U.mt_begin; i0 < U.mt_end; i0 += 32) {
-        const int i = i0 + lane;
-        const bool live = i < U.mt_end && tile_live<kWalkMask>(p, p.mtiles[i], U.kbeg);
-        n_live += __popc(__ballot_sync(0xffffffffu, live));
-      }
-      if (n_live > 0) {
-        if (!mbar_wait_warp(&c.kv_full, (kv_waits++) & 1, status, lim)) break;
-        // The two halves advance independently: each issues S^T/dP^T of its next tile as soon as the tile's
-        // Q/dO are loaded and its A_h/B_h are free, and that tile's gradient MMAs as soon as its warpgroup has
-        // written P^T and dS^T; whichever half is ready goes first. Half 0 issues the unit's first gradient
-        // MMAs (they overwrite dV/dK) before half 1's; a Q/dO stage is released after both halves' gradient
-        // MMAs of its tile.
-        int ti[2] = {0, 0};          // unit-local index of the half's next tile
-        bool sdp_next[2] = {true, true};
-        int grads_done[2] = {-1, -1};  // last tile whose gradient MMAs the half issued
-        uint64_t idle_since = 0;
-        int spins = 0;
-        while (ti[0] < n_live || ti[1] < n_live) {
-          bool prog = false;
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            if (ti[h] >= n_live) continue;
-            const uint32_t i = qc + ti[h];  // global tile number: stage, phases
-            const int s = i & 1;
-            if (sdp_next[h]) {
-              bool r = ready(&c.q_full[s], (i >> 1) & 1) && ready(&c.do_full[s], (i >> 1) & 1);
-              // A_h and B_h of this half's previous tile (possibly the previous unit's last)
-              if (r && i >= 1) r = ready(&c.dv_done[h], (i - 1) & 1) && ready(&c.dq_free[h], (i - 1) & 1);
-              if (!r) continue;
-              tc_fence_after();
-              const uint32_t rows = s * kTileBytes + h * 8192;
-              if (leader) {
-#pragma unroll
-                for (int ks = 0; ks < kD / 16; ++ks) {
-                  const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
-                  umma_bf16(tmem + col_a(h), sdesc_add(dK_k, off), sdesc_add(dQ_k, rows + off), idS, ks > 0);
-                }
-#pragma unroll
-                for (int ks = 0; ks < kD / 16; ++ks) {
-                  const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
-                  umma_bf16(tmem + col_b(h), sdesc_add(dV_k, off), sdesc_add(dDO_k, rows + off), idS, ks > 0);
-                }
-                umma_commit(&c.sdp_full[h]);
-              }
-              __syncwarp();
-              sdp_next[h] = false;
-              prog = true;
-            } else {
-              bool r = ready(&c.pds_full[h], i & 1);
-              if (r && ti[h] == 0)
-                r = h == 0 ? (n_units == 0 || ready(&c.acc_free, (n_units - 1) & 1)) : grads_done[0] >= 0;
-              if (!r) continue;
-              tc_fence_after();
-              issue_grads(i, h, ti[h] == 0);
-              grads_done[h] = ti[h];
-              if (grads_done[1 - h] >= ti[h]) {  // both halves are done with this tile's Q/dO stage
-                if (leader) {
-                  umma_commit(&c.do_empty[s]);
-                  umma_commit(&c.q_empty[s]);
-                }
-                __syncwarp();
-              }
-              ++ti[h];
-              sdp_next[h] = true;
-              prog = true;
-            }
-          }
-          if (prog) {
-            idle_since = 0;
-            spins = 0;
-            continue;
-          }
-          // nothing ready: back off briefly (the gradient warps share this SM quarter), and give up after the
-          // wait limit or once another role has recorded an error
-          __nanosleep(32);
-          if (++spins < 64) continue;
-          spins = 0;
-          int give_up = 0;
-          if (lane == 0) {
-            const uint64_t now = globaltimer_ns();
-            if (idle_since == 0) idle_since = now;
-            if (*reinterpret_cast<volatile int*>(status) != 0) give_up = 1;
-            else if (now - idle_since > lim) {
-              atomicCAS(status, 0, kStatusTimeout);
-              give_up = 1;
-            }
-          }
-          if (__shfl_sync(0xffffffffu, give_up, 0)) {
+      bool first = true;
+      // live query tiles in order (mt, then nxt); the liveness of the tile after nxt is loaded at the top of
+      // a tile and read at its end, so no load stalls the issue of a tile's MMAs
+      auto live_from = [&](int i) -> int {
+        while (i < U.mt_end && !tile_live<kWalkMask>(p, p.mtiles[i], U.kbeg)) ++i;
+        return i;
+      };
+      int mt = live_from(U.mt_begin);
+      int nxt = mt < U.mt_end ? live_from(mt + 1) : U.mt_end;
+      while (mt < U.mt_end) {
+        const bool live_c = nxt < U.mt_end && nxt + 1 < U.mt_end && tile_live<kWalkMask>(p, p.mtiles[nxt + 1], U.kbeg);
+        const int s = qc & 1;
+        if (first) {  // a unit's first tile waits for the unit's K/V
+          if (!mbar_wait_warp(&c.kv_full, (kv_waits++) & 1, status, lim)) { ok = false; break; }
+          if (!issue_sdp(qc, 0) || !issue_sdp(qc, 1)) { ok = false; break; }
+        }
+        for (int h = 0; h < 2 && ok; ++h) {
+          if (!mbar_wait_warp(&c.pds_full[h], qc & 1, status, lim)) { ok = false; break; }
+          if (first && h == 0 && n_units >= 1 && !mbar_wait_warp(&c.acc_free, (n_units - 1) & 1, status, lim)) {
             ok = false;
             break;
           }
+          tc_fence_after();
+          if (leader) {
+            // dQ^T of the half's rows = K^T dS^T -> B_h, first: the gradient warps read it out and reduce it
+            // while the tensor core runs the half's dV and dK
+#pragma unroll
+            for (int ks = 0; ks < 128 / 16; ++ks)
+              umma_bf16(tmem + col_b(h), sdesc_add(dK_mn, ks * 2048), sdesc_add(dS_mn, h * 16384 + ks * 2048), idQ,
+                        ks > 0);
+            umma_commit(&c.dq_full[h]);
+            // dV += P^T dO over the half's 64 rows (A = P^T_h from TMEM)
+#pragma unroll
+            for (int k4 = 0; k4 < 4; ++k4) {
+              const uint32_t acc = (first && h == 0 && k4 == 0) ? 0u : 1u;
+              umma_bf16_ts(tmem + kColDV, tmem + col_a(h) + 8 * k4,
+                           sdesc_add(dDO_mn, s * kTileBytes + (64 * h + 16 * k4) * 128), idKV, acc);
+            }
+            umma_commit(&c.dv_done[h]);
+            if (h == 1) umma_commit(&c.do_empty[s]);
+            // dK += dS^T Q over the half's rows (the next tile's dS^T is written only after its S^T/dP^T, whose
+            // commit covers this MMA)
+#pragma unroll
+            for (int k4 = 0; k4 < 4; ++k4) {
+              const uint32_t acc = (first && h == 0 && k4 == 0) ? 0u : 1u;
+              umma_bf16(tmem + kColDK, sdesc_add(dS_k, h * 16384 + k4 * 32),
+                        sdesc_add(dQ_mn, s * kTileBytes + (64 * h + 16 * k4) * 128), idKV, acc);
+            }
+            if (h == 1) umma_commit(&c.q_empty[s]);
+          }
+          __syncwarp();
+          // this half of the unit's next tile, as soon as A_h and B_h are free
+          if (nxt < U.mt_end && !issue_sdp(qc + 1, h)) { ok = false; break; }
         }
         if (!ok) break;
-        qc += n_live;
-      } else if (n_units >= 1 && !mbar_wait_warp(&c.acc_free, (n_units - 1) & 1, status, lim)) {
-        // A unit without live query tiles (possible under a block mask) issues no MMA; it still waits for
-        // the previous unit's dK/dV read-out before signalling its own, so that acc_full never runs two
-        // phases ahead of the gradient warps (its parity would then name the wrong phase).
-        break;
+        first = false;
+        ++qc;
+        int nn = U.mt_end;
+        if (nxt < U.mt_end) {
+          nn = nxt + 1;
+          if (nn < U.mt_end && !live_c) nn = live_from(nn + 1);
+        }
+        mt = nxt;
+        nxt = nn;
       }
+      if (!ok) break;
+      // A unit without live query tiles (possible under a block mask) issues no MMA; it still waits for the
+      // previous unit's dK/dV read-out before signalling its own, so that acc_full never runs two phases ahead
+      // of the gradient warps (its parity would then name the wrong phase).
+      if (first && n_units >= 1 && !mbar_wait_warp(&c.acc_free, (n_units - 1) & 1, status, lim)) break;
       if (leader) {
-        if (n_live > 0) umma_commit(&c.kv_empty);  // K/V were loaded for this unit
+        if (!first) umma_commit(&c.kv_empty);  // K/V were loaded for this unit
         umma_commit(&c.acc_full);
       }
       __syncwarp();
