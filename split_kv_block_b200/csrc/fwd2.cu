@@ -1,5 +1,5 @@
-// Split-KV forward on sm_100a, head_dim 128: two query tiles per CTA, scores
-// in 64-key sub-tiles with two score buffers per query tile.
+// Split-KV forward on sm_100a (head_dim 64 and 128): two query tiles per CTA,
+// scores in 64-key sub-tiles with two score buffers per query tile.
 //
 // Same mathematics as fwd.cu (per forward unit: partial softmax
 // attention of one 128-row query tile over one item's key range, normalized
@@ -33,13 +33,7 @@
 namespace skv {
 namespace {
 
-constexpr int kD = 128;
-constexpr int kSub = 64;                   // keys per score sub-tile
-constexpr int kTileBytes = 128 * kD * 2;   // a 128 x 128 bf16 tile
-constexpr int kQ0 = 0;                     // Q of tile 0 and tile 1
-constexpr int kK0 = kQ0 + 2 * kTileBytes;  // two K stages
-constexpr int kV0 = kK0 + 2 * kTileBytes;  // two V stages
-constexpr int kCtl = kV0 + 2 * kTileBytes;
+constexpr int kSub = 64;  // keys per score sub-tile
 
 struct Ctl {
   uint64_t sched_full[2], sched_empty[2];
@@ -55,8 +49,20 @@ struct Ctl {
   uint32_t tmem_base;
   int32_t merge_slot;  // tail merge: slot being merged (broadcast)
 };
-constexpr int kSmemBytes = kCtl + static_cast<int>(sizeof(Ctl));
-static_assert(kSmemBytes <= 232448, "shared memory budget");
+// Shared memory of the head_dim-D kernel: Q of both query tiles, two K and two V stages. A tile is 128
+// rows of D bf16, stored as D / 64 column groups of 128 rows x 128 bytes (one 128-byte swizzle atom per
+// row), 16 KB each.
+template <int D>
+struct FwdLayout {
+  static constexpr int kHalves = D / 64;              // 64-column groups of a row
+  static constexpr int kTileBytes = 128 * D * 2;      // a 128 x D bf16 tile
+  static constexpr int kQ0 = 0;                       // Q of tile 0 and tile 1
+  static constexpr int kK0 = kQ0 + 2 * kTileBytes;    // two K stages
+  static constexpr int kV0 = kK0 + 2 * kTileBytes;    // two V stages
+  static constexpr int kCtl = kV0 + 2 * kTileBytes;
+  static constexpr int kSmemBytes = kCtl + static_cast<int>(sizeof(Ctl));
+  static_assert(kSmemBytes <= 232448, "shared memory budget");
+};
 
 __device__ __forceinline__ uint32_t col_s(int t, int b) { return 128u * t + 64u * b; }  // score buffer b of tile t
 __device__ __forceinline__ uint32_t col_o(int t) { return 256u + 128u * t; }            // O of tile t
@@ -112,12 +118,14 @@ __device__ __forceinline__ float exp_row64(const uint32_t (&sv)[64], float sl2, 
 
 // kMerge: the LSE merge runs in the kernel's tail (skv_attn_fwd_merged). kMask: a block-sparse mask;
 // every role walks the pair's list of live key tiles and the softmax masks the rows whose block is off.
-template <bool kMerge, bool kMask>
+template <int D, bool kMerge, bool kMask>
 __global__ void __launch_bounds__(384, 1)
     fwd2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                 const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
+  using L = FwdLayout<D>;
+  constexpr int kD = D, kTileBytes = L::kTileBytes, kQ0 = L::kQ0, kK0 = L::kK0, kV0 = L::kV0;
   extern __shared__ __align__(1024) uint8_t smem[];
-  Ctl& c = *reinterpret_cast<Ctl*>(smem + kCtl);
+  Ctl& c = *reinterpret_cast<Ctl*>(smem + L::kCtl);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   int* status = p.status;
   const uint64_t lim = p.timeout_ns;
@@ -188,7 +196,7 @@ __global__ void __launch_bounds__(384, 1)
           const MTile M = p.mtiles[U.mt];
           if (q_iss[t] >= 1 && !mbar_wait(&c.q_empty[t], (q_iss[t] - 1) & 1, status, lim)) { ok = false; break; }
           mbar_arrive_expect_tx(&c.q_full[t], kTileBytes);
-          for (int db = 0; db < 2; ++db)
+          for (int db = 0; db < L::kHalves; ++db)
             tma_load_3d(smem + kQ0 + t * kTileBytes + db * 16384, &tmQ, &c.q_full[t], db * 64, U.g * p.G, M.tok0);
           ++q_iss[t];
         }
@@ -201,12 +209,12 @@ __global__ void __launch_bounds__(384, 1)
           const uint32_t use = kv >> 1;
           if (use >= 1 && !mbar_wait(&c.k_empty[st], (use - 1) & 1, status, lim)) { ok = false; break; }
           mbar_arrive_expect_tx(&c.k_full[st], kTileBytes);
-          for (int db = 0; db < 2; ++db)
+          for (int db = 0; db < L::kHalves; ++db)
             tma_load_3d(smem + kK0 + st * kTileBytes + db * 16384, &tmK, &c.k_full[st], db * 64, kvh, kb - kshift);
           ++k_iss;
           if (use >= 1 && !mbar_wait(&c.v_empty[st], (use - 1) & 1, status, lim)) { ok = false; break; }
           mbar_arrive_expect_tx(&c.v_full[st], kTileBytes);
-          for (int db = 0; db < 2; ++db)
+          for (int db = 0; db < L::kHalves; ++db)
             tma_load_3d(smem + kV0 + st * kTileBytes + db * 16384, &tmV, &c.v_full[st], db * 64, kvh, kb - kshift);
           ++v_iss;
         }
@@ -465,16 +473,23 @@ __global__ void __launch_bounds__(384, 1)
 
 }  // namespace
 
-int fwd2_smem_bytes() { return kSmemBytes; }
-
-cudaError_t launch_fwd2(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const FwdParams& p,
-                        int grid, cudaStream_t stream) {
-  auto kern = p.tile_mask ? (p.o ? fwd2_kernel<true, true> : fwd2_kernel<false, true>)
-                          : (p.o ? fwd2_kernel<true, false> : fwd2_kernel<false, false>);
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+template <int D>
+cudaError_t launch_fwd2_d(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const FwdParams& p,
+                          int grid, cudaStream_t stream) {
+  auto kern = p.tile_mask ? (p.o ? fwd2_kernel<D, true, true> : fwd2_kernel<D, false, true>)
+                          : (p.o ? fwd2_kernel<D, true, false> : fwd2_kernel<D, false, false>);
+  constexpr int smem = FwdLayout<D>::kSmemBytes;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  kern<<<grid, 384, kSmemBytes, stream>>>(tq, tk, tv, p);
+  kern<<<grid, 384, smem, stream>>>(tq, tk, tv, p);
   return cudaGetLastError();
+}
+
+int fwd2_smem_bytes(int d) { return d == 64 ? FwdLayout<64>::kSmemBytes : FwdLayout<128>::kSmemBytes; }
+
+cudaError_t launch_fwd2(int d, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                        const FwdParams& p, int grid, cudaStream_t stream) {
+  return d == 64 ? launch_fwd2_d<64>(tq, tk, tv, p, grid, stream) : launch_fwd2_d<128>(tq, tk, tv, p, grid, stream);
 }
 
 }  // namespace skv

@@ -95,9 +95,9 @@ int fwd_smem_bytes(int d);
 int bwd_smem_bytes(int d);
 cudaError_t launch_fwd(int d, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                        const FwdParams& p, int grid, cudaStream_t stream);
-cudaError_t launch_fwd2(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const FwdParams& p,
-                        int grid, cudaStream_t stream);  // head_dim 128: pairs of query tiles
-int fwd2_smem_bytes();
+cudaError_t launch_fwd2(int d, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                        const FwdParams& p, int grid, cudaStream_t stream);  // pairs of query tiles
+int fwd2_smem_bytes(int d);
 // CTAs of the forward launch: one per SM, at most one per work unit (pair for head_dim 128)
 int fwd_grid(int d, int sms, long long n_units, long long n_pairs);
 cudaError_t launch_merge(int d, const MergeParams& p, cudaStream_t stream);
