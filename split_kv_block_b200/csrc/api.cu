@@ -255,7 +255,7 @@ int run_fwd(const PlanHeader* h, const void* plan, const void* q, const void* k,
   }
   int sms = num_sms();
   if (sms <= 0) return cuda_fail(cudaGetLastError());
-  const int grid = fwd_grid(h->d, sms, h->n_fwd, h->n_fwd_pairs);
+  const int grid = fwd_grid(sms, h->n_fwd_pairs);
   cudaError_t e = mark(SKV_KERNEL_FWD, 0, stream);
   if (e == cudaSuccess) e = launch_fwd(h->d, tq, tk, tv, p, grid, stream);
   if (e == cudaSuccess) e = mark(SKV_KERNEL_FWD, 1, stream);

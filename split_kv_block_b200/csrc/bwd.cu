@@ -389,7 +389,6 @@ __global__ void __launch_bounds__(256, 1)
   }
 }
 
-int bwd_smem_bytes(int d) { return d == 64 ? BwdSmem<64>::kDyn : bwd2_smem_bytes(); }
 
 cudaError_t launch_bwd(int d, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                        const CUtensorMap& tdo, const BwdParams& p, int grid, cudaStream_t stream) {

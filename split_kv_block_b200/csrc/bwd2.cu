@@ -586,8 +586,6 @@ __global__ void __launch_bounds__(384, 1)
 
 }  // namespace
 
-int bwd2_smem_bytes() { return kSmemBytes; }
-
 cudaError_t launch_bwd2(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tdo,
                         const BwdParams& p, int grid, cudaStream_t stream) {
   const bool m = p.tile_mask != nullptr;

@@ -18,18 +18,12 @@
 
 namespace skv {
 
-int fwd_smem_bytes(int d) { return fwd2_smem_bytes(d); }
-
 cudaError_t launch_fwd(int d, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                        const FwdParams& p, int grid, cudaStream_t stream) {
   return launch_fwd2(d, tq, tk, tv, p, grid, stream);
 }
 
 // one persistent CTA per SM, at most one per pair of forward units
-int fwd_grid(int d, int sms, long long n_units, long long n_pairs) {
-  (void)d;
-  (void)n_units;
-  return static_cast<int>(n_pairs < sms ? n_pairs : sms);
-}
+int fwd_grid(int sms, long long n_pairs) { return static_cast<int>(n_pairs < sms ? n_pairs : sms); }
 
 }  // namespace skv

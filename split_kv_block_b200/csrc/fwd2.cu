@@ -485,8 +485,6 @@ cudaError_t launch_fwd2_d(const CUtensorMap& tq, const CUtensorMap& tk, const CU
   return cudaGetLastError();
 }
 
-int fwd2_smem_bytes(int d) { return d == 64 ? FwdLayout<64>::kSmemBytes : FwdLayout<128>::kSmemBytes; }
-
 cudaError_t launch_fwd2(int d, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                         const FwdParams& p, int grid, cudaStream_t stream) {
   return d == 64 ? launch_fwd2_d<64>(tq, tk, tv, p, grid, stream) : launch_fwd2_d<128>(tq, tk, tv, p, grid, stream);

@@ -91,15 +91,12 @@ struct BwdParams {
   float scale_log2;         // log2(e) / sqrt(d)
 };
 
-int fwd_smem_bytes(int d);
-int bwd_smem_bytes(int d);
 cudaError_t launch_fwd(int d, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                        const FwdParams& p, int grid, cudaStream_t stream);
 cudaError_t launch_fwd2(int d, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                         const FwdParams& p, int grid, cudaStream_t stream);  // pairs of query tiles
-int fwd2_smem_bytes(int d);
-// CTAs of the forward launch: one per SM, at most one per work unit (pair for head_dim 128)
-int fwd_grid(int d, int sms, long long n_units, long long n_pairs);
+// CTAs of the forward launch: one per SM, at most one per pair of forward units
+int fwd_grid(int sms, long long n_pairs);
 cudaError_t launch_merge(int d, const MergeParams& p, cudaStream_t stream);
 // D = rowsum(dO * O) and the zeroed dQ accumulator per (token, head) row; also zeroes dK/dV of
 // the K/V rows no query attends to (rows dead[2i] .. dead[2i+1] for i < n_dead, device array;
@@ -111,7 +108,6 @@ cudaError_t launch_bwd(int d, const CUtensorMap& tq, const CUtensorMap& tk, cons
                        const CUtensorMap& tdo, const BwdParams& p, int grid, cudaStream_t stream);
 cudaError_t launch_bwd2(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tdo,
                         const BwdParams& p, int grid, cudaStream_t stream);  // head_dim 128
-int bwd2_smem_bytes();
 cudaError_t launch_dq_cast(const float* dq_acc, __nv_bfloat16* dq, float scale, long long n, cudaStream_t stream);
 cudaError_t launch_dq_scale(const float* dq_acc, float* dq, float scale, long long n, cudaStream_t stream);
 // Context parallelism: combine of the ranks' (O_r, LSE_r), and the sum of the ranks' fp32 dQ partials.

@@ -127,7 +127,7 @@ extern "C" int skv_attn_fwd_noalloc(const void* plan, const skv_problem* prob, c
   e = cudaGetDevice(&dev_id);
   if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev_id);
   if (e != cudaSuccess) return skv_record_cuda_error(static_cast<int>(e));
-  const int grid = fwd_grid(h->d, sms, h->n_fwd, h->n_fwd_pairs);
+  const int grid = fwd_grid(sms, h->n_fwd_pairs);
   e = launch_fwd(h->d, tq, tk, tv, p, grid, stream);
   if (e != cudaSuccess) return skv_record_cuda_error(static_cast<int>(e));
 
