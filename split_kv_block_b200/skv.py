@@ -356,9 +356,10 @@ def check_inputs(plan: Plan, q, k, v, do=None):
             raise ValueError(f"{name}: expected contiguous cuda bf16 {shape}, got {tuple(t.shape)} {t.dtype} {t.device}")
 
 
-def forward(plan: Plan, q, k, v, ws=None, stream=None, fused=True):
-    """Split-KV forward + LSE merge: one launch (fused, the default) or the
-    forward and merge calls in turn. Returns (o bf16 [Nq,Hq,d], lse fp32 [Nq,Hq])."""
+def forward(plan: Plan, q, k, v, ws=None, stream=None, fused=False):
+    """Split-KV forward + LSE merge: the forward and merge calls in turn (the
+    default, the faster on B200), or one launch with the merge in the
+    forward's tail (fused). Returns (o bf16 [Nq,Hq,d], lse fp32 [Nq,Hq])."""
     import torch
     check_inputs(plan, q, k, v)
     if ws is None:
