@@ -21,7 +21,7 @@
 //     reduction into the shared dQ accumulator writes 128 consecutive floats
 //     of a row per warpgroup instruction.
 //   * Q and dO tiles are double-buffered.
-// Warp roles: 0 scheduler + TMA producer, 1 and 3 MMA issuers of halves 0 and 1, 2 TMEM allocator,
+// Warp roles: 0 scheduler + TMA producer, 1 MMA issuer, 2 TMEM allocator,
 // 4..7 warpgroup 0 (rows 0..63), 8..11 warpgroup 1 (rows 64..127).
 #include <cuda_runtime.h>
 
@@ -48,8 +48,7 @@ struct Ctl {
   uint64_t dq_full[2], dq_free[2];
   uint64_t acc_full, acc_free;
   uint64_t meta_full[2][2];  // [warpgroup][tile parity]
-  uint64_t grads_issued[2];  // per half: its gradient MMAs of a tile are issued (orders the halves' dV/dK)
-  uint64_t final_mma[2];
+  uint64_t final_mma;
   int32_t sched[2];
   uint32_t tmem_base;
 };
@@ -94,13 +93,11 @@ __global__ void __launch_bounds__(384, 1)
   if (tid == 0) {
     for (int i = 0; i < 2; ++i) {
       mbar_init(&c.sched_full[i], 1);
-      mbar_init(&c.sched_empty[i], 2 + 8);  // both issuers and the eight gradient warps
+      mbar_init(&c.sched_empty[i], 1 + 8);
       mbar_init(&c.q_full[i], 1);
-      mbar_init(&c.q_empty[i], 2);          // released by both issuers
+      mbar_init(&c.q_empty[i], 1);
       mbar_init(&c.do_full[i], 1);
-      mbar_init(&c.do_empty[i], 2);
-      mbar_init(&c.grads_issued[i], 1);
-      mbar_init(&c.final_mma[i], 1);
+      mbar_init(&c.do_empty[i], 1);
       mbar_init(&c.pds_full[i], 128);
       mbar_init(&c.sdp_full[i], 1);
       mbar_init(&c.dv_done[i], 1);
@@ -110,9 +107,10 @@ __global__ void __launch_bounds__(384, 1)
       mbar_init(&c.meta_full[i][1], 128);
     }
     mbar_init(&c.kv_full, 1);
-    mbar_init(&c.kv_empty, 2);
-    mbar_init(&c.acc_full, 2);
+    mbar_init(&c.kv_empty, 1);
+    mbar_init(&c.acc_full, 1);
     mbar_init(&c.acc_free, 256);
+    mbar_init(&c.final_mma, 1);
     fence_mbar_init();
   }
   if (warp == 2) {
@@ -201,15 +199,10 @@ __global__ void __launch_bounds__(384, 1)
         }
       }
     }
-  } else if (warp == 1 || warp == 3) {
-    // ------------------------------------------------ MMA issuer of half h
-    // One warp per half (warp 1: rows 0..63, warp 3: rows 64..127), each running its half's fixed sequence
-    // with blocking waits, so a half waiting for its buffers never holds up the other. The halves' gradient
-    // MMAs alternate (half 0 of tile i, half 1 of tile i, half 0 of tile i + 1, ...), so dV and dK
-    // accumulate in a fixed order and half 0's first MMAs of a unit (which overwrite dV/dK) come first.
+  } else if (warp == 1) {
+    // ---------------------------------------------------------- MMA issuer
     // All 32 lanes run the loop (stage indices and descriptors stay warp-uniform); one elected lane issues
     // the MMAs and their commits.
-    const int h = warp == 1 ? 0 : 1;
     const bool leader = elect_one();
     constexpr uint32_t idS = idesc_bf16(128, 64, false, false);   // S^T_h = K Q_h^T, dP^T_h = V dO_h^T
     constexpr uint32_t idKV = idesc_bf16(128, kD, false, true);   // dV += P^T dO, dK += dS^T Q (half's rows)
@@ -276,54 +269,47 @@ __global__ void __launch_bounds__(384, 1)
         const int s = qc & 1;
         if (first) {  // a unit's first tile waits for the unit's K/V
           if (!mbar_wait_warp(&c.kv_full, (kv_waits++) & 1, status, lim)) { ok = false; break; }
-          if (!issue_sdp(qc, h)) { ok = false; break; }
+          if (!issue_sdp(qc, 0) || !issue_sdp(qc, 1)) { ok = false; break; }
         }
-        // this half's gradient MMAs of tile qc: after its warpgroup has written P^T and dS^T, and after the
-        // other half's previous gradient MMAs (half 0 of tile qc before half 1 of tile qc before half 0 of
-        // tile qc + 1); half 0's first ones of a unit also wait for the previous unit's dK/dV read-out
-        if (!mbar_wait_warp(&c.pds_full[h], qc & 1, status, lim)) { ok = false; break; }
-        if (h == 0) {
-          if (qc >= 1 && !mbar_wait_warp(&c.grads_issued[1], (qc - 1) & 1, status, lim)) { ok = false; break; }
-          if (first && n_units >= 1 && !mbar_wait_warp(&c.acc_free, (n_units - 1) & 1, status, lim)) {
+        for (int h = 0; h < 2 && ok; ++h) {
+          if (!mbar_wait_warp(&c.pds_full[h], qc & 1, status, lim)) { ok = false; break; }
+          if (first && h == 0 && n_units >= 1 && !mbar_wait_warp(&c.acc_free, (n_units - 1) & 1, status, lim)) {
             ok = false;
             break;
           }
-        } else if (!mbar_wait_warp(&c.grads_issued[0], qc & 1, status, lim)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        if (leader) {
-          // dQ^T of the half's rows = K^T dS^T -> B_h, first: the gradient warps read it out and reduce it
-          // while the tensor core runs the half's dV and dK
+          tc_fence_after();
+          if (leader) {
+            // dQ^T of the half's rows = K^T dS^T -> B_h, first: the gradient warps read it out and reduce it
+            // while the tensor core runs the half's dV and dK
 #pragma unroll
-          for (int ks = 0; ks < 128 / 16; ++ks)
-            umma_bf16(tmem + col_b(h), sdesc_add(dK_mn, ks * 2048), sdesc_add(dS_mn, h * 16384 + ks * 2048), idQ,
-                      ks > 0);
-          umma_commit(&c.dq_full[h]);
-          // dV += P^T dO over the half's 64 rows (A = P^T_h from TMEM)
+            for (int ks = 0; ks < 128 / 16; ++ks)
+              umma_bf16(tmem + col_b(h), sdesc_add(dK_mn, ks * 2048), sdesc_add(dS_mn, h * 16384 + ks * 2048), idQ,
+                        ks > 0);
+            umma_commit(&c.dq_full[h]);
+            // dV += P^T dO over the half's 64 rows (A = P^T_h from TMEM)
 #pragma unroll
-          for (int k4 = 0; k4 < 4; ++k4) {
-            const uint32_t acc = (first && h == 0 && k4 == 0) ? 0u : 1u;
-            umma_bf16_ts(tmem + kColDV, tmem + col_a(h) + 8 * k4,
-                         sdesc_add(dDO_mn, s * kTileBytes + (64 * h + 16 * k4) * 128), idKV, acc);
+            for (int k4 = 0; k4 < 4; ++k4) {
+              const uint32_t acc = (first && h == 0 && k4 == 0) ? 0u : 1u;
+              umma_bf16_ts(tmem + kColDV, tmem + col_a(h) + 8 * k4,
+                           sdesc_add(dDO_mn, s * kTileBytes + (64 * h + 16 * k4) * 128), idKV, acc);
+            }
+            umma_commit(&c.dv_done[h]);
+            if (h == 1) umma_commit(&c.do_empty[s]);
+            // dK += dS^T Q over the half's rows (the next tile's dS^T is written only after its S^T/dP^T, whose
+            // commit covers this MMA)
+#pragma unroll
+            for (int k4 = 0; k4 < 4; ++k4) {
+              const uint32_t acc = (first && h == 0 && k4 == 0) ? 0u : 1u;
+              umma_bf16(tmem + kColDK, sdesc_add(dS_k, h * 16384 + k4 * 32),
+                        sdesc_add(dQ_mn, s * kTileBytes + (64 * h + 16 * k4) * 128), idKV, acc);
+            }
+            if (h == 1) umma_commit(&c.q_empty[s]);
           }
-          umma_commit(&c.dv_done[h]);
-          umma_commit(&c.do_empty[s]);  // released once both halves' MMAs reading it have completed
-          // dK += dS^T Q over the half's rows (the next tile's dS^T is written only after its S^T/dP^T, whose
-          // commit covers this MMA)
-#pragma unroll
-          for (int k4 = 0; k4 < 4; ++k4) {
-            const uint32_t acc = (first && h == 0 && k4 == 0) ? 0u : 1u;
-            umma_bf16(tmem + kColDK, sdesc_add(dS_k, h * 16384 + k4 * 32),
-                      sdesc_add(dQ_mn, s * kTileBytes + (64 * h + 16 * k4) * 128), idKV, acc);
-          }
-          umma_commit(&c.q_empty[s]);
-          mbar_arrive(&c.grads_issued[h]);  // issued, so the other half's next gradient MMAs queue behind them
+          __syncwarp();
+          // this half of the unit's next tile, as soon as A_h and B_h are free
+          if (nxt < U.mt_end && !issue_sdp(qc + 1, h)) { ok = false; break; }
         }
-        __syncwarp();
-        // this half of the unit's next tile, as soon as A_h and B_h are free
-        if (nxt < U.mt_end && !issue_sdp(qc + 1, h)) { ok = false; break; }
+        if (!ok) break;
         first = false;
         ++qc;
         int nn = U.mt_end;
@@ -335,9 +321,9 @@ __global__ void __launch_bounds__(384, 1)
         nxt = nn;
       }
       if (!ok) break;
-      // A unit without live query tiles (possible under a block mask) issues no MMA; both issuers still wait
-      // for the previous unit's dK/dV read-out before signalling their part of its acc_full, so that acc_full
-      // never runs two phases ahead of the gradient warps (its parity would then name the wrong phase).
+      // A unit without live query tiles (possible under a block mask) issues no MMA; it still waits for the
+      // previous unit's dK/dV read-out before signalling its own, so that acc_full never runs two phases ahead
+      // of the gradient warps (its parity would then name the wrong phase).
       if (first && n_units >= 1 && !mbar_wait_warp(&c.acc_free, (n_units - 1) & 1, status, lim)) break;
       if (leader) {
         if (!first) umma_commit(&c.kv_empty);  // K/V were loaded for this unit
@@ -346,9 +332,9 @@ __global__ void __launch_bounds__(384, 1)
       __syncwarp();
       ++n_units;
     }
-    if (leader) umma_commit(&c.final_mma[h]);
+    if (leader) umma_commit(&c.final_mma);
     __syncwarp();
-    mbar_wait_warp(&c.final_mma[h], 0, nullptr, lim);
+    mbar_wait_warp(&c.final_mma, 0, nullptr, lim);
   } else if (warp >= 4) {
     // ------------------------- softmax gradient, dQ drain, dK/dV epilogue
     const int wg = (warp - 4) >> 2;          // warpgroup: rows [64 wg, 64 wg + 64) of the tile
