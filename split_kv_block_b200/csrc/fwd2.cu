@@ -1,16 +1,16 @@
 // Split-KV forward on sm_100a (head_dim 64 and 128): two query tiles per CTA,
 // scores in 64-key sub-tiles with two score buffers per query tile.
 //
-// Same mathematics as fwd.cu (per forward unit: partial softmax
-// attention of one 128-row query tile over one item's key range, normalized
-// partial output and log-sum-exp; "Split-KV: Breaking the Context
-// Parallelism Bottleneck in Diffusion Drafter Training", section "Split-KV's
-// Core Mechanism"), arranged so that the tensor core does not wait for the
-// softmax:
+// Per forward unit: the partial softmax attention of one 128-row query tile
+// over one item's key range, its normalized partial output and log-sum-exp
+// ("Split-KV: Breaking the Context Parallelism Bottleneck in Diffusion
+// Drafter Training", section "Split-KV's Core Mechanism"; the masking rules
+// are stated in fwd.cu), arranged so that the tensor core does not wait for
+// the softmax:
 //   * a work unit is a pair of forward units of the same item; every 128-key
 //     K/V tile loaded by TMA serves both query tiles;
 //   * scores come in sub-tiles of 64 keys (S = Q K^T with N = 64). Each query
-//     tile has two 64-column score buffers in TMEM and its 128-column O.
+//     tile has two 64-column score buffers in TMEM and its O (D columns).
 //     P overwrites the first 32 columns of its buffer (bf16 pairs) and feeds
 //     O += P V from TMEM. While the softmax works on one buffer, the next
 //     sub-tile's S is computed into the other, so a tile's softmax runs from

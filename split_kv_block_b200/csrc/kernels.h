@@ -14,7 +14,7 @@ struct FwdParams {
   const int32_t* tok_kend;
   const FwdUnit* units;
   const int32_t* part_off;  // [P+1] units of each work queue
-  const FwdPair* pairs;     // head_dim 128 kernel: pairs of units
+  const FwdPair* pairs;     // pairs of forward units (two query tiles per CTA)
   const int32_t* pair_off;  // [P+1] pairs of each work queue
   int32_t* counters;        // [P] queue heads, zero at launch (P: the plan's work queues)
   int* status;
