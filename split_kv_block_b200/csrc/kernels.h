@@ -77,9 +77,9 @@ struct BwdParams {
   long long* stamps;
   unsigned long long timeout_ns;
   // Deterministic dQ (det != 0): units are taken from det_order through counters[0] instead of the
-  // partition queues, and each warp adds its dQ rows with a plain read-modify-write once the turn
-  // counter of its (query tile, kv head, warp) equals the unit's rank, so the fp32 sum over key tiles
-  // runs in ascending key order whatever the timing.
+  // work queues, and each warp adds its dQ rows (fp32 reductions that complete before the turn passes)
+  // once the turn counter of its (query tile, kv head, warp) equals the unit's rank, so the fp32 sum
+  // over key tiles runs in ascending key order whatever the timing.
   const int32_t* rank;      // [n_bwd]
   const int32_t* det_order; // [n_bwd]
   int32_t* turn;            // [n_mtiles * Hkv][8], zero at launch
