@@ -399,7 +399,8 @@ def run_workload(args, name, steps, warmup, rank, world, local_rank, e2e, sub_ch
         kernels["bwd"] = tensor_roof("bwd_kernel", f_bwd_all / K, kms[skv.SKV_KERNEL_BWD])
     roofline = dict(kernels["bwd" if backward else "fwd"])
     roofline["step_frac"] = round(flops_rank / K / (peaks["bf16_tflops"] * 1e12) / (total / K), 4)
-    kernels_per_step = (1 if fused else 2) + (3 if backward else 0)
+    # forward: plan upload, forward (+ merge); backward: plan upload, prep, backward, dQ cast
+    kernels_per_step = (2 if fused else 3) + (4 if backward else 0)
 
     rec = {
         "workload": f"{name}: {WORKLOAD_TEXT[name]}", "value": round(value, 3), "unit": "TFLOP/s", "steps": K,

@@ -36,7 +36,11 @@ int cuda_fail(cudaError_t e) {
 // The plan's device section is copied into the workspace from a pinned
 // staging slot owned by the library; each slot is reused only after the copy
 // that read it has completed, so the caller may reuse its plan buffer as soon
-// as a call returns.
+// as a call returns. The slots are mapped host memory (portable, so a kernel
+// on any GPU of the process reads them), and the copy is a kernel that reads
+// them over the bus: on B200 a copy-engine transfer between two kernels of one
+// stream took about 9 us of stream time for any size up to 160 KB, and the
+// kernel takes 2.5 to 5 us less per call on the 160 KB plan of a 32K context.
 struct Staging {
   void* host = nullptr;
   size_t cap = 0;
@@ -49,8 +53,21 @@ Staging g_stage[kSlots];
 int g_stage_next = 0;
 std::vector<void*> g_retired;  // outgrown staging buffers, released with the process
 
+// Copies `total` bytes from mapped host memory `src` to device memory `dst`
+// (both 16-byte aligned): 16 bytes per thread and step, the last total % 16
+// bytes by the first threads of block 0.
+__global__ void __launch_bounds__(256) upload_kernel(uint4* __restrict__ dst, const uint4* __restrict__ src,
+                                                     size_t n16, size_t total) {
+  const size_t stride = static_cast<size_t>(gridDim.x) * blockDim.x;
+  for (size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n16; i += stride) dst[i] = src[i];
+  const size_t tail = total - n16 * 16;
+  if (blockIdx.x == 0 && threadIdx.x < tail)
+    reinterpret_cast<uint8_t*>(dst)[n16 * 16 + threadIdx.x] =
+        reinterpret_cast<const uint8_t*>(src)[n16 * 16 + threadIdx.x];
+}
+
 // Copies `zeros` zero bytes followed by the n bytes at src to dst, in one
-// host-to-device copy.
+// launch of upload_kernel from the staging slot.
 int upload(const void* src, size_t n, void* dst, cudaStream_t stream, size_t zeros = 0) {
   std::lock_guard<std::mutex> lock(g_stage_mu);
   Staging& s = g_stage[g_stage_next];
@@ -74,7 +91,7 @@ int upload(const void* src, size_t n, void* dst, cudaStream_t stream, size_t zer
     size_t cap = size_t(1) << 20;
     while (cap < total) cap <<= 1;
     void* fresh = nullptr;
-    e = cudaHostAlloc(&fresh, cap, cudaHostAllocDefault);
+    e = cudaHostAlloc(&fresh, cap, cudaHostAllocMapped | cudaHostAllocPortable);
     if (e != cudaSuccess) return cuda_fail(e);
     if (s.host) g_retired.push_back(s.host);
     s.host = fresh;
@@ -82,7 +99,13 @@ int upload(const void* src, size_t n, void* dst, cudaStream_t stream, size_t zer
   }
   std::memset(s.host, 0, zeros);
   std::memcpy(static_cast<uint8_t*>(s.host) + zeros, src, n);
-  e = cudaMemcpyAsync(dst, s.host, total, cudaMemcpyHostToDevice, stream);
+  void* src_dev = nullptr;
+  e = cudaHostGetDevicePointer(&src_dev, s.host, 0);
+  if (e != cudaSuccess) return cuda_fail(e);
+  const size_t n16 = total / 16;
+  const int grid = static_cast<int>(std::max<size_t>(1, std::min<size_t>(2 * 148, (n16 + 255) / 256)));
+  upload_kernel<<<grid, 256, 0, stream>>>(static_cast<uint4*>(dst), static_cast<const uint4*>(src_dev), n16, total);
+  e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e);
   e = cudaEventRecord(s.done, stream);
   if (e != cudaSuccess) return cuda_fail(e);
