@@ -98,6 +98,39 @@ def test_tiny_4k_forward_and_backward():
     _case(prob)
 
 
+def test_plan_buffer_is_free_once_the_call_returns():
+    """The forward and the backward take the plan's device section through the
+    library's own staging slot (copied there during the call, read by the upload
+    kernel when the stream reaches it), so the caller may overwrite its plan
+    buffer as soon as a call returns, before the GPU has run that call."""
+    prob = synth.make_problem(synth.WORKLOADS["tiny_4k"], seed=0)
+    q, k, v, do = synth.make_tensors(prob, seed=0, backward=True)
+    qd, kd, vd, dod = _dev(q, k, v, do)
+    plan = skv.skv_plan(prob, skv.SKV_PLAN_LPT)
+    orig = plan.buf.copy()
+    ws = skv.alloc_workspace(plan)
+    Nq, Hq, d = prob.num_tokens_q, prob.num_q_heads, prob.head_dim
+    o = torch.empty(Nq, Hq, d, dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty(Nq, Hq, dtype=torch.float32, device="cuda")
+    dq, dk, dv = torch.empty_like(qd), torch.empty_like(kd), torch.empty_like(vd)
+    stream = torch.cuda.current_stream()
+    torch.cuda.synchronize()
+    torch.cuda._sleep(20_000_000)  # about 10 ms: the call is enqueued long before the stream reaches it
+    skv.skv_attn_fwd(plan, qd, kd, vd, ws, stream)
+    plan.buf[:] = 0xA5
+    torch.cuda.synchronize()
+    plan.buf[:] = orig
+    skv.skv_lse_merge(plan, ws, o, lse, stream)
+    torch.cuda._sleep(20_000_000)
+    skv.skv_attn_bwd(plan, qd, kd, vd, o, lse, dod, dq, dk, dv, ws, stream)
+    plan.buf[:] = 0x5A
+    torch.cuda.synchronize()
+    plan.buf[:] = orig
+    assert skv.skv_status(ws) == 0
+    check_forward(prob, q, k, v, o.cpu(), lse.cpu())
+    check_backward(prob, q, k, v, do, [dq.cpu(), dk.cpu(), dv.cpu()])
+
+
 def test_tiny_4k_static_plan():
     prob = synth.make_problem(synth.WORKLOADS["tiny_4k"], seed=1)
     _case(prob, seed=1, policy=skv.SKV_PLAN_STATIC)
