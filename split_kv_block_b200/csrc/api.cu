@@ -48,9 +48,11 @@ struct Staging {
   bool pending = false;
 };
 constexpr int kSlots = 4;
+constexpr int kMaxDevices = 64;
 std::mutex g_stage_mu;
-Staging g_stage[kSlots];
-int g_stage_next = 0;
+// Slots per device: a slot's event belongs to the device it was created on.
+Staging g_stage[kMaxDevices][kSlots];
+int g_stage_next[kMaxDevices] = {};
 std::vector<void*> g_retired;  // outgrown staging buffers, released with the process
 
 // Copies `total` bytes from mapped host memory `src` to device memory `dst`
@@ -69,10 +71,13 @@ __global__ void __launch_bounds__(256) upload_kernel(uint4* __restrict__ dst, co
 // Copies `zeros` zero bytes followed by the n bytes at src to dst, in one
 // launch of upload_kernel from the staging slot.
 int upload(const void* src, size_t n, void* dst, cudaStream_t stream, size_t zeros = 0) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (dev < 0 || dev >= kMaxDevices) return SKV_EUNSUPPORTED;
   std::lock_guard<std::mutex> lock(g_stage_mu);
-  Staging& s = g_stage[g_stage_next];
-  g_stage_next = (g_stage_next + 1) % kSlots;
-  cudaError_t e;
+  Staging& s = g_stage[dev][g_stage_next[dev]];
+  g_stage_next[dev] = (g_stage_next[dev] + 1) % kSlots;
   if (s.pending) {
     e = cudaEventSynchronize(s.done);
     if (e != cudaSuccess) return cuda_fail(e);
