@@ -36,7 +36,11 @@
  * launch: bad values return SKV_EINVAL, unsupported shapes SKV_EUNSUPPORTED.
  *
  * Memory: the library allocates no device memory. The caller provides the
- * workspace `ws` (device, 256-byte aligned) sized by skv_plan_size().
+ * workspace `ws` (device, 256-byte aligned) sized by skv_plan_size(). For the
+ * plan uploads the library keeps four pinned, mapped host staging slots per
+ * device (grown on demand, released when the process exits); a call copies
+ * the plan's device section into a slot before it returns, and a small kernel
+ * on the call's stream copies the slot into `ws`.
  */
 #ifndef SKV_H_
 #define SKV_H_
