@@ -766,10 +766,25 @@ PlanHeader layout_of(const Prob& q, int policy, const Built& b) {
   return h;
 }
 
-template <class T>
-void copy_to(uint8_t* base, uint64_t off, const std::vector<T>& v) {
-  if (!v.empty()) std::memcpy(base + off, v.data(), v.size() * sizeof(T));
-}
+// Writes a plan front to back: each array at its offset, zeros in the gaps before it. Offsets must come
+// in ascending order (layout_of places the arrays in the order write_plan puts them).
+struct PlanWriter {
+  uint8_t* base;
+  uint64_t cur;
+  void zero_to(uint64_t off) {
+    if (off > cur) std::memset(base + cur, 0, off - cur);
+    cur = std::max(cur, off);
+  }
+  void put(uint64_t off, const void* src, size_t bytes) {
+    zero_to(off);
+    if (bytes) std::memcpy(base + off, src, bytes);
+    cur = std::max(cur, off + bytes);
+  }
+  template <class T>
+  void put(uint64_t off, const std::vector<T>& v) {
+    put(off, v.data(), v.size() * sizeof(T));
+  }
+};
 
 }  // namespace
 
@@ -855,32 +870,34 @@ int write_plan(const skv_problem* prob, int policy, int shard, void* plan, size_
   if (rc != SKV_OK) return rc;
   PlanHeader h = layout_of(q, policy, b);
   if (plan_bytes < h.total_bytes) return SKV_EWORKSPACE;
-  uint8_t* base = static_cast<uint8_t*>(plan);
-  std::memset(base, 0, h.total_bytes);
   h.fingerprint = problem_fingerprint(prob);
-  std::memcpy(base, &h, sizeof(h));
-  copy_to(base, h.items_off, b.items);
-  copy_to(base, h.load_off, b.load);
-  copy_to(base, h.dead_off, b.dead);
-  copy_to(base, h.bwd_part_host_off, b.bwd_part);
-  uint8_t* dev = base + h.dev_off;
-  copy_to(dev, h.dev.mtiles, b.mtiles);
-  copy_to(dev, h.dev.tok_kend, b.tok_kend);
-  copy_to(dev, h.dev.fwd_units, b.fwd);
-  copy_to(dev, h.dev.fwd_part_off, b.fwd_part_off);
-  copy_to(dev, h.dev.fwd_pairs, b.pairs);
-  copy_to(dev, h.dev.fwd_pair_off, b.pair_off);
-  copy_to(dev, h.dev.merge_off, b.merge_off);
-  copy_to(dev, h.dev.merge_list, b.merge_list);
-  copy_to(dev, h.dev.bwd_units, b.bwd);
-  copy_to(dev, h.dev.bwd_part_off, b.bwd_part_off);
-  copy_to(dev, h.dev.dead, b.dead);
-  copy_to(dev, h.dev.tile_mask, b.tile_mask);
-  copy_to(dev, h.dev.pair_tile_off, b.pair_tile_off);
-  copy_to(dev, h.dev.unit_tile_off, b.unit_tile_off);
-  copy_to(dev, h.dev.live_tiles, b.live_tiles);
-  copy_to(dev, h.dev.bwd_rank, b.bwd_rank);
-  copy_to(dev, h.dev.bwd_det_order, b.bwd_det_order);
+  // The arrays in layout order; only the alignment gaps between them are zeroed, so every byte of the
+  // plan is written once and the same problem always gives the same bytes.
+  PlanWriter w{static_cast<uint8_t*>(plan), 0};
+  w.put(0, &h, sizeof(h));
+  w.put(h.items_off, b.items);
+  w.put(h.load_off, b.load);
+  w.put(h.dead_off, b.dead);
+  w.put(h.bwd_part_host_off, b.bwd_part);
+  const uint64_t dev = h.dev_off;
+  w.put(dev + h.dev.mtiles, b.mtiles);
+  w.put(dev + h.dev.tok_kend, b.tok_kend);
+  w.put(dev + h.dev.fwd_units, b.fwd);
+  w.put(dev + h.dev.fwd_part_off, b.fwd_part_off);
+  w.put(dev + h.dev.fwd_pairs, b.pairs);
+  w.put(dev + h.dev.fwd_pair_off, b.pair_off);
+  w.put(dev + h.dev.merge_off, b.merge_off);
+  w.put(dev + h.dev.merge_list, b.merge_list);
+  w.put(dev + h.dev.bwd_units, b.bwd);
+  w.put(dev + h.dev.bwd_part_off, b.bwd_part_off);
+  w.put(dev + h.dev.dead, b.dead);
+  w.put(dev + h.dev.tile_mask, b.tile_mask);
+  w.put(dev + h.dev.pair_tile_off, b.pair_tile_off);
+  w.put(dev + h.dev.unit_tile_off, b.unit_tile_off);
+  w.put(dev + h.dev.live_tiles, b.live_tiles);
+  w.put(dev + h.dev.bwd_rank, b.bwd_rank);
+  w.put(dev + h.dev.bwd_det_order, b.bwd_det_order);
+  w.zero_to(h.total_bytes);
   if (partition_load) std::memcpy(partition_load, b.load.data(), b.load.size() * sizeof(int64_t));
   return SKV_OK;
 }

@@ -191,6 +191,40 @@ def test_plans_do_not_depend_on_earlier_calls():
             assert skv.skv_plan(p, pol).buf.tobytes() == ref[name][pol], (name, pol)
 
 
+def test_plan_bytes_do_not_depend_on_the_buffer_contents():
+    """skv_plan writes every byte of the plan, the alignment gaps between its
+    arrays included: a buffer full of 0xFF and a zeroed one give the same bytes
+    (plain, block-masked, shard and deterministic-backward arrays)."""
+    rng = np.random.default_rng(5)
+    probs = [synth.make_problem(synth.WORKLOADS["ctx32k"], seed=0),
+             synth.make_problem(synth.WORKLOADS["ctx32k_sparse"], seed=0),
+             synth.make_problem(synth.WORKLOADS["batch8_logu"], seed=3),
+             synth.random_small_problem(rng, max_len=900, max_anchors=5, d=64, heads=((4, 1),))]
+    for p in probs:
+        for pol in (skv.SKV_PLAN_LPT, skv.SKV_PLAN_STATIC, skv.SKV_PLAN_LPT | skv.SKV_PLAN_PARTITION_QUEUES):
+            try:
+                sizes = skv.skv_plan_size(p, pol)
+            except skv.SkvError:
+                continue
+            a = np.zeros(sizes.plan_bytes, np.uint8)
+            b = np.full(sizes.plan_bytes, 0xFF, np.uint8)
+            skv.skv_plan(p, pol, sizes=sizes, buf=a)
+            skv.skv_plan(p, pol, sizes=sizes, buf=b)
+            assert a.tobytes() == b.tobytes(), pol
+        for part in range(min(3, p.num_partitions)):
+            sizes = skv.skv_plan_shard_size(p, part)
+            bufs = []
+            for fill in (0x00, 0xFF):
+                buf = np.full(sizes.plan_bytes, fill, np.uint8)
+                loads = np.zeros(p.num_partitions, np.int64)
+                rc = skv.lib().skv_plan_shard(skv._ProblemArgs(p).ref(), skv.SKV_PLAN_LPT, part,
+                                              ctypes.c_void_p(buf.ctypes.data), buf.nbytes,
+                                              ctypes.c_void_p(loads.ctypes.data))
+                assert rc == 0
+                bufs.append(buf.tobytes())
+            assert bufs[0] == bufs[1], part
+
+
 def _fake_dev(n=8):
     """Non-NULL, 256-byte aligned addresses that no call may dereference: every
     call below is refused on the host before it enqueues anything."""
